@@ -1,0 +1,148 @@
+/*
+ * taylor_attn.h -- C ABI of libtaylor_attn.so: causal attention whose
+ * exponential kernel is replaced by its truncated Taylor series, evaluated
+ * through n additive recurrent states, on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Expanding Attention: A Taylor-Series Route to Linear-Time
+ * Transformers with a Fixed Number of Recurrent States" (arXiv 2610.20637),
+ * abstract.  With x = tau * q.k for unit-norm q, k (the caller normalises),
+ *     K(q, k) = sum_{m=0}^{n-1} x^m / m!
+ *             = sum_m (tau^m / m!) <phi_m(q), phi_m(k)>,
+ * where phi_m packs the binom(d_k+m-1, m) monomials x_{i1}...x_{im},
+ * i1 <= ... <= im, each times sqrt(m!/alpha!) (alpha = index multiplicities).
+ * The causal history is the state S = sum_j phi(k_j) [v_j | 1]^T (F rows,
+ * d_v + 1 columns, F = binom(d_k+n-1, n-1)), and
+ *     o_i = y[0:d_v] / y[d_v],   y = (c (.) phi(q_i))^T S_{<=i},
+ * c = tau^m/m! per feature.  Causality is inclusive (token i sees j <= i).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Sizes: 1 <= n <= 5, 1 <= d_k <= 64, 4 <= d_v <= 256 with d_v % 4 == 0,
+ *   B, H, N >= 0 with B*H*N < 2^31 tokens.  Anything else returns
+ *   TAYLOR_ERR_UNSUPPORTED (sizes out of range) or TAYLOR_ERR_INVALID_ARG
+ *   (negative sizes, NULL required pointers, non-finite tau).
+ * - Tensors are dense, row-major, caller-owned DEVICE pointers on the current
+ *   device, aligned to 16 bytes (else TAYLOR_ERR_MISALIGNED):
+ *     q, k  [B][H][N][d_k]   bf16 (the plain calls) or fp32 (the _f32 calls)
+ *     v     [B][H][N][d_v]   same dtype as q, k
+ *     out   [B][H][N][d_v]   fp32
+ *     state [B][H][stride]   fp32, stride = taylor_attn_state_stride(); per
+ *           head: S_v[F][d_v] row-major, then z[F] (the ones column of
+ *           [v | 1]), then zero padding up to stride (a multiple of 32
+ *           floats).  The state holds pure phi(k): it does not depend on tau.
+ *   Feature f follows taylor_attn_feature_index(): degree-major, and inside a
+ *   degree the non-decreasing index tuples in lexicographic order.
+ * - Every call is asynchronous on `stream` (may be 0, the legacy default
+ *   stream) and returns after enqueueing.  Status TAYLOR_OK means the work
+ *   was enqueued; launch failures are reported as TAYLOR_ERR_CUDA.  Calls
+ *   keep no state between them and are safe from several host threads.
+ * - Division is IEEE fp32 (no epsilon): for even n the denominator can reach
+ *   zero for un-normalised inputs and the output is then inf/nan.
+ */
+#ifndef TAYLOR_ATTN_H
+#define TAYLOR_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define TAYLOR_API __attribute__((visibility("default")))
+#else
+#define TAYLOR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum taylor_attn_status {
+    TAYLOR_OK = 0,
+    TAYLOR_ERR_INVALID_ARG = -1,   /* NULL pointer, negative size, bad tau   */
+    TAYLOR_ERR_UNSUPPORTED = -2,   /* n, d_k, d_v or total size out of range  */
+    TAYLOR_ERR_MISALIGNED = -3,    /* a pointer not 16-byte aligned           */
+    TAYLOR_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed    */
+    TAYLOR_ERR_OUT_OF_MEMORY = -5  /* stream-ordered workspace alloc failed   */
+};
+
+/* Short English text for a status code (static storage, never NULL). */
+TAYLOR_API const char* taylor_attn_strerror(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+TAYLOR_API int taylor_attn_version(void);
+
+/* F = sum_{m<n} binom(d_k+m-1, m) = binom(d_k+n-1, n-1), the packed width
+ * of phi (abstract: the m-th state is binom(d+m-1, m) wide).  Returns -1
+ * when (d_k, n) is outside the supported range.  Host only. */
+TAYLOR_API int64_t taylor_attn_num_features(int d_k, int n);
+
+/* Floats per head of a state: F*(d_v+1) rounded up to a multiple of 32.
+ * At d_k = 16, d_v = 64, n = 3: F*(d_v+1) = 9,945 (the abstract's count of
+ * elements per head), stride 9,952.  Returns -1 when unsupported.  Host only. */
+TAYLOR_API int64_t taylor_attn_state_stride(int d_k, int d_v, int n);
+
+/* The packed feature order, written to HOST memory: deg[F] receives the
+ * degree m of each feature, idx[F * max(n-1, 1)] its indices i1 <= ... <= im
+ * followed by -1 padding.  Returns TAYLOR_OK or an error code. */
+TAYLOR_API int taylor_attn_feature_index(int d_k, int n, int32_t* deg, int32_t* idx);
+
+/* Step 1 of the path, exposed on its own (abstract: tensor-power
+ * factorisation).  For T vectors x[T][d_k] (fp32, device) writes
+ * phi[T][F] (fp32, device), phi_f(x) = sqrt(m!/alpha!) prod_t x[i_t]; with
+ * query_side != 0 each feature is also multiplied by tau^m/m!. */
+TAYLOR_API int taylor_attn_feature_map(const float* x, float* phi, int64_t T, int d_k, int n,
+                            float tau, int query_side, cudaStream_t stream);
+
+/* Causal prefill from the empty state (abstract: prefill admits a parallel
+ * scan because states are additive across chunks).  q, k, v are bf16.
+ * Writes out[B][H][N][d_v] and, when state_out != NULL, the state after all
+ * N tokens.  N == 0 writes a zero state.  Takes stream-ordered workspace
+ * with cudaMallocAsync/cudaFreeAsync on `stream` (TAYLOR_ERR_OUT_OF_MEMORY
+ * if that fails); accumulation is fp32. */
+TAYLOR_API int taylor_attn_prefill(const void* q, const void* k, const void* v, float* out,
+                        float* state_out, int B, int H, int N, int d_k, int d_v, int n,
+                        float tau, cudaStream_t stream);
+
+/* Same as taylor_attn_prefill with fp32 q, k, v; every product and sum is
+ * fp32 on CUDA cores (no reduced-precision tensor-core operand). */
+TAYLOR_API int taylor_attn_prefill_f32(const float* q, const float* k, const float* v, float* out,
+                            float* state_out, int B, int H, int N, int d_k, int d_v, int n,
+                            float tau, cudaStream_t stream);
+
+/* One new token per (b, h) against carried states (abstract: per-token
+ * decoding latency is constant in N).  q, k [B][H][d_k] and v [B][H][d_v]
+ * are bf16; state_inout [B][H][stride] is read and overwritten in place with
+ * S + phi(k)[v | 1]^T; out [B][H][d_v] receives the read-out after that
+ * update.  No workspace. */
+TAYLOR_API int taylor_attn_decode(const void* q, const void* k, const void* v, float* state_inout,
+                       float* out, int B, int H, int d_k, int d_v, int n, float tau,
+                       cudaStream_t stream);
+
+/* taylor_attn_decode with fp32 q, k, v. */
+TAYLOR_API int taylor_attn_decode_f32(const float* q, const float* k, const float* v, float* state_inout,
+                           float* out, int B, int H, int d_k, int d_v, int n, float tau,
+                           cudaStream_t stream);
+
+/* out = a + b over B*H states (abstract: states are additive across chunks,
+ * so the state of a concatenation is the sum of the parts' states).  out may
+ * alias a or b.  No workspace. */
+TAYLOR_API int taylor_attn_state_merge(const float* a, const float* b, float* out, int B, int H,
+                            int d_k, int d_v, int n, cudaStream_t stream);
+
+/* Opt-in kernel timing, for benchmarks.  With on != 0, every kernel this
+ * library launches from the calling host thread is bracketed by two CUDA
+ * events on its stream (not usable inside CUDA graph capture). */
+TAYLOR_API int taylor_attn_timing_enable(int on);
+
+/* Waits for the recorded events of the calling thread, clears them, and
+ * writes up to max_kernels entries: names[64 * i] (NUL-terminated kernel
+ * name), launches[i], total_ms[i] (summed device time).  Returns the number
+ * of distinct kernels seen (may exceed max_kernels) or an error code. */
+TAYLOR_API int taylor_attn_timing_read(int max_kernels, char* names, int* launches,
+                                       float* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TAYLOR_ATTN_H */

@@ -211,7 +211,7 @@ def state_of(k: np.ndarray, v: np.ndarray, n: int) -> np.ndarray:
     v = np.asarray(v, dtype=np.float64)
     phik = feature_map(k, n)
     v1 = np.concatenate([v, np.ones(v.shape[:-1] + (1,), dtype=np.float64)], axis=-1)
-    return np.einsum("...jf,...jc->...fc", phik, v1)
+    return np.matmul(np.swapaxes(phik, -1, -2), v1)
 
 
 def state_merge(a: np.ndarray, b: np.ndarray) -> np.ndarray:

@@ -1,0 +1,51 @@
+// Launchers shared between the translation units of libtaylor_attn (not part
+// of the public ABI).  Each returns the CUDA error of its launch(es).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ta {
+
+// Opt-in per-launch event timing (timing.cu).  TA_TIMED brackets one launch.
+namespace timing {
+bool enabled();
+void begin(cudaStream_t s, const char* name);
+void end(cudaStream_t s);
+}  // namespace timing
+
+#define TA_TIMED(stream, name, ...)              \
+    do {                                         \
+        ::ta::timing::begin((stream), (name));   \
+        __VA_ARGS__;                             \
+        ::ta::timing::end((stream));             \
+    } while (0)
+
+template <typename Tin>
+cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state, float* out,
+                          int BH, int d, int dv, int n, float tau, int64_t F, int64_t stride,
+                          cudaStream_t stream);
+
+cudaError_t launch_merge(const float* a, const float* b, float* out, int64_t count, int num_sms,
+                         cudaStream_t stream);
+
+cudaError_t launch_feature_map(const float* x, float* phi, int64_t T, int d, int n, float tau,
+                               int query_side, int64_t F, cudaStream_t stream);
+
+// Chunked prefill on CUDA cores (fp32 arithmetic), in three launches:
+// per-group states, an exclusive scan over groups, then per-chunk outputs.
+struct CcPlan {
+    int G;         // tokens per group (multiple of 64)
+    int NG;        // groups per head
+    size_t ws_bytes;
+};
+CcPlan plan_prefill_cc(int BH, int N, int d, int dv, int n, int64_t F, int64_t stride);
+
+template <typename Tin>
+cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
+                              float* state_out, float* workspace, const CcPlan& plan, int BH,
+                              int N, int d, int dv, int n, float tau, int64_t F, int64_t stride,
+                              cudaStream_t stream);
+
+}  // namespace ta

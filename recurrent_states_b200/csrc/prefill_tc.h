@@ -1,0 +1,26 @@
+// Tensor-core (tcgen05) prefill specialisations.  try_prefill returns
+// kNotApplicable when no specialisation covers the shape, else a
+// taylor_attn status.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ta {
+namespace tc {
+
+constexpr int kNotApplicable = 1;
+
+int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, float* out,
+                float* state_out, int BH, int N, int d, int dv, int n, float tau, int64_t F,
+                int64_t stride, cudaStream_t stream);
+
+// fp32 inputs never take the tensor-core path.
+inline int try_prefill(const float*, const float*, const float*, float*, float*, int, int, int, int,
+                       int, float, int64_t, int64_t, cudaStream_t) {
+    return kNotApplicable;
+}
+
+}  // namespace tc
+}  // namespace ta

@@ -1,0 +1,261 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle, on the
+same seeded inputs.  Outputs: row-scaled max error; states: block-scaled max
+error per (b, h, degree); tolerances 2e-3 (bf16 inputs, fp32 accumulation)
+and 1e-5 (fp32 path).  Integer layout: exact."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import c_oracle as C
+from oracle import taylor_oracle as T
+from recurrent_states_b200 import synth
+from recurrent_states_b200 import taylor_attn as TA
+from tests.gpu_common import TOL, f64, sample_rows, state_block_errors
+from tests.metrics import row_scaled_max_err
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _prefill(dtype, q, k, v, n, tau, state=True):
+    fn = TA.taylor_attn_prefill if dtype == "bf16" else TA.taylor_attn_prefill_f32
+    out, st = fn(q.to(DEV), k.to(DEV), v.to(DEV), n, tau, state_out=True if state else None)
+    torch.cuda.synchronize()
+    return out, st
+
+
+# ------------------------------------------------------------------ feature map
+
+@pytest.mark.parametrize("d,n", [(16, 3), (16, 5), (64, 3), (3, 4), (1, 5), (37, 2)])
+@pytest.mark.parametrize("query", [False, True])
+def test_feature_map_matches_oracle(d, n, query):
+    rng = np.random.default_rng(d * 10 + n)
+    x = rng.standard_normal((77, d)).astype(np.float32)
+    tau = 2.0
+    phi = TA.taylor_attn_feature_map(torch.from_numpy(x).to(DEV), n, tau, query_side=query)
+    ref = T.feature_map(x.astype(np.float64), n)
+    if query:
+        ref = ref * T.query_coeffs(d, n, tau)
+    got = f64(phi)
+    assert got.shape == ref.shape
+    np.testing.assert_allclose(got, ref, rtol=2e-6, atol=1e-6 * np.abs(ref).max())
+
+
+# ------------------------------------------------------------------ prefill, full comparison
+
+CASES = [
+    # (B, H, N, d_k, d_v, n)  several tiles and a ragged tail
+    (1, 1, 256, 16, 16, 3),
+    (2, 3, 1000, 16, 64, 3),
+    (1, 2, 700, 16, 64, 1),
+    (1, 2, 700, 16, 64, 2),
+    (1, 2, 700, 16, 64, 4),
+    (1, 1, 300, 16, 64, 5),
+    (1, 2, 1100, 64, 64, 3),
+    (1, 1, 333, 32, 32, 3),
+    (2, 1, 129, 5, 8, 4),
+    (1, 1, 77, 64, 256, 2),
+]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,H,N,d,dv,n", CASES)
+def test_prefill_matches_oracle(dtype, B, H, N, d, dv, n):
+    tau = 2.0
+    q, k, v = synth.qkv(B, H, N, d, dv, seed=N + n, dtype=dtype)
+    out, st = _prefill(dtype, q, k, v, n, tau)
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    assert row_scaled_max_err(f64(out), ref_out) <= TOL[dtype]
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL[dtype]
+
+
+def test_tiny_config_fp32():
+    """B1 H1 N256 d_k16 d_v16 n3 (F=153), fp32, tau 2, seed 0."""
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w["B"], w["H"], w["N"], w["d_k"], w["d_v"], seed=0, dtype="f32")
+    out, st = _prefill("f32", q, k, v, w["n"], w["tau"])
+    ref_out = T.attention_direct(f64(q), f64(k), f64(v), w["n"], w["tau"])
+    ref_out2, ref_st = T.attention_recurrent(f64(q), f64(k), f64(v), w["n"], w["tau"])
+    assert row_scaled_max_err(f64(out), ref_out) <= TOL["f32"]
+    assert row_scaled_max_err(f64(out), ref_out2) <= TOL["f32"]
+    assert state_block_errors(st, ref_st, 16, 16, 3) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 127, 128, 129, 255, 257])
+def test_prefill_edge_lengths(N):
+    q, k, v = synth.qkv(1, 2, N, 16, 64, seed=N, dtype="bf16")
+    out, st = _prefill("bf16", q, k, v, 3, 2.0)
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), 3, 2.0)
+    assert row_scaled_max_err(f64(out), ref_out) <= TOL["bf16"]
+    assert state_block_errors(st, ref_st, 16, 64, 3) <= TOL["bf16"]
+    # the first token attends only to itself
+    np.testing.assert_allclose(f64(out)[..., 0, :], f64(v)[..., 0, :], rtol=1e-5, atol=1e-6)
+
+
+def test_prefill_empty_inputs():
+    stride = TA.taylor_attn_state_stride(16, 64, 3)
+    e = torch.empty((2, 3, 0, 16), dtype=torch.bfloat16, device=DEV)
+    ev = torch.empty((2, 3, 0, 64), dtype=torch.bfloat16, device=DEV)
+    st = torch.full((2, 3, stride), 7.0, device=DEV)
+    out, st = TA.taylor_attn_prefill(e, e, ev, 3, 2.0, state_out=st)
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and (st == 0).all()
+    e0 = torch.empty((0, 3, 5, 16), dtype=torch.bfloat16, device=DEV)
+    out, _ = TA.taylor_attn_prefill(e0, e0, torch.empty((0, 3, 5, 64), dtype=torch.bfloat16, device=DEV), 3, 2.0)
+    assert out.shape == (0, 3, 5, 64)
+
+
+def test_prefill_is_deterministic():
+    q, k, v = synth.qkv(1, 4, 2000, 16, 64, seed=5)
+    o1, s1 = _prefill("bf16", q, k, v, 3, 2.0)
+    o2, s2 = _prefill("bf16", q, k, v, 3, 2.0)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_state_padding_is_zero():
+    q, k, v = synth.qkv(1, 2, 300, 16, 64, seed=9)
+    _, st = _prefill("bf16", q, k, v, 3, 2.0)
+    F = TA.taylor_attn_num_features(16, 3)
+    assert (st[..., F * 65:] == 0).all()
+
+
+# ------------------------------------------------------------------ the named workloads
+
+def test_main_prefill_full_size():
+    """B1 H8 N4096 d_k16 d_v64 n3, bf16 normalised q, k, tau 2, seed 0: every
+    output and the whole state against the recurrent oracle."""
+    w = synth.WORKLOADS["main_prefill"]
+    q, k, v = synth.qkv(w["B"], w["H"], w["N"], w["d_k"], w["d_v"], seed=0, dtype="bf16")
+    out, st = _prefill("bf16", q, k, v, w["n"], w["tau"])
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), w["n"], w["tau"])
+    assert row_scaled_max_err(f64(out), ref_out) <= TOL["bf16"]
+    assert state_block_errors(st, ref_st, 16, 64, 3) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5])
+def test_order_sweep_full_size(n):
+    """B1 H8 N8192 d_k16 d_v64, n = 1..5, bf16 normalised, tau 2: sampled rows
+    by the pairwise form, and two heads' states by the oracle's sum."""
+    w = synth.WORKLOADS["order_sweep"]
+    q, k, v = synth.qkv(w["B"], w["H"], w["N"], w["d_k"], w["d_v"], seed=0, dtype="bf16")
+    out, st = _prefill("bf16", q, k, v, n, w["tau"])
+    H, N = w["H"], w["N"]
+    qd, kd, vd = f64(q)[0], f64(k)[0], f64(v)[0]
+    rows = sample_rows(N, 96, seed=n)
+    heads = np.repeat(np.arange(H), len(rows))
+    rr = np.tile(rows, H)
+    ref, _ = C.direct_rows(qd, kd, vd, n, w["tau"], heads, rr)
+    got = f64(out)[0][heads, rr]
+    assert row_scaled_max_err(got, ref) <= TOL["bf16"]
+    hs = [0, H - 1]
+    ref_st = C.state(kd[hs], vd[hs], n)
+    assert state_block_errors(st[0, hs], ref_st, 16, 64, n) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("n", [1, 3, 5])
+def test_order_sweep_unnormalised_odd_orders(n):
+    """q, k ~ N(0, 4) without normalisation (the case the pages say diverges
+    from softmax).  For odd n the kernel is positive, so the quotient is well
+    conditioned; sampled rows against the pairwise form."""
+    w = synth.WORKLOADS["order_sweep"]
+    q, k, v = synth.qkv(1, 8, w["N"], 16, 64, seed=1, dtype="bf16", normalise=False, qk_var=4.0)
+    out, _ = _prefill("bf16", q, k, v, n, w["tau"], state=False)
+    rows = sample_rows(w["N"], 48, seed=10 + n)
+    heads = np.repeat(np.arange(8), len(rows))
+    rr = np.tile(rows, 8)
+    ref, _ = C.direct_rows(f64(q)[0], f64(k)[0], f64(v)[0], n, w["tau"], heads, rr)
+    assert row_scaled_max_err(f64(out)[0][heads, rr], ref) <= TOL["bf16"]
+
+
+def test_large_head_full_size():
+    """B4 H16 N32768 d_k64 d_v64 n3 (F=2145), bf16 normalised, tau 2: sampled
+    rows of four heads by the pairwise form; two heads' states."""
+    w = synth.WORKLOADS["large_head"]
+    q, k, v = synth.qkv(w["B"], w["H"], w["N"], w["d_k"], w["d_v"], seed=0, dtype="bf16")
+    out, st = _prefill("bf16", q, k, v, w["n"], w["tau"])
+    N = w["N"]
+    flat = [(0, 0), (1, 5), (2, 10), (3, 15)]
+    qd = np.stack([f64(q[b, h]) for b, h in flat])
+    kd = np.stack([f64(k[b, h]) for b, h in flat])
+    vd = np.stack([f64(v[b, h]) for b, h in flat])
+    rows = sample_rows(N, 40, seed=3)
+    heads = np.repeat(np.arange(len(flat)), len(rows))
+    rr = np.tile(rows, len(flat))
+    ref, _ = C.direct_rows(qd, kd, vd, w["n"], w["tau"], heads, rr)
+    outc = out.cpu()
+    got = np.stack([f64(outc[flat[h][0], flat[h][1], r]) for h, r in zip(heads, rr)])
+    assert row_scaled_max_err(got, ref) <= TOL["bf16"]
+    ref_st = C.state(kd[[0, 3]], vd[[0, 3]], w["n"])
+    got_st = torch.stack([st[0, 0], st[3, 15]])
+    assert state_block_errors(got_st, ref_st, 64, 64, 3) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------------ decode and merge
+
+def _prefix_states(B, H, d, dv, n, prefix, distinct, seed):
+    """Float64 states of `distinct` random prefixes (oracle), assigned to the
+    (b, h) heads round-robin; returned in the library layout, fp32."""
+    q, k, v = synth.qkv(1, distinct, prefix, d, dv, seed=seed, dtype="bf16")
+    ref = C.state(f64(k)[0], f64(v)[0], n)                      # [distinct, F, dv+1]
+    idx = np.arange(B * H) % distinct
+    logical = ref[idx].reshape(B, H, ref.shape[-2], ref.shape[-1])
+    return TA.state_flat(torch.from_numpy(logical), d, dv, n)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_config_steps(dtype):
+    """B64 H16 d_k16 d_v64 n3 from states of 65,536-token random prefixes
+    (16 distinct prefixes, oracle-built); 16 decode steps against the oracle's
+    step from the same fp32 state."""
+    w = synth.WORKLOADS["decode"]
+    B, H, d, dv, n, tau = w["B"], w["H"], w["d_k"], w["d_v"], w["n"], w["tau"]
+    st0 = _prefix_states(B, H, d, dv, n, w["prefix"], 16, seed=0)
+    st = st0.to(DEV)
+    ref_S = f64(TA.state_logical(st0, d, dv, n))
+    fn = TA.taylor_attn_decode if dtype == "bf16" else TA.taylor_attn_decode_f32
+    for step in range(16):
+        qs, ks, vs = synth.decode_tokens(B, H, d, dv, step, dtype=dtype)
+        out = fn(qs.to(DEV), ks.to(DEV), vs.to(DEV), st, n, tau)
+        ref_o, ref_S = T.decode_step(f64(qs), f64(ks), f64(vs), ref_S, n, tau)
+        assert row_scaled_max_err(f64(out), ref_o) <= TOL[dtype], step
+    assert state_block_errors(st, ref_S, d, dv, n) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("d,dv,n", [(16, 16, 3), (16, 64, 5), (64, 64, 3), (7, 12, 2)])
+def test_decode_from_zero_equals_prefill_reference(d, dv, n):
+    N = 150
+    q, k, v = synth.qkv(2, 2, N, d, dv, seed=d + dv + n, dtype="f32")
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, 1.5)
+    st = torch.zeros((2, 2, TA.taylor_attn_state_stride(d, dv, n)), device=DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    outs = []
+    for i in range(N):
+        outs.append(TA.taylor_attn_decode_f32(qd[:, :, i].contiguous(), kd[:, :, i].contiguous(),
+                                              vd[:, :, i].contiguous(), st, n, 1.5))
+    got = torch.stack(outs, dim=2)
+    assert row_scaled_max_err(f64(got), ref_out) <= TOL["f32"]
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL["f32"]
+
+
+def test_merge_and_split_prefill():
+    """state(A) + state(B) from two prefills equals the oracle's state of A+B,
+    and prefill then decode continues the sequence."""
+    d, dv, n = 16, 64, 3
+    q, k, v = synth.qkv(2, 4, 900, d, dv, seed=77)
+    _, sa = _prefill("bf16", q[:, :, :500].contiguous(), k[:, :, :500].contiguous(),
+                     v[:, :, :500].contiguous(), n, 2.0)
+    _, sb = _prefill("bf16", q[:, :, 500:].contiguous(), k[:, :, 500:].contiguous(),
+                     v[:, :, 500:].contiguous(), n, 2.0)
+    merged = TA.taylor_attn_state_merge(sa, sb, d, dv, n)
+    torch.cuda.synchronize()
+    ref_st = C.state(f64(k), f64(v), n)
+    assert state_block_errors(merged, ref_st, d, dv, n) <= TOL["bf16"]
+    # elementwise sum is exact up to one fp32 rounding
+    exact = (sa.double() + sb.double())
+    assert ((merged.double() - exact).abs() <= exact.abs() * 2 ** -24 + 1e-30).all()
+    # in-place (aliased) merge
+    sa2 = sa.clone()
+    TA.taylor_attn_state_merge(sa2, sb, d, dv, n, out=sa2)
+    torch.cuda.synchronize()
+    assert torch.equal(sa2, merged)
