@@ -62,7 +62,8 @@ enum taylor_attn_status {
     TAYLOR_ERR_UNSUPPORTED = -2,   /* n, d_k, d_v or total size out of range  */
     TAYLOR_ERR_MISALIGNED = -3,    /* a pointer not 16-byte aligned           */
     TAYLOR_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed    */
-    TAYLOR_ERR_OUT_OF_MEMORY = -5  /* stream-ordered workspace alloc failed   */
+    TAYLOR_ERR_OUT_OF_MEMORY = -5, /* stream-ordered workspace alloc failed   */
+    TAYLOR_ERR_SCRATCH_LIMIT = -6  /* work exceeds the fixed no-alloc scratch */
 };
 
 /* Short English text for a status code (static storage, never NULL). */
@@ -128,6 +129,28 @@ TAYLOR_API int taylor_attn_decode_f32(const float* q, const float* k, const floa
  * alias a or b.  No workspace. */
 TAYLOR_API int taylor_attn_state_merge(const float* a, const float* b, float* out, int B, int H,
                             int d_k, int d_v, int n, cudaStream_t stream);
+
+/* taylor_attn_prefill_f32 for callers that cannot allocate device memory
+ * (a plugin whose host framework owns all device memory, a serving loop that
+ * reserves memory up front and must not see an allocation fail mid-step).
+ * The paper has no counterpart: this is a deployment variant.  The scratch
+ * for the scan across token groups lives in one fixed file-scope device array
+ * of taylor_attn_prefill_noalloc_scratch_floats() floats (16 MiB), held on
+ * every GPU that loads the library until the process exits; the call makes no
+ * cudaMalloc/cudaFree or other allocating call.  Work needing more scratch
+ * than that (B*H * groups * stride floats; the B1 H8 N4096 d_k16 d_v64 n3
+ * shape needs about 2.5 million) returns TAYLOR_ERR_SCRATCH_LIMIT before any launch.
+ * The first call on a device looks up the array's device address (make it
+ * before any stream capture).  All calls on a device share the array: calls
+ * that overlap on the GPU race and must be serialised by the caller.  Same
+ * arguments, layouts and results as taylor_attn_prefill_f32. */
+TAYLOR_API int taylor_attn_prefill_f32_noalloc(const float* q, const float* k, const float* v,
+                                               float* out, float* state_out, int B, int H, int N,
+                                               int d_k, int d_v, int n, float tau,
+                                               cudaStream_t stream);
+
+/* Size in floats of the fixed scratch used by taylor_attn_prefill_f32_noalloc. */
+TAYLOR_API int64_t taylor_attn_prefill_noalloc_scratch_floats(void);
 
 /* Opt-in kernel timing, for benchmarks.  With on != 0, every kernel this
  * library launches from the calling host thread is bracketed by two CUDA

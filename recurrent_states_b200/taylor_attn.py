@@ -23,6 +23,7 @@ TAYLOR_ERR_UNSUPPORTED = -2
 TAYLOR_ERR_MISALIGNED = -3
 TAYLOR_ERR_CUDA = -4
 TAYLOR_ERR_OUT_OF_MEMORY = -5
+TAYLOR_ERR_SCRATCH_LIMIT = -6
 
 # name -> (restype, argtypes); the exported surface of the header
 _P = ctypes.c_void_p
@@ -41,6 +42,8 @@ SIGNATURES = {
     "taylor_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_decode_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_state_merge": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "taylor_attn_prefill_f32_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "taylor_attn_prefill_noalloc_scratch_floats": (_I64, []),
     "taylor_attn_timing_enable": (_I, [_I]),
     "taylor_attn_timing_read": (_I, [_I, _P, _P, _P]),
 }
@@ -185,6 +188,18 @@ def taylor_attn_prefill(q, k, v, n: int, tau: float, out=None, state_out=None, s
 def taylor_attn_prefill_f32(q, k, v, n: int, tau: float, out=None, state_out=None, stream=None):
     """taylor_attn_prefill with fp32 q, k, v."""
     return _prefill("taylor_attn_prefill_f32", q, k, v, n, tau, out, state_out, stream)
+
+
+def taylor_attn_prefill_f32_noalloc(q, k, v, n: int, tau: float, out=None, state_out=None, stream=None):
+    """taylor_attn_prefill_f32 without any device allocation inside the call:
+    its scratch is a fixed array in the library (see the header).  The caller
+    passes every input and output; outputs are created here only when not
+    given."""
+    return _prefill("taylor_attn_prefill_f32_noalloc", q, k, v, n, tau, out, state_out, stream)
+
+
+def taylor_attn_prefill_noalloc_scratch_floats() -> int:
+    return int(lib().taylor_attn_prefill_noalloc_scratch_floats())
 
 
 def _decode(name, q, k, v, state, n, tau, out, stream):
