@@ -63,7 +63,8 @@ enum taylor_attn_status {
     TAYLOR_ERR_MISALIGNED = -3,    /* a pointer not 16-byte aligned           */
     TAYLOR_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed    */
     TAYLOR_ERR_OUT_OF_MEMORY = -5, /* stream-ordered workspace alloc failed   */
-    TAYLOR_ERR_SCRATCH_LIMIT = -6  /* work exceeds the fixed no-alloc scratch */
+    TAYLOR_ERR_SCRATCH_LIMIT = -6, /* work exceeds the fixed no-alloc scratch */
+    TAYLOR_ERR_TIMEOUT = -7        /* a bounded device-side wait ran out      */
 };
 
 /* Short English text for a status code (static storage, never NULL). */
@@ -151,6 +152,15 @@ TAYLOR_API int taylor_attn_prefill_f32_noalloc(const float* q, const float* k, c
 
 /* Size in floats of the fixed scratch used by taylor_attn_prefill_f32_noalloc. */
 TAYLOR_API int64_t taylor_attn_prefill_noalloc_scratch_floats(void);
+
+/* Kernels that wait on asynchronous copies (mbarriers) bound every wait;
+ * when a bound runs out the kernel sets a bit in a device error word and
+ * returns early (its outputs are then incomplete).  This call reads that word
+ * for the current device (a synchronous device-to-host copy that waits for
+ * all prior work), stores it in *flags, clears it when clear != 0, and
+ * returns TAYLOR_ERR_TIMEOUT if any bit was set, else TAYLOR_OK.
+ * Bits: 1 = decode state load, 2 = decode state store, 4 = prefill pipeline. */
+TAYLOR_API int taylor_attn_device_errors(int clear, unsigned int* flags);
 
 /* Opt-in kernel timing, for benchmarks.  With on != 0, every kernel this
  * library launches from the calling host thread is bracketed by two CUDA

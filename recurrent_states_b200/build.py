@@ -24,7 +24,7 @@ FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC,-fvisibility=hidden",
     "-shared", "-cudart", "static",
-    "--expt-relaxed-constexpr",
+    "--expt-relaxed-constexpr", "--extended-lambda",
     "-I", os.path.join(ROOT, "include"),
 ]
 

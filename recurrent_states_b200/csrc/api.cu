@@ -121,6 +121,7 @@ const char* taylor_attn_strerror(int status) {
         case TAYLOR_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
         case TAYLOR_ERR_OUT_OF_MEMORY: return "stream-ordered workspace allocation failed";
         case TAYLOR_ERR_SCRATCH_LIMIT: return "work needs more than the fixed no-alloc scratch";
+        case TAYLOR_ERR_TIMEOUT: return "a bounded device-side wait ran out (see taylor_attn_device_errors)";
         default: return "unknown status";
     }
 }

@@ -24,9 +24,11 @@ constexpr int kMaxDv = 256;
 
 TA_HD int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 
+// binom(a, b) for the library's range (a <= 68, b <= 4): 32-bit arithmetic
+// suffices (largest intermediate 814385 * 68).
 TA_HD int64_t binom(int a, int b) {
     if (b < 0 || a < 0 || b > a) return 0;
-    int64_t r = 1;
+    int r = 1;
     for (int i = 1; i <= b; ++i) r = r * (a - b + i) / i;
     return r;
 }

@@ -3,80 +3,201 @@
 // y = (c (.) phi(q))^T S and o = y[0:d_v] / y[d_v].
 //
 // The step is bound by HBM: each head's fp32 state (F*(d_v+1) floats) is read
-// once and written once.  One CTA per head; each thread owns one 16-byte
-// column group of the S_v rows it visits, so a warp moves whole 128-byte
-// lines with 128-bit loads and stores.  The state rows of a thread are loaded
-// into registers before the feature map is evaluated, so the loads are in
-// flight while phi(q), phi(k) are computed.  The read-out sum over rows is a
-// shared-memory reduction across row sets; the normaliser's sum over z is a
-// warp-shuffle reduction.
+// once and written once.  One CTA per head.
+//
+// Main path (d_v in {16, 32, 64, 128}, state <= 110 KB): one thread issues a
+// single bulk (TMA) copy of the head's state into shared memory, completing
+// on an mbarrier, while the block evaluates phi(q), phi(k) from the static
+// feature table.  The block then updates the state in shared memory with
+// 128-bit accesses (each thread owns one 16-byte column group of the rows it
+// visits), accumulates the read-out, and one thread streams the state back
+// with a bulk store.  No state element passes through registers for longer
+// than one update, so occupancy is set by shared memory (5 CTAs per SM at
+// d_k 16, d_v 64, n 3) and every CTA's whole state is in flight at once.
+// The read-out sum over rows is a warp-shuffle plus shared-memory reduction.
+//
+// Fallback path (other d_v or larger states): the same arithmetic with
+// register-staged 128-bit loads and stores, one feature tile at a time.
+#include <mutex>
+
 #include "common.cuh"
+#include "feature_table.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace ta {
 
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr uint32_t kWaitPolls = 1u << 22;  // bound on mbarrier polls (seconds of wall time)
+constexpr int kTmaMaxBytes = 110 * 1024;
+
+template <typename Tin, int DV4>
+__global__ void __launch_bounds__(kThreads, 5)
+decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                  float* __restrict__ state, float* __restrict__ out, int d, int n, float tau, int F,
+                  int64_t stride, uint32_t bytes, unsigned int* __restrict__ err) {
+    constexpr int DV = DV4 * 4;
+    constexpr int RS = kThreads / DV4;  // row sets
+    extern __shared__ __align__(128) unsigned char dsm[];
+    __shared__ float xq[kMaxDk], xk[kMaxDk], vv[DV], qc[kMaxN];
+    __shared__ float4 red[kWarps][DV4];
+    __shared__ float zr[kWarps];
+    __shared__ __align__(8) uint64_t bar;
+
+    float* S = reinterpret_cast<float*>(dsm);
+    const uint32_t soff = (bytes + 127u) & ~127u;
+    float* pk = reinterpret_cast<float*>(dsm + soff);
+    float* pq = pk + ((F + 3) & ~3);
+
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x;
+    float* gS = state + (int64_t)bh * stride;
+
+    if (tid == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        ptx::mbar_arrive_expect_tx(&bar, bytes);
+        ptx::bulk_g2s(S, gS, bytes, &bar);
+    }
+    // while the state streams in: the new token and the feature map
+    if (tid < d) {
+        xq[tid] = ldf(q + (int64_t)bh * d + tid);
+        xk[tid] = ldf(k + (int64_t)bh * d + tid);
+    }
+    if (tid < DV) vv[tid] = ldf(v + (int64_t)bh * DV + tid);
+    if (tid < n) qc[tid] = query_coeff(tid, tau);
+    __syncthreads();
+    const PackedFeat* tab = feat_table(d, n);
+    for (int f = tid; f < F; f += kThreads) {
+        pk[f] = eval_desc(get_desc(tab, d, n, f, tau, qc, false), xk);
+        pq[f] = eval_desc(get_desc(tab, d, n, f, tau, qc, true), xq);
+    }
+    // every thread observes the copy's completion itself; the block agrees
+    // on the outcome so that a timeout leaves as one
+    const bool landed = ptx::mbar_wait(&bar, 0, kWaitPolls);
+    if (!__syncthreads_and(landed)) {
+        if (tid == 0) atomicOr(err, kErrDecodeLoad);
+        if (!landed) ptx::mbar_wait(&bar, 0, kWaitPolls);  // one more bound for the copy in flight
+        return;
+    }
+
+    const int cg = tid % DV4, rs = tid / DV4;
+    const float4 v4 = reinterpret_cast<const float4*>(vv)[cg];
+    float4* S4 = reinterpret_cast<float4*>(S);
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int r = rs; r < F; r += RS) {
+        const float a = pk[r], b = pq[r];
+        float4 s = S4[r * DV4 + cg];
+        s.x = fmaf(a, v4.x, s.x);
+        s.y = fmaf(a, v4.y, s.y);
+        s.z = fmaf(a, v4.z, s.z);
+        s.w = fmaf(a, v4.w, s.w);
+        S4[r * DV4 + cg] = s;
+        y.x = fmaf(b, s.x, y.x);
+        y.y = fmaf(b, s.y, y.y);
+        y.z = fmaf(b, s.z, y.z);
+        y.w = fmaf(b, s.w, y.w);
+    }
+    float yz = 0.f;
+    float* Z = S + F * DV;
+    for (int f = tid; f < F; f += kThreads) {
+        const float z = Z[f] + pk[f];
+        Z[f] = z;
+        yz = fmaf(pq[f], z, yz);
+    }
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        ptx::bulk_s2g(gS, S, bytes);
+        ptx::bulk_commit();
+    }
+
+    // read-out: lanes sharing a column group sit DV4 apart inside a warp
+#pragma unroll
+    for (int o = DV4; o < 32; o <<= 1) {
+        y.x += __shfl_xor_sync(0xffffffffu, y.x, o);
+        y.y += __shfl_xor_sync(0xffffffffu, y.y, o);
+        y.z += __shfl_xor_sync(0xffffffffu, y.z, o);
+        y.w += __shfl_xor_sync(0xffffffffu, y.w, o);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) yz += __shfl_xor_sync(0xffffffffu, yz, o);
+    const int warp = tid >> 5, lane = tid & 31;
+    if (lane < DV4) red[warp][lane] = y;
+    if (lane == 0) zr[warp] = yz;
+    __syncthreads();
+    if (tid < DV) {
+        const int g = tid >> 2, c = tid & 3;
+        float acc = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float4 t = red[w][g];
+            acc += c == 0 ? t.x : c == 1 ? t.y : c == 2 ? t.z : t.w;
+            den += zr[w];
+        }
+        out[(int64_t)bh * DV + tid] = acc / den;
+    }
+    if (tid == 0) ptx::bulk_wait_read_all();
+}
+
 constexpr int kFeatTile = 1024;  // features whose phi(q), phi(k) sit in smem at once
 constexpr int kRows = 10;        // S_v rows per thread held in registers per batch
 
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads)
-decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-              float* __restrict__ state, float* __restrict__ out, int d, int dv, int n,
-              float tau, int F, int64_t stride) {
-    __shared__ float xs_q[kMaxDk], xs_k[kMaxDk], vs[kMaxDv];
+decode_generic_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                      float* __restrict__ state, float* __restrict__ out, int d, int dv, int n,
+                      float tau, int F, int64_t stride) {
+    __shared__ float xs_q[kMaxDk], xs_k[kMaxDk], vs[kMaxDv], qc[kMaxN];
     __shared__ float pk[kFeatTile], pq[kFeatTile];
     __shared__ float4 red[kThreads];
-    __shared__ float zred[kThreads / 32];
+    __shared__ float zred[kWarps];
 
     const int bh = blockIdx.x;
     const int tid = threadIdx.x;
     const int dv4 = dv >> 2;
-    const int rsets = kThreads / dv4;      // row sets (threads sharing a column group)
+    const int rsets = kThreads / dv4;
     const int cg = tid % dv4;
     const int rs = tid / dv4;
     const bool active = rs < rsets;
 
     float* Sv = state + (int64_t)bh * stride;
     float* Z = Sv + (int64_t)F * dv;
+    const PackedFeat* tab = feat_table(d, n);
 
     for (int i = tid; i < d; i += kThreads) {
         xs_q[i] = ldf(q + (int64_t)bh * d + i);
         xs_k[i] = ldf(k + (int64_t)bh * d + i);
     }
     for (int i = tid; i < dv; i += kThreads) vs[i] = ldf(v + (int64_t)bh * dv + i);
+    if (tid < n) qc[tid] = query_coeff(tid, tau);
 
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
     float yz = 0.f;
 
     for (int fb = 0; fb < F; fb += kFeatTile) {
         const int fe = min(F, fb + kFeatTile);
-        // first batch of rows: issue the loads before the feature map
-        float4 s[kRows];
-        float zz[kFeatTile / kThreads];
-        int r0 = fb + rs;
-#pragma unroll
-        for (int i = 0; i < kRows; ++i) {
-            const int r = r0 + i * rsets;
-            if (active && r < fe) s[i] = *reinterpret_cast<const float4*>(Sv + (int64_t)r * dv + cg * 4);
-        }
-#pragma unroll
-        for (int i = 0; i < kFeatTile / kThreads; ++i) {
-            const int f = fb + tid + i * kThreads;
-            if (f < fe) zz[i] = Z[f];
-        }
-        __syncthreads();  // xs_q, xs_k, vs ready; previous tile's pk/pq consumed
+        __syncthreads();  // inputs ready; previous tile's pk/pq consumed
         for (int f = fb + tid; f < fe; f += kThreads) {
-            const FeatDesc dk = make_desc(d, n, f, tau, false);
-            const FeatDesc dq = make_desc(d, n, f, tau, true);
-            pk[f - fb] = eval_desc(dk, xs_k);
-            pq[f - fb] = eval_desc(dq, xs_q);
+            pk[f - fb] = eval_desc(get_desc(tab, d, n, f, tau, qc, false), xs_k);
+            pq[f - fb] = eval_desc(get_desc(tab, d, n, f, tau, qc, true), xs_q);
         }
         __syncthreads();
         const float4 v4 = active ? *reinterpret_cast<const float4*>(vs + cg * 4) : make_float4(0, 0, 0, 0);
-        for (;;) {
+        for (int r0 = fb + rs; r0 < fe; r0 += kRows * rsets) {
+            float4 s[kRows];
+#pragma unroll
+            for (int i = 0; i < kRows; ++i) {
+                const int r = r0 + i * rsets;
+                if (active && r < fe) s[i] = *reinterpret_cast<const float4*>(Sv + (int64_t)r * dv + cg * 4);
+            }
 #pragma unroll
             for (int i = 0; i < kRows; ++i) {
                 const int r = r0 + i * rsets;
@@ -94,26 +215,14 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
                     y.w = fmaf(b, t.w, y.w);
                 }
             }
-            r0 += kRows * rsets;
-            if (r0 >= fe) break;
-#pragma unroll
-            for (int i = 0; i < kRows; ++i) {
-                const int r = r0 + i * rsets;
-                if (active && r < fe) s[i] = *reinterpret_cast<const float4*>(Sv + (int64_t)r * dv + cg * 4);
-            }
         }
-#pragma unroll
-        for (int i = 0; i < kFeatTile / kThreads; ++i) {
-            const int f = fb + tid + i * kThreads;
-            if (f < fe) {
-                const float z = zz[i] + pk[f - fb];
-                Z[f] = z;
-                yz = fmaf(pq[f - fb], z, yz);
-            }
+        for (int f = fb + tid; f < fe; f += kThreads) {
+            const float z = Z[f] + pk[f - fb];
+            Z[f] = z;
+            yz = fmaf(pq[f - fb], z, yz);
         }
     }
 
-    // reduce y over row sets, yz over the block
     red[tid] = y;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) yz += __shfl_xor_sync(0xffffffffu, yz, o);
@@ -128,28 +237,65 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
         }
         float den = 0.f;
 #pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) den += zred[w];
+        for (int w = 0; w < kWarps; ++w) den += zred[w];
         out[(int64_t)bh * dv + tid] = acc / den;
     }
+}
+
+constexpr int kMaxDevices = 64;
+
+template <typename Tin, int DV4>
+cudaError_t launch_tma(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
+                       int n, float tau, int F, int64_t stride, uint32_t bytes, size_t dyn,
+                       unsigned int* err, cudaStream_t stream) {
+    auto fn = decode_tma_kernel<Tin, DV4>;
+    if (dyn > 48 * 1024) {
+        static std::once_flag once[kMaxDevices];
+        static cudaError_t set_err[kMaxDevices];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        std::call_once(once[dev], [&]() {
+            set_err[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxBytes + 8192);
+        });
+        if (set_err[dev] != cudaSuccess) return set_err[dev];
+    }
+    TA_TIMED(stream, "decode_tma_kernel",
+             fn<<<BH, kThreads, dyn, stream>>>(q, k, v, state, out, d, n, tau, F, stride, bytes, err));
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 template <typename Tin>
-cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state, float* out,
-                          int BH, int d, int dv, int n, float tau, int64_t F, int64_t stride,
-                          cudaStream_t stream) {
+cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH,
+                          int d, int dv, int n, float tau, int64_t F, int64_t stride, cudaStream_t stream) {
     if (BH == 0) return cudaSuccess;
-    TA_TIMED(stream, "decode_kernel",
-             decode_kernel<Tin><<<BH, kThreads, 0, stream>>>(q, k, v, state, out, d, dv, n, tau, (int)F,
-                                                             stride));
+    const int64_t used_bytes = F * (dv + 1) * 4;
+    const uint32_t bytes = (uint32_t)((used_bytes + 15) / 16 * 16);
+    const size_t dyn = ((bytes + 127u) & ~127u) + 2 * (size_t)((F + 3) & ~3) * 4;
+    unsigned int* err = device_error_word();
+    const bool tma_ok = err != nullptr && used_bytes <= kTmaMaxBytes && dyn <= (size_t)kTmaMaxBytes + 8192;
+    if (tma_ok) {
+        switch (dv) {
+            case 16: return launch_tma<Tin, 4>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn, err, stream);
+            case 32: return launch_tma<Tin, 8>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn, err, stream);
+            case 64: return launch_tma<Tin, 16>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn, err, stream);
+            case 128: return launch_tma<Tin, 32>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn, err, stream);
+            default: break;
+        }
+    }
+    TA_TIMED(stream, "decode_generic_kernel",
+             decode_generic_kernel<Tin><<<BH, kThreads, 0, stream>>>(q, k, v, state, out, d, dv, n, tau,
+                                                                     (int)F, stride));
     return cudaGetLastError();
 }
 
-template cudaError_t launch_decode<float>(const float*, const float*, const float*, float*, float*,
-                                          int, int, int, int, float, int64_t, int64_t, cudaStream_t);
+template cudaError_t launch_decode<float>(const float*, const float*, const float*, float*, float*, int, int,
+                                          int, int, float, int64_t, int64_t, cudaStream_t);
 template cudaError_t launch_decode<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
-                                                  const __nv_bfloat16*, float*, float*, int, int, int,
-                                                  int, float, int64_t, int64_t, cudaStream_t);
+                                                  const __nv_bfloat16*, float*, float*, int, int, int, int,
+                                                  float, int64_t, int64_t, cudaStream_t);
 
 }  // namespace ta

@@ -5,6 +5,7 @@
 // be checked on the device.  One CTA per 32 vectors; each thread owns one
 // feature column and unranks it once.
 #include "common.cuh"
+#include "feature_table.cuh"
 #include "internal.h"
 
 namespace ta {
@@ -17,13 +18,16 @@ __global__ void __launch_bounds__(256)
 feature_map_kernel(const float* __restrict__ x, float* __restrict__ phi, int64_t T, int d, int n,
                    float tau, int query_side, int64_t F) {
     __shared__ float xs[kVec][kMaxDk];
+    __shared__ float qc[kMaxN];
+    if (threadIdx.x < n) qc[threadIdx.x] = query_coeff(threadIdx.x, tau);
+    const PackedFeat* tab = feat_table(d, n);
     const int64_t t0 = (int64_t)blockIdx.x * kVec;
     const int nv = (int)min64(kVec, T - t0);
     for (int i = threadIdx.x; i < nv * d; i += blockDim.x) xs[i / d][i % d] = x[t0 * d + i];
     __syncthreads();
     for (int64_t f = threadIdx.x + (int64_t)blockIdx.y * blockDim.x; f < F;
          f += (int64_t)gridDim.y * blockDim.x) {
-        const FeatDesc fd = make_desc(d, n, f, tau, query_side != 0);
+        const FeatDesc fd = get_desc(tab, d, n, f, tau, qc, query_side != 0);
         for (int i = 0; i < nv; ++i) phi[(t0 + i) * F + f] = eval_desc(fd, xs[i]);
     }
 }

@@ -22,6 +22,12 @@ void end(cudaStream_t s);
         ::ta::timing::end((stream));             \
     } while (0)
 
+// Device address of the error word (errors.cu) on the current device.
+unsigned int* device_error_word();
+constexpr unsigned int kErrDecodeLoad = 1u;
+constexpr unsigned int kErrDecodeStore = 2u;
+constexpr unsigned int kErrPrefillPipe = 4u;
+
 template <typename Tin>
 cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state, float* out,
                           int BH, int d, int dv, int n, float tau, int64_t F, int64_t stride,
@@ -41,6 +47,11 @@ struct CcPlan {
     size_t ws_bytes;
 };
 CcPlan plan_prefill_cc(int BH, int N, int d, int dv, int n, int64_t F, int64_t stride);
+
+// In place: W[bh][g] <- sum_{g' < g} W[bh][g'] over the first `used` floats
+// of each state; state_out[bh] (if not NULL) <- the total, zero padded.
+cudaError_t launch_state_scan(float* W, float* state_out, int BH, int NG, int64_t stride, int64_t used,
+                              cudaStream_t stream);
 
 template <typename Tin>
 cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,

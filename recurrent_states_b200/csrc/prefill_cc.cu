@@ -15,6 +15,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "feature_table.cuh"
 #include "internal.h"
 
 namespace ta {
@@ -47,7 +48,7 @@ group_state_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, float* 
     const bool active = rs < rsets;
     const int dpad = (d + 3) & ~3;
 
-    if (tid < nf) ds[tid] = make_desc(d, n, f0 + tid, 0.f, false);
+    if (tid < nf) ds[tid] = get_desc(feat_table(d, n), d, n, f0 + tid, 0.f, nullptr, false);
 
     float4 acc[RPT];
 #pragma unroll
@@ -185,6 +186,9 @@ chunk_out_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     const Tin* qb = q + (int64_t)bh * N * d;
     const Tin* kb = k + (int64_t)bh * N * d;
     const Tin* vb = v + (int64_t)bh * N * dv;
+    const PackedFeat* tab = feat_table(d, n);
+    __shared__ float qc[kMaxN];
+    if (tid < n) qc[tid] = query_coeff(tid, tau);
     for (int e = tid; e < kC * d; e += kThreads) {
         const int r = e / d, s = e % d;
         qs[r * dq + s] = r < nq ? ldf(qb + (q0 + r) * d + s) : 0.f;
@@ -236,7 +240,7 @@ chunk_out_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             for (int f0 = 0; f0 < F; f0 += kFTC) {
                 const int nf = min(kFTC, F - f0);
                 __syncthreads();
-                if (tid < nf) ds[tid] = make_desc(d, n, f0 + tid, tau, true);
+                if (tid < nf) ds[tid] = get_desc(tab, d, n, f0 + tid, tau, qc, true);
                 for (int e = tid; e < nf * cw; e += kThreads) {
                     const int r = e / cw, c = e % cw;
                     Ss[r * 64 + c] = Sg[(int64_t)(f0 + r) * dv + cb + c];
@@ -342,6 +346,13 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
     TA_TIMED(stream, "cc_chunk_out_kernel",
              fc<<<gC, kThreads, L.total, stream>>>(q, k, v, W, out, N, d, dv, n, tau, plan.G, plan.NG,
                                                    (int)F, stride));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_scan(float* W, float* state_out, int BH, int NG, int64_t stride, int64_t used,
+                              cudaStream_t stream) {
+    const dim3 g((unsigned)((stride + kThreads - 1) / kThreads), BH);
+    TA_TIMED(stream, "scan_kernel", scan_kernel<<<g, kThreads, 0, stream>>>(W, state_out, NG, stride, used));
     return cudaGetLastError();
 }
 

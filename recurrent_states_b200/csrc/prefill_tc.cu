@@ -1,12 +1,509 @@
-// Tensor-core prefill specialisations (tcgen05, sm_100a).
+// Chunked causal prefill on the sm_100a tensor cores (tcgen05, TMEM), for
+// d_k = 16, n <= 3 (F <= 153, padded to 160) and d_v = 64 with bf16 inputs.
+//
+// Method (arXiv 2610.20637, abstract): the kernel is an inner product of
+// packed tensor powers, so the causal history is the state
+// S = sum_j phi(k_j) [v_j | 1]^T, and states are additive across chunks, so
+// prefill is a scan.  With chunks of C = 128 tokens:
+//   1. tc_chunk_state:  dS_c = Phi_K,c^T [V_c | 1]           (tensor cores)
+//   2. scan:            S_<c = sum_{c' < c} dS_c', final state  (CUDA cores)
+//   3. tc_chunk_out:    Y_c = (poly(tau Q_c K_c^T) (.) causal mask) [V_c | 1]
+//                             + (c (.) Phi_Q,c) S_<c,   o = Y[:, :64] / Y[:, 64]
+// Every contraction runs as tcgen05.mma (bf16 operands in shared memory, fp32
+// accumulators in TMEM).  bf16 holds 8 significant bits, which alone would
+// cost ~4e-3 in the outputs; each operand produced in fp32 (Phi_Q, Phi_K, the
+// pairwise weights P and the carried state S) is therefore split into
+// hi = bf16(x) and lo = bf16(x - hi) and contracted as hi*hi' + hi*lo' +
+// lo*hi' (or hi*B + lo*B when B is an exact bf16 input), which keeps about 16
+// significant bits with fp32 accumulation and bf16's full exponent range.
+// The normaliser rides along as column 64 of [V | 1 | 0...] (N = 80), so the
+// denominator comes out of the same MMAs as the numerator.
+//
+// The feature map for d_k = 16 is evaluated in closed form with compile-time
+// indices: phi = [1, x_i, w_ab x_a x_b (a <= b)], w = sqrt(2) for a < b, 1 for
+// a = b, times tau^m/m! on the query side; degrees >= n are zeroed.
+#include <mutex>
+
+#include "../../include/taylor_attn.h"
+#include "common.cuh"
+#include "feature_table.cuh"
+#include "internal.h"
 #include "prefill_tc.h"
+#include "ptx.cuh"
+#include "tcgen05.cuh"
 
 namespace ta {
 namespace tc {
 
-int try_prefill(const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, float*, float*, int,
-                int, int, int, int, float, int64_t, int64_t, cudaStream_t) {
-    return kNotApplicable;
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kC = 128;       // tokens per chunk (MMA M)
+constexpr int kD = 16;        // d_k
+constexpr int kDV = 64;       // d_v
+constexpr int kNV = 80;       // columns of [V | 1 | 0 ...]  (MMA N)
+constexpr int kFP = 160;      // features padded to a multiple of 16
+constexpr int kThreads = 256;
+constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr float kSqrt2 = (float)cx_sqrt(2.0);
+
+// Shared-memory layouts (bytes).  K-major operands use LBO = 128; MN-major
+// operands use SBO = 128 (see tcgen05.cuh).
+constexpr uint32_t kSboQK = 2 * 128;                 // Q, K: [128][16] K-major
+constexpr uint32_t kLboV1 = (kNV / 8) * 128;         // [V|1]: [K=128 keys][80] MN-major
+constexpr uint32_t kSboP = (kC / 8) * 128;           // P: [128][128] K-major
+constexpr uint32_t kSboPhiQ = (kFP / 8) * 128;       // Phi_Q: [128][160] K-major
+constexpr uint32_t kLboS = (kNV / 8) * 128;          // S: [K=160][80] MN-major
+constexpr uint32_t kLboPhiK = (256 / 8) * 128;       // Phi_K^T: [K=128 tokens][256] MN-major
+
+// chunk_out
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kC * kD * 2;
+constexpr uint32_t kOffV1 = kOffK + kC * kD * 2;
+constexpr uint32_t kOffPh = kOffV1 + kC * kNV * 2;
+constexpr uint32_t kOffPl = kOffPh + kC * kC * 2;
+constexpr uint32_t kOffQh = kOffPl + kC * kC * 2;
+constexpr uint32_t kOffQl = kOffQh + kC * kFP * 2;
+constexpr uint32_t kOffSh = kOffQl + kC * kFP * 2;
+constexpr uint32_t kOffSl = kOffSh + kFP * kNV * 2;
+constexpr uint32_t kSmemOut = kOffSl + kFP * kNV * 2;   // 227,328 bytes
+// chunk_state
+constexpr uint32_t kOffV1s = 0;
+constexpr uint32_t kOffAh = kOffV1s + kC * kNV * 2;
+constexpr uint32_t kOffAl = kOffAh + 256 * kC * 2;
+constexpr uint32_t kSmemState = kOffAl + 256 * kC * 2;  // 151,552 bytes
+
+static_assert(kSmemOut <= 232448 - 256, "chunk_out shared memory");
+
+__device__ __forceinline__ uint32_t kmaj(int r, int kgroup, uint32_t sbo) {
+    return (uint32_t)(r >> 3) * sbo + (uint32_t)kgroup * 128u + (uint32_t)(r & 7) * 16u;
+}
+__device__ __forceinline__ uint32_t mnmaj(int k, int ngroup, uint32_t lbo) {
+    return (uint32_t)ngroup * 128u + (uint32_t)(k >> 3) * lbo + (uint32_t)(k & 7) * 16u;
+}
+
+__device__ __forceinline__ void ld_row16(const bf16* p, float (&x)[16]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// Writes the 160 padded features of one token, scaled per degree by
+// (e0, e1, e2), as hi/lo bf16 groups of 8 through `put(group, hi, lo)`.
+template <typename Put>
+__device__ __forceinline__ void phi16_groups(const float (&x)[16], float e0, float e1, float e2, Put put) {
+    float buf[8];
+    int f = 0;
+    auto emit = [&](float val) {
+        buf[f & 7] = val;
+        ++f;
+        if ((f & 7) == 0) {
+            uint4 hi, lo;
+            split8(buf, hi, lo);
+            put((f >> 3) - 1, hi, lo);
+        }
+    };
+    emit(e0);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) emit(e1 * x[i]);
+    const float e2o = e2 * kSqrt2;
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+#pragma unroll
+        for (int b = a; b < 16; ++b) emit((a == b ? e2 : e2o) * x[a] * x[b]);
+    }
+#pragma unroll
+    for (int i = 153; i < kFP; ++i) emit(0.f);
+}
+
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
+    const bool ok = ptx::mbar_wait(bar, parity, kWaitPolls);
+    return __syncthreads_and(ok) != 0;
+}
+
+// ---------------------------------------------------------------- 1. chunk states
+__global__ void __launch_bounds__(kThreads, 1)
+tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, float* __restrict__ W, int N,
+                      int n, int F, int64_t stride, int NC, unsigned int* __restrict__ err) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    __shared__ __align__(8) uint64_t mb;
+    __shared__ uint32_t tslot;
+    uint8_t* sV1 = sm + kOffV1s;
+    uint8_t* sAh = sm + kOffAh;
+    uint8_t* sAl = sm + kOffAl;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, bh = blockIdx.y;
+    const int64_t t0 = (int64_t)c * kC;
+    const int nv = (int)min64(kC, (int64_t)N - t0);
+    const int row = (warp & 3) * 32 + lane;
+    const int half = warp >> 2;
+
+    if (tid == 0) {
+        ptx::mbar_init(&mb, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tslot, 256);
+        tmem_relinquish();
+    }
+
+    const bool valid = row < nv;
+    if (half == 0) {
+        // Phi_K of token `row`, as columns of the MN-major A operand (features contiguous)
+        float x[16];
+        if (valid) {
+            ld_row16(k + ((int64_t)bh * N + t0 + row) * kD, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = 0.f;
+        }
+        const float e0 = valid ? 1.f : 0.f, e1 = n >= 2 ? 1.f : 0.f, e2 = n >= 3 ? 1.f : 0.f;
+        phi16_groups(x, e0, e1, e2, [&](int g, uint4 hi, uint4 lo) {
+            *reinterpret_cast<uint4*>(sAh + mnmaj(row, g, kLboPhiK)) = hi;
+            *reinterpret_cast<uint4*>(sAl + mnmaj(row, g, kLboPhiK)) = lo;
+        });
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int g = kFP / 8; g < 32; ++g) {
+            *reinterpret_cast<uint4*>(sAh + mnmaj(row, g, kLboPhiK)) = z4;
+            *reinterpret_cast<uint4*>(sAl + mnmaj(row, g, kLboPhiK)) = z4;
+        }
+    } else {
+        // [v | 1 | 0] of token `row`, MN-major B operand
+        const uint4* vr = reinterpret_cast<const uint4*>(v + ((int64_t)bh * N + t0 + row) * kDV);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const uint4 val = valid ? __ldg(vr + g) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, g, kLboV1)) = val;
+        }
+        const uint4 one = make_uint4(valid ? 0x3F80u : 0u, 0, 0, 0);  // bf16 1.0 in column 64
+        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 8, kLboV1)) = one;
+        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 9, kLboV1)) = make_uint4(0, 0, 0, 0);
+    }
+    ptx::fence_proxy_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = tslot;
+
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(128, kNV, 1, 1);
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            const uint32_t d = tbase + tile * 128;
+#pragma unroll
+            for (int ks = 0; ks < kC / 16; ++ks) {
+                const uint32_t aoff = tile * 16 * 128 + ks * 2 * kLboPhiK;
+                const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
+                mma_bf16(d, smem_desc(sAh + aoff, kLboPhiK, 128), b, id, ks > 0 ? 1u : 0u);
+                mma_bf16(d, smem_desc(sAl + aoff, kLboPhiK, 128), b, id, 1u);
+            }
+        }
+        mma_commit(&mb);
+    }
+    const bool ok = wait_all(&mb, 0);
+    fence_after_sync();
+    if (ok) {
+        // warps 0-3 read tile 0 (features 0..127), warps 4-7 tile 1 (128..255)
+        const int f = half * 128 + row;
+        const uint32_t ta = tbase + ((uint32_t)((warp & 3) * 32) << 16) + half * 128;
+        float a[32], b[32], z[16];
+        tmem_ld32(ta, a);
+        tmem_ld32(ta + 32, b);
+        tmem_ld16(ta + 64, z);
+        tmem_ld_wait();
+        if (f < F) {
+            float* Wc = W + ((int64_t)bh * NC + c) * stride;
+            float4* dst = reinterpret_cast<float4*>(Wc + (int64_t)f * kDV);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[8 + i] = make_float4(b[4 * i], b[4 * i + 1], b[4 * i + 2], b[4 * i + 3]);
+            Wc[(int64_t)F * kDV + f] = z[0];
+        }
+    } else if (tid == 0) {
+        atomicOr(err, kErrPrefillPipe);
+    }
+    if (!ok) ptx::mbar_wait(&mb, 0, kWaitPolls);
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, 256);
+    }
+}
+
+// ---------------------------------------------------------------- 3. chunk outputs
+__global__ void __launch_bounds__(kThreads, 1)
+tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+                    const float* __restrict__ W, float* __restrict__ out, int N, int n, float tau, int F,
+                    int64_t stride, int NC, unsigned int* __restrict__ err) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    __shared__ __align__(8) uint64_t mb_s, mb_o;
+    __shared__ uint32_t tslot;
+    uint8_t* sQ = sm + kOffQ;
+    uint8_t* sK = sm + kOffK;
+    uint8_t* sV1 = sm + kOffV1;
+    uint8_t* sPh = sm + kOffPh;
+    uint8_t* sPl = sm + kOffPl;
+    uint8_t* sQh = sm + kOffQh;
+    uint8_t* sQl = sm + kOffQl;
+    uint8_t* sSh = sm + kOffSh;
+    uint8_t* sSl = sm + kOffSl;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, bh = blockIdx.y;
+    const int64_t t0 = (int64_t)c * kC;
+    const int nv = (int)min64(kC, (int64_t)N - t0);
+    const int row = (warp & 3) * 32 + lane;
+    const int half = warp >> 2;
+    const bool valid = row < nv;
+    const bool inter = c > 0;
+
+    if (tid == 0) {
+        ptx::mbar_init(&mb_s, 1);
+        ptx::mbar_init(&mb_o, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tslot, 256);
+        tmem_relinquish();
+    }
+
+    if (half == 0) {
+        // q, k rows (K-major [128][16]) and Phi_Q of token `row` (K-major [128][160])
+        const int64_t tok = (int64_t)bh * N + t0 + row;
+        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0, k0 = q0, k1 = q0;
+        if (valid) {
+            const uint4* qr = reinterpret_cast<const uint4*>(q + tok * kD);
+            const uint4* kr = reinterpret_cast<const uint4*>(k + tok * kD);
+            q0 = __ldg(qr);
+            q1 = __ldg(qr + 1);
+            k0 = __ldg(kr);
+            k1 = __ldg(kr + 1);
+        }
+        *reinterpret_cast<uint4*>(sQ + kmaj(row, 0, kSboQK)) = q0;
+        *reinterpret_cast<uint4*>(sQ + kmaj(row, 1, kSboQK)) = q1;
+        *reinterpret_cast<uint4*>(sK + kmaj(row, 0, kSboQK)) = k0;
+        *reinterpret_cast<uint4*>(sK + kmaj(row, 1, kSboQK)) = k1;
+        if (inter) {
+            float x[16];
+            const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                x[2 * i] = __uint_as_float(w[i] << 16);
+                x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+            }
+            const float e1 = n >= 2 ? tau : 0.f, e2 = n >= 3 ? 0.5f * tau * tau : 0.f;
+            phi16_groups(x, valid ? 1.f : 0.f, e1, e2, [&](int g, uint4 hi, uint4 lo) {
+                *reinterpret_cast<uint4*>(sQh + kmaj(row, g, kSboPhiQ)) = hi;
+                *reinterpret_cast<uint4*>(sQl + kmaj(row, g, kSboPhiQ)) = lo;
+            });
+        }
+    } else {
+        // [v | 1 | 0] (MN-major [K=128 keys][80]) and the carried state S_<c
+        // (MN-major [K=160 features][80], hi and lo)
+        const uint4* vr = reinterpret_cast<const uint4*>(v + ((int64_t)bh * N + t0 + row) * kDV);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const uint4 val = valid ? __ldg(vr + g) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, g, kLboV1)) = val;
+        }
+        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 8, kLboV1)) = make_uint4(valid ? 0x3F80u : 0u, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 9, kLboV1)) = make_uint4(0, 0, 0, 0);
+        if (inter) {
+            const float* Sg = W + ((int64_t)bh * NC + c) * stride;
+            const int u0 = tid - kThreads / 2;
+            for (int u = u0; u < kFP * 8; u += kThreads / 2) {
+                const int f = u >> 3, g = u & 7;
+                float x[8];
+                if (f < F) {
+                    const float4 a = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8));
+                    const float4 b = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8) + 1);
+                    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+                    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) x[i] = 0.f;
+                }
+                uint4 hi, lo;
+                split8(x, hi, lo);
+                *reinterpret_cast<uint4*>(sSh + mnmaj(f, g, kLboS)) = hi;
+                *reinterpret_cast<uint4*>(sSl + mnmaj(f, g, kLboS)) = lo;
+            }
+            for (int f = u0; f < kFP; f += kThreads / 2) {
+                float x[8] = {f < F ? __ldg(Sg + (int64_t)F * kDV + f) : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                uint4 hi, lo;
+                split8(x, hi, lo);
+                *reinterpret_cast<uint4*>(sSh + mnmaj(f, 8, kLboS)) = hi;
+                *reinterpret_cast<uint4*>(sSl + mnmaj(f, 8, kLboS)) = lo;
+                *reinterpret_cast<uint4*>(sSh + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(sSl + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = tslot;
+    const uint32_t tA = tbase;          // scores, columns [0, 128)
+    const uint32_t tO = tbase + 128;    // [numerator | denominator], columns [128, 208)
+
+    if (tid == 0) {
+        mma_bf16(tA, smem_desc(sQ, 128, kSboQK), smem_desc(sK, 128, kSboQK), idesc_bf16(128, 128, 0, 0), 0u);
+        mma_commit(&mb_s);
+        if (inter) {
+            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < kFP / 16; ++ks) {
+                const uint64_t ah = smem_desc(sQh + ks * 256, 128, kSboPhiQ);
+                const uint64_t al = smem_desc(sQl + ks * 256, 128, kSboPhiQ);
+                const uint64_t bh_ = smem_desc(sSh + ks * 2 * kLboS, kLboS, 128);
+                const uint64_t bl_ = smem_desc(sSl + ks * 2 * kLboS, kLboS, 128);
+                mma_bf16(tO, ah, bh_, id, ks > 0 ? 1u : 0u);
+                mma_bf16(tO, ah, bl_, id, 1u);
+                mma_bf16(tO, al, bh_, id, 1u);
+            }
+        }
+    }
+
+    // pairwise weights P = poly(tau q.k) under the causal mask, hi/lo, K-major
+    bool ok = wait_all(&mb_s, 0);
+    fence_after_sync();
+    if (ok) {
+        const uint32_t ta = tA + ((uint32_t)((warp & 3) * 32) << 16) + half * 64;
+        float s0[32], s1[32];
+        tmem_ld32(ta, s0);
+        tmem_ld32(ta + 32, s1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int j = g * 8 + e;
+                const int key = half * 64 + j;
+                const float sc = j < 32 ? s0[j] : s1[j - 32];
+                const float x = tau * sc;
+                float w = 1.f;
+                if (n >= 3) w = 1.f + x * (1.f + 0.5f * x);
+                else if (n == 2) w = 1.f + x;
+                p[e] = (valid && key <= row) ? w : 0.f;
+            }
+            uint4 hi, lo;
+            split8(p, hi, lo);
+            const int kg = half * 8 + g;
+            *reinterpret_cast<uint4*>(sPh + kmaj(row, kg, kSboP)) = hi;
+            *reinterpret_cast<uint4*>(sPl + kmaj(row, kg, kSboP)) = lo;
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (tid == 0) {
+        if (ok) {
+            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < kC / 16; ++ks) {
+                const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
+                mma_bf16(tO, smem_desc(sPh + ks * 256, 128, kSboP), b, id, (inter || ks > 0) ? 1u : 0u);
+                mma_bf16(tO, smem_desc(sPl + ks * 256, 128, kSboP), b, id, 1u);
+            }
+        }
+        mma_commit(&mb_o);  // tracks every MMA issued so far, also on the error path
+    }
+    const bool done = wait_all(&mb_o, 0);
+    ok = ok && done;
+    fence_after_sync();
+    if (ok) {
+        const uint32_t ta = tO + ((uint32_t)((warp & 3) * 32) << 16);
+        float o[32], dn[16];
+        tmem_ld32(ta + half * 32, o);
+        tmem_ld16(ta + kDV, dn);
+        tmem_ld_wait();
+        if (valid) {
+            const float den = dn[0];
+            float4* dst = reinterpret_cast<float4*>(out + ((int64_t)bh * N + t0 + row) * kDV + half * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(o[4 * i] / den, o[4 * i + 1] / den, o[4 * i + 2] / den, o[4 * i + 3] / den);
+        }
+    } else {
+        if (tid == 0) atomicOr(err, kErrPrefillPipe);
+        // the MMAs in flight get one more bound before TMEM is released
+        if (!done) ptx::mbar_wait(&mb_o, 0, kWaitPolls);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, 256);
+    }
+}
+
+constexpr int kMaxDevices = 64;
+
+cudaError_t set_smem_once(const void* fn, int bytes, std::once_flag* once, cudaError_t* res) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&]() {
+        res[dev] = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    });
+    return res[dev];
+}
+
+}  // namespace
+
+int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, float* out,
+                float* state_out, int BH, int N, int d, int dv, int n, float tau, int64_t F, int64_t stride,
+                cudaStream_t stream) {
+    if (d != kD || dv != kDV || n > 3 || N <= 0 || BH <= 0) return kNotApplicable;
+    unsigned int* err = device_error_word();
+    if (!err) return TAYLOR_ERR_CUDA;
+
+    static std::once_flag once_a[kMaxDevices], once_c[kMaxDevices];
+    static cudaError_t res_a[kMaxDevices], res_c[kMaxDevices];
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(tc_chunk_state_kernel), (int)kSmemState, once_a, res_a);
+    if (e == cudaSuccess)
+        e = set_smem_once(reinterpret_cast<const void*>(tc_chunk_out_kernel), (int)kSmemOut, once_c, res_c);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return TAYLOR_ERR_CUDA;
+    }
+
+    const int NC = (N + kC - 1) / kC;
+    const size_t ws_bytes = (size_t)BH * NC * stride * sizeof(float);
+    float* W = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&W), ws_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return TAYLOR_ERR_OUT_OF_MEMORY;
+    }
+    const dim3 grid(NC, BH);
+    TA_TIMED(stream, "tc_chunk_state_kernel",
+             tc_chunk_state_kernel<<<grid, kThreads, kSmemState, stream>>>(k, v, W, N, n, (int)F, stride, NC, err));
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = launch_state_scan(W, state_out, BH, NC, stride, F * (dv + 1), stream);
+    if (e == cudaSuccess) {
+        TA_TIMED(stream, "tc_chunk_out_kernel",
+                 tc_chunk_out_kernel<<<grid, kThreads, kSmemOut, stream>>>(q, k, v, W, out, N, n, tau, (int)F,
+                                                                           stride, NC, err));
+        e = cudaGetLastError();
+    }
+    const cudaError_t e2 = cudaFreeAsync(W, stream);
+    if (e == cudaSuccess) e = e2;
+    if (e == cudaSuccess) return TAYLOR_OK;
+    return e == cudaErrorMemoryAllocation ? TAYLOR_ERR_OUT_OF_MEMORY : TAYLOR_ERR_CUDA;
 }
 
 }  // namespace tc

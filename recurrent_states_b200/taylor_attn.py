@@ -24,6 +24,7 @@ TAYLOR_ERR_MISALIGNED = -3
 TAYLOR_ERR_CUDA = -4
 TAYLOR_ERR_OUT_OF_MEMORY = -5
 TAYLOR_ERR_SCRATCH_LIMIT = -6
+TAYLOR_ERR_TIMEOUT = -7
 
 # name -> (restype, argtypes); the exported surface of the header
 _P = ctypes.c_void_p
@@ -44,6 +45,7 @@ SIGNATURES = {
     "taylor_attn_state_merge": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "taylor_attn_prefill_f32_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_prefill_noalloc_scratch_floats": (_I64, []),
+    "taylor_attn_device_errors": (_I, [_I, _P]),
     "taylor_attn_timing_enable": (_I, [_I]),
     "taylor_attn_timing_read": (_I, [_I, _P, _P, _P]),
 }
@@ -246,6 +248,15 @@ def taylor_attn_state_merge(a, b, d_k: int, d_v: int, n: int, out=None, stream=N
     _check(lib().taylor_attn_state_merge(_ptr(a), _ptr(b), _ptr(out), B, H, d_k, d_v, n, _stream(stream)),
            "taylor_attn_state_merge")
     return out
+
+
+def taylor_attn_device_errors(clear: bool = True) -> int:
+    """Bits of the device error word (bounded waits that ran out); 0 if none."""
+    flags = ctypes.c_uint(0)
+    rc = lib().taylor_attn_device_errors(int(bool(clear)), ctypes.addressof(flags))
+    if rc not in (TAYLOR_OK, TAYLOR_ERR_TIMEOUT):
+        raise TaylorAttnError(rc, "taylor_attn_device_errors")
+    return int(flags.value)
 
 
 # --------------------------------------------------------------- kernel timing

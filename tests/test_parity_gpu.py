@@ -222,7 +222,8 @@ def test_decode_config_steps(dtype):
     assert state_block_errors(st, ref_S, d, dv, n) <= TOL[dtype]
 
 
-@pytest.mark.parametrize("d,dv,n", [(16, 16, 3), (16, 64, 5), (64, 64, 3), (7, 12, 2)])
+@pytest.mark.parametrize("d,dv,n", [(16, 16, 3), (16, 32, 2), (16, 64, 3), (16, 128, 3), (16, 64, 5),
+                                    (64, 64, 3), (7, 12, 2), (32, 64, 4)])
 def test_decode_from_zero_equals_prefill_reference(d, dv, n):
     N = 150
     q, k, v = synth.qkv(2, 2, N, d, dv, seed=d + dv + n, dtype="f32")
@@ -259,3 +260,8 @@ def test_merge_and_split_prefill():
     TA.taylor_attn_state_merge(sa2, sb, d, dv, n, out=sa2)
     torch.cuda.synchronize()
     assert torch.equal(sa2, merged)
+
+
+def test_no_device_timeouts_recorded():
+    """Every bounded wait in the runs above completed: the error word is clear."""
+    assert TA.taylor_attn_device_errors(clear=True) == 0
