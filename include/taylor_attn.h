@@ -98,9 +98,12 @@ TAYLOR_API int taylor_attn_feature_map(const float* x, float* phi, int64_t T, in
 /* Causal prefill from the empty state (abstract: prefill admits a parallel
  * scan because states are additive across chunks).  q, k, v are bf16.
  * Writes out[B][H][N][d_v] and, when state_out != NULL, the state after all
- * N tokens.  N == 0 writes a zero state.  Takes stream-ordered workspace
- * with cudaMallocAsync/cudaFreeAsync on `stream` (TAYLOR_ERR_OUT_OF_MEMORY
- * if that fails); accumulation is fp32. */
+ * N tokens.  N == 0 writes a zero state.  Takes stream-ordered workspace on
+ * `stream` (one fp32 state per 64-128 tokens per head) from a memory pool the
+ * library creates per device; up to 1 GiB of freed workspace stays cached in
+ * that pool for later calls (taylor_attn_release_workspace returns it).
+ * TAYLOR_ERR_OUT_OF_MEMORY if the workspace cannot be had; accumulation is
+ * fp32. */
 TAYLOR_API int taylor_attn_prefill(const void* q, const void* k, const void* v, float* out,
                         float* state_out, int B, int H, int N, int d_k, int d_v, int n,
                         float tau, cudaStream_t stream);
@@ -110,6 +113,10 @@ TAYLOR_API int taylor_attn_prefill(const void* q, const void* k, const void* v, 
 TAYLOR_API int taylor_attn_prefill_f32(const float* q, const float* k, const float* v, float* out,
                             float* state_out, int B, int H, int N, int d_k, int d_v, int n,
                             float tau, cudaStream_t stream);
+
+/* Returns the prefill workspace cached in the current device's pool to the
+ * driver (synchronises the device first). */
+TAYLOR_API int taylor_attn_release_workspace(void);
 
 /* One new token per (b, h) against carried states (abstract: per-token
  * decoding latency is constant in N).  q, k [B][H][d_k] and v [B][H][d_v]

@@ -75,7 +75,7 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, float* out, float* st
     float* ws = nullptr;
     const bool need_ws = plan.NG > 1 || state_out != nullptr;
     if (need_ws) {
-        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), plan.ws_bytes, stream);
+        cudaError_t e = ta::workspace_alloc(reinterpret_cast<void**>(&ws), plan.ws_bytes, stream);
         if (e != cudaSuccess) {
             cudaGetLastError();
             return TAYLOR_ERR_OUT_OF_MEMORY;
@@ -84,7 +84,7 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, float* out, float* st
     cudaError_t e = ta::launch_prefill_cc(q, k, v, out, state_out, ws, plan, (int)BH, N, d_k, d_v,
                                           n, tau, F, stride, stream);
     if (ws) {
-        cudaError_t e2 = cudaFreeAsync(ws, stream);
+        cudaError_t e2 = ta::workspace_free(ws, stream);
         if (e == cudaSuccess) e = e2;
     }
     return cuda_status(e);

@@ -22,6 +22,10 @@ void end(cudaStream_t s);
         ::ta::timing::end((stream));             \
     } while (0)
 
+// Stream-ordered workspace from the library's per-device pool (workspace.cu).
+cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
+cudaError_t workspace_free(void* ptr, cudaStream_t stream);
+
 // Device address of the error word (errors.cu) on the current device.
 unsigned int* device_error_word();
 constexpr unsigned int kErrDecodeLoad = 1u;

@@ -101,35 +101,48 @@ group_state_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, float* 
 }
 
 // ---------------------------------------------------------------- B
-__global__ void __launch_bounds__(kThreads)
+// Exclusive scan over the NG group states of a head, in place.  Each thread
+// owns 4 consecutive state elements (one float4 column) of one head and keeps
+// the loads of kScanRun groups in flight before it adds them up.  The final
+// running sum is the state after every group; elements past F*(d_v+1) (the
+// padding, never written by the producers) are written as zeros there.
+constexpr int kScanThreads = 128;
+constexpr int kScanRun = 32;
+
+__global__ void __launch_bounds__(kScanThreads)
 scan_kernel(float* __restrict__ W, float* __restrict__ state_out, int NG, int64_t stride,
             int64_t used) {
     const int bh = blockIdx.y;
-    const int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (e >= stride) return;
-    if (e >= used) {
-        if (state_out) state_out[(int64_t)bh * stride + e] = 0.f;
-        return;
-    }
-    float* base = W + (int64_t)bh * NG * stride + e;
-    float run = 0.f;
-    int g = 0;
-    for (; g + 8 <= NG; g += 8) {
-        float x[8];
+    const int64_t e4 = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
+    const int64_t s4 = stride / 4;
+    if (e4 >= s4) return;
+    float4* base = reinterpret_cast<float4*>(W + (int64_t)bh * NG * stride) + e4;
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g0 = 0; g0 < NG; g0 += kScanRun) {
+        float4 x[kScanRun];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) x[j] = base[(int64_t)(g + j) * stride];
+        for (int j = 0; j < kScanRun; ++j)
+            if (g0 + j < NG) x[j] = base[(int64_t)(g0 + j) * s4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            base[(int64_t)(g + j) * stride] = run;
-            run += x[j];
+        for (int j = 0; j < kScanRun; ++j) {
+            if (g0 + j < NG) {
+                base[(int64_t)(g0 + j) * s4] = run;
+                run.x += x[j].x;
+                run.y += x[j].y;
+                run.z += x[j].z;
+                run.w += x[j].w;
+            }
         }
     }
-    for (; g < NG; ++g) {
-        const float x = base[(int64_t)g * stride];
-        base[(int64_t)g * stride] = run;
-        run += x;
+    if (state_out) {
+        const int64_t e = e4 * 4;
+        float4 r = run;
+        if (e + 0 >= used) r.x = 0.f;
+        if (e + 1 >= used) r.y = 0.f;
+        if (e + 2 >= used) r.z = 0.f;
+        if (e + 3 >= used) r.w = 0.f;
+        reinterpret_cast<float4*>(state_out + (int64_t)bh * stride)[e4] = r;
     }
-    if (state_out) state_out[(int64_t)bh * stride + e] = run;
 }
 
 // ---------------------------------------------------------------- C
@@ -333,9 +346,9 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
 #undef TA_LAUNCH_A
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // B
-    const dim3 gB((unsigned)((stride + kThreads - 1) / kThreads), BH);
+    const dim3 gB((unsigned)((stride / 4 + kScanThreads - 1) / kScanThreads), BH);
     TA_TIMED(stream, "cc_scan_kernel",
-             scan_kernel<<<gB, kThreads, 0, stream>>>(W, state_out, plan.NG, stride, F * (dv + 1)));
+             scan_kernel<<<gB, kScanThreads, 0, stream>>>(W, state_out, plan.NG, stride, F * (dv + 1)));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // C
@@ -351,8 +364,8 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
 
 cudaError_t launch_state_scan(float* W, float* state_out, int BH, int NG, int64_t stride, int64_t used,
                               cudaStream_t stream) {
-    const dim3 g((unsigned)((stride + kThreads - 1) / kThreads), BH);
-    TA_TIMED(stream, "scan_kernel", scan_kernel<<<g, kThreads, 0, stream>>>(W, state_out, NG, stride, used));
+    const dim3 g((unsigned)((stride / 4 + kScanThreads - 1) / kScanThreads), BH);
+    TA_TIMED(stream, "scan_kernel", scan_kernel<<<g, kScanThreads, 0, stream>>>(W, state_out, NG, stride, used));
     return cudaGetLastError();
 }
 

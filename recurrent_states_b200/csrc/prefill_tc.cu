@@ -55,7 +55,8 @@ constexpr uint32_t kLboV1 = (kNV / 8) * 128;         // [V|1]: [K=128 keys][80] 
 constexpr uint32_t kSboP = (kC / 8) * 128;           // P: [128][128] K-major
 constexpr uint32_t kSboPhiQ = (kFP / 8) * 128;       // Phi_Q: [128][160] K-major
 constexpr uint32_t kLboS = (kNV / 8) * 128;          // S: [K=160][80] MN-major
-constexpr uint32_t kLboPhiK = (256 / 8) * 128;       // Phi_K^T: [K=128 tokens][256] MN-major
+constexpr uint32_t kLboVT = 16 * 128;                // [V|1|0]^T: [M=128 rows][K=128 tokens] MN-major
+constexpr uint32_t kLboPhiK = (kFP / 8) * 128;       // Phi_K: [K=128 tokens][N=160] MN-major
 
 // chunk_out
 constexpr uint32_t kOffQ = 0;
@@ -68,11 +69,12 @@ constexpr uint32_t kOffQl = kOffQh + kC * kFP * 2;
 constexpr uint32_t kOffSh = kOffQl + kC * kFP * 2;
 constexpr uint32_t kOffSl = kOffSh + kFP * kNV * 2;
 constexpr uint32_t kSmemOut = kOffSl + kFP * kNV * 2;   // 227,328 bytes
-// chunk_state
-constexpr uint32_t kOffV1s = 0;
-constexpr uint32_t kOffAh = kOffV1s + kC * kNV * 2;
-constexpr uint32_t kOffAl = kOffAh + 256 * kC * 2;
-constexpr uint32_t kSmemState = kOffAl + 256 * kC * 2;  // 151,552 bytes
+// chunk_state (transposed: dS^T = [V|1|0]^T Phi_K, so D has the v column on
+// the TMEM lanes and the feature on the TMEM columns)
+constexpr uint32_t kOffVT = 0;
+constexpr uint32_t kOffBh = kOffVT + 128 * kC * 2;
+constexpr uint32_t kOffBl = kOffBh + kC * kFP * 2;
+constexpr uint32_t kSmemState = kOffBl + kC * kFP * 2;  // 114,688 bytes: two CTAs per SM
 
 static_assert(kSmemOut <= 232448 - 256, "chunk_out shared memory");
 
@@ -94,32 +96,36 @@ __device__ __forceinline__ void ld_row16(const bf16* p, float (&x)[16]) {
     }
 }
 
-// Writes the 160 padded features of one token, scaled per degree by
-// (e0, e1, e2), as hi/lo bf16 groups of 8 through `put(group, hi, lo)`.
-template <typename Put>
+// Writes features [8*G0, 8*G1) of the 160 padded features of one token,
+// scaled per degree by (e0, e1, e2), as hi/lo bf16 groups of 8 through
+// `put(group, hi, lo)`.  All indices are compile-time constants after
+// unrolling, so features outside the range cost nothing.
+template <int G0, int G1, typename Put>
 __device__ __forceinline__ void phi16_groups(const float (&x)[16], float e0, float e1, float e2, Put put) {
     float buf[8];
     int f = 0;
-    auto emit = [&](float val) {
-        buf[f & 7] = val;
-        ++f;
-        if ((f & 7) == 0) {
-            uint4 hi, lo;
-            split8(buf, hi, lo);
-            put((f >> 3) - 1, hi, lo);
+    auto emit = [&](auto make) {
+        if (f >= 8 * G0 && f < 8 * G1) {
+            buf[f & 7] = make();
+            if ((f & 7) == 7) {
+                uint4 hi, lo;
+                split8(buf, hi, lo);
+                put(f >> 3, hi, lo);
+            }
         }
+        ++f;
     };
-    emit(e0);
+    emit([&] { return e0; });
 #pragma unroll
-    for (int i = 0; i < 16; ++i) emit(e1 * x[i]);
+    for (int i = 0; i < 16; ++i) emit([&] { return e1 * x[i]; });
     const float e2o = e2 * kSqrt2;
 #pragma unroll
     for (int a = 0; a < 16; ++a) {
 #pragma unroll
-        for (int b = a; b < 16; ++b) emit((a == b ? e2 : e2o) * x[a] * x[b]);
+        for (int b = a; b < 16; ++b) emit([&] { return (a == b ? e2 : e2o) * x[a] * x[b]; });
     }
 #pragma unroll
-    for (int i = 153; i < kFP; ++i) emit(0.f);
+    for (int i = 153; i < kFP; ++i) emit([&] { return 0.f; });
 }
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
@@ -128,15 +134,20 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- 1. chunk states
-__global__ void __launch_bounds__(kThreads, 1)
+// dS_c^T [128 x 160] = [V_c | 1 | 0]^T [128 x 128 tokens] x Phi_K,c [128 tokens x 160]
+// with Phi_K as hi + lo.  Lane c < 64 of D is column c of S_v, lane 64 is z.
+// The result is staged in shared memory in the state layout and written with
+// one bulk copy.
+__global__ void __launch_bounds__(kThreads, 2)
 tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, float* __restrict__ W, int N,
                       int n, int F, int64_t stride, int NC, unsigned int* __restrict__ err) {
     extern __shared__ __align__(1024) uint8_t sm[];
     __shared__ __align__(8) uint64_t mb;
     __shared__ uint32_t tslot;
-    uint8_t* sV1 = sm + kOffV1s;
-    uint8_t* sAh = sm + kOffAh;
-    uint8_t* sAl = sm + kOffAl;
+    uint8_t* sVT = sm + kOffVT;
+    uint8_t* sBh = sm + kOffBh;
+    uint8_t* sBl = sm + kOffBl;
+    float* sOut = reinterpret_cast<float*>(sm + kOffBh);  // reused once the MMAs are done
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, bh = blockIdx.y;
@@ -144,6 +155,7 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
     const int nv = (int)min64(kC, (int64_t)N - t0);
     const int row = (warp & 3) * 32 + lane;
     const int half = warp >> 2;
+    const bool valid = row < nv;
 
     if (tid == 0) {
         ptx::mbar_init(&mb, 1);
@@ -154,39 +166,35 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
         tmem_relinquish();
     }
 
-    const bool valid = row < nv;
-    if (half == 0) {
-        // Phi_K of token `row`, as columns of the MN-major A operand (features contiguous)
-        float x[16];
-        if (valid) {
-            ld_row16(k + ((int64_t)bh * N + t0 + row) * kD, x);
-        } else {
+    // token `row`: half its features (one K row of the MN-major B operand)
+    // and half its [v | 1 | 0] column (one K column of the MN-major A operand)
+    const int64_t tok = (int64_t)bh * N + t0 + row;
+    const uint4* vr = reinterpret_cast<const uint4*>(v + tok * kDV) + half * 4;
+    uint4 val[4];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = 0.f;
-        }
-        const float e0 = valid ? 1.f : 0.f, e1 = n >= 2 ? 1.f : 0.f, e2 = n >= 3 ? 1.f : 0.f;
-        phi16_groups(x, e0, e1, e2, [&](int g, uint4 hi, uint4 lo) {
-            *reinterpret_cast<uint4*>(sAh + mnmaj(row, g, kLboPhiK)) = hi;
-            *reinterpret_cast<uint4*>(sAl + mnmaj(row, g, kLboPhiK)) = lo;
-        });
-        const uint4 z4 = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int g = kFP / 8; g < 32; ++g) {
-            *reinterpret_cast<uint4*>(sAh + mnmaj(row, g, kLboPhiK)) = z4;
-            *reinterpret_cast<uint4*>(sAl + mnmaj(row, g, kLboPhiK)) = z4;
-        }
+    for (int g = 0; g < 4; ++g) val[g] = valid ? __ldg(vr + g) : make_uint4(0, 0, 0, 0);
+    float x[16];
+    if (valid) {
+        ld_row16(k + tok * kD, x);
     } else {
-        // [v | 1 | 0] of token `row`, MN-major B operand
-        const uint4* vr = reinterpret_cast<const uint4*>(v + ((int64_t)bh * N + t0 + row) * kDV);
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            const uint4 val = valid ? __ldg(vr + g) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, g, kLboV1)) = val;
-        }
-        const uint4 one = make_uint4(valid ? 0x3F80u : 0u, 0, 0, 0);  // bf16 1.0 in column 64
-        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 8, kLboV1)) = one;
-        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 9, kLboV1)) = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 16; ++i) x[i] = 0.f;
     }
+#pragma unroll
+    for (int g = 0; g < 4; ++g) *reinterpret_cast<uint4*>(sVT + mnmaj(row, half * 4 + g, kLboVT)) = val[g];
+    if (half == 1) {
+        *reinterpret_cast<uint4*>(sVT + mnmaj(row, 8, kLboVT)) = make_uint4(valid ? 0x3F80u : 0u, 0, 0, 0);
+#pragma unroll
+        for (int g = 9; g < 16; ++g) *reinterpret_cast<uint4*>(sVT + mnmaj(row, g, kLboVT)) = make_uint4(0, 0, 0, 0);
+    }
+    const float e0 = valid ? 1.f : 0.f, e1 = n >= 2 ? 1.f : 0.f, e2 = n >= 3 ? 1.f : 0.f;
+    auto put = [&](int g, uint4 hi, uint4 lo) {
+        *reinterpret_cast<uint4*>(sBh + mnmaj(row, g, kLboPhiK)) = hi;
+        *reinterpret_cast<uint4*>(sBl + mnmaj(row, g, kLboPhiK)) = lo;
+    };
+    if (half == 0) phi16_groups<0, 10>(x, e0, e1, e2, put);
+    else phi16_groups<10, 20>(x, e0, e1, e2, put);
+
     ptx::fence_proxy_async_smem();
     fence_before_sync();
     __syncthreads();
@@ -194,46 +202,54 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
     const uint32_t tbase = tslot;
 
     if (tid == 0) {
-        const uint32_t id = idesc_bf16(128, kNV, 1, 1);
+        const uint32_t id = idesc_bf16(128, kFP, 1, 1);
 #pragma unroll
-        for (int tile = 0; tile < 2; ++tile) {
-            const uint32_t d = tbase + tile * 128;
-#pragma unroll
-            for (int ks = 0; ks < kC / 16; ++ks) {
-                const uint32_t aoff = tile * 16 * 128 + ks * 2 * kLboPhiK;
-                const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
-                mma_bf16(d, smem_desc(sAh + aoff, kLboPhiK, 128), b, id, ks > 0 ? 1u : 0u);
-                mma_bf16(d, smem_desc(sAl + aoff, kLboPhiK, 128), b, id, 1u);
-            }
+        for (int ks = 0; ks < kC / 16; ++ks) {
+            const uint64_t a = smem_desc(sVT + ks * 2 * kLboVT, kLboVT, 128);
+            mma_bf16(tbase, a, smem_desc(sBh + ks * 2 * kLboPhiK, kLboPhiK, 128), id, ks > 0 ? 1u : 0u);
+            mma_bf16(tbase, a, smem_desc(sBl + ks * 2 * kLboPhiK, kLboPhiK, 128), id, 1u);
         }
         mma_commit(&mb);
     }
     const bool ok = wait_all(&mb, 0);
     fence_after_sync();
+    const uint32_t bytes = (uint32_t)(((int64_t)F * (kDV + 1) * 4 + 15) / 16 * 16);
     if (ok) {
-        // warps 0-3 read tile 0 (features 0..127), warps 4-7 tile 1 (128..255)
-        const int f = half * 128 + row;
-        const uint32_t ta = tbase + ((uint32_t)((warp & 3) * 32) << 16) + half * 128;
-        float a[32], b[32], z[16];
-        tmem_ld32(ta, a);
-        tmem_ld32(ta + 32, b);
-        tmem_ld16(ta + 64, z);
-        tmem_ld_wait();
-        if (f < F) {
-            float* Wc = W + ((int64_t)bh * NC + c) * stride;
-            float4* dst = reinterpret_cast<float4*>(Wc + (int64_t)f * kDV);
+        // warps 0,1 (+4,5) hold S_v columns 0..63 on their lanes; warp 2 lane 0
+        // (+ warp 6) holds z.  Warp w and w+4 split the 160 feature columns.
+        const int wq = warp & 3;
+        if (wq < 3) {
+            const int col = wq * 32 + lane;
+            const uint32_t ta = tbase + ((uint32_t)(wq * 32) << 16);
+            const int fb = half * 80;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+            for (int part = 0; part < 5; ++part) {
+                float r[16];
+                tmem_ld16(ta + fb + part * 16, r);
+                tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[8 + i] = make_float4(b[4 * i], b[4 * i + 1], b[4 * i + 2], b[4 * i + 3]);
-            Wc[(int64_t)F * kDV + f] = z[0];
+                for (int i = 0; i < 16; ++i) {
+                    const int f = fb + part * 16 + i;
+                    if (f < F) {
+                        if (col < kDV) sOut[f * kDV + col] = r[i];
+                        else if (col == kDV) sOut[F * kDV + f] = r[i];
+                    }
+                }
+            }
         }
+        if (tid < 4) sOut[F * (kDV + 1) + tid] = 0.f;  // tail of the last 16-byte unit
+        ptx::fence_proxy_async_smem();
     } else if (tid == 0) {
         atomicOr(err, kErrPrefillPipe);
     }
     if (!ok) ptx::mbar_wait(&mb, 0, kWaitPolls);
     fence_before_sync();
     __syncthreads();
+    if (ok && tid == 0) {
+        ptx::bulk_s2g(W + ((int64_t)bh * NC + c) * stride, sOut, bytes);
+        ptx::bulk_commit();
+        ptx::bulk_wait_read_all();
+    }
     if (warp == 0) {
         fence_after_sync();
         tmem_dealloc(tbase, 256);
@@ -241,13 +257,23 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
 }
 
 // ---------------------------------------------------------------- 3. chunk outputs
-__global__ void __launch_bounds__(kThreads, 1)
+// Warps 0-7 stage operands, build Phi_Q, S_<c and P, and run the epilogue;
+// warp 8 allocates TMEM and issues every MMA, driven by mbarriers that the
+// other warps arrive on, so no warp waits for the MMA issue itself.
+constexpr int kOutThreads = kThreads + 32;
+
+__device__ __forceinline__ void compute_bar_sync() {
+    asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");
+}
+
+__global__ void __launch_bounds__(kOutThreads, 1)
 tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                     const float* __restrict__ W, float* __restrict__ out, int N, int n, float tau, int F,
                     int64_t stride, int NC, unsigned int* __restrict__ err) {
     extern __shared__ __align__(1024) uint8_t sm[];
-    __shared__ __align__(8) uint64_t mb_s, mb_o;
+    __shared__ __align__(8) uint64_t mb_ld, mb_s, mb_o, bar_qk, bar_ops, bar_p;
     __shared__ uint32_t tslot;
+    __shared__ int mma_fail;
     uint8_t* sQ = sm + kOffQ;
     uint8_t* sK = sm + kOffK;
     uint8_t* sV1 = sm + kOffV1;
@@ -257,43 +283,126 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     uint8_t* sQl = sm + kOffQl;
     uint8_t* sSh = sm + kOffSh;
     uint8_t* sSl = sm + kOffSl;
+    // the carried state arrives as fp32 in the P buffers, which are free
+    // until the pairwise weights are written
+    const float* sS32 = reinterpret_cast<const float*>(sPh);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, bh = blockIdx.y;
     const int64_t t0 = (int64_t)c * kC;
     const int nv = (int)min64(kC, (int64_t)N - t0);
-    const int row = (warp & 3) * 32 + lane;
-    const int half = warp >> 2;
-    const bool valid = row < nv;
     const bool inter = c > 0;
+    const uint32_t sbytes = (uint32_t)(((int64_t)F * (kDV + 1) * 4 + 15) / 16 * 16);
 
     if (tid == 0) {
+        ptx::mbar_init(&mb_ld, 1);
         ptx::mbar_init(&mb_s, 1);
         ptx::mbar_init(&mb_o, 1);
+        ptx::mbar_init(&bar_qk, kThreads);
+        ptx::mbar_init(&bar_ops, kThreads);
+        ptx::mbar_init(&bar_p, kThreads);
+        mma_fail = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0) {
+    if (warp == 8) {
         tmem_alloc(&tslot, 256);
         tmem_relinquish();
     }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = tslot;
+    const uint32_t tA = tbase;          // scores, columns [0, 128)
+    const uint32_t tO = tbase + 128;    // [numerator | denominator], columns [128, 208)
 
-    if (half == 0) {
-        // q, k rows (K-major [128][16]) and Phi_Q of token `row` (K-major [128][160])
+    if (warp == 8) {
+        // ------------------------------------------------ MMA issue (one thread)
+        if (lane == 0) {
+            if (inter) {
+                ptx::mbar_arrive_expect_tx(&mb_ld, sbytes);
+                ptx::bulk_g2s(sPh, W + ((int64_t)bh * NC + c) * stride, sbytes, &mb_ld);
+            }
+            bool good = ptx::mbar_wait(&bar_qk, 0, kWaitPolls);
+            fence_after_sync();
+            if (good)
+                mma_bf16(tA, smem_desc(sQ, 128, kSboQK), smem_desc(sK, 128, kSboQK), idesc_bf16(128, 128, 0, 0), 0u);
+            mma_commit(&mb_s);
+            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
+            if (inter && good) {
+                good = ptx::mbar_wait(&bar_ops, 0, kWaitPolls);
+                fence_after_sync();
+                if (good) {
+#pragma unroll
+                    for (int ks = 0; ks < kFP / 16; ++ks) {
+                        const uint64_t ah = smem_desc(sQh + ks * 256, 128, kSboPhiQ);
+                        const uint64_t al = smem_desc(sQl + ks * 256, 128, kSboPhiQ);
+                        const uint64_t bh_ = smem_desc(sSh + ks * 2 * kLboS, kLboS, 128);
+                        const uint64_t bl_ = smem_desc(sSl + ks * 2 * kLboS, kLboS, 128);
+                        mma_bf16(tO, ah, bh_, id, ks > 0 ? 1u : 0u);
+                        mma_bf16(tO, ah, bl_, id, 1u);
+                        mma_bf16(tO, al, bh_, id, 1u);
+                    }
+                }
+            }
+            if (good) {
+                good = ptx::mbar_wait(&bar_p, 0, kWaitPolls);
+                fence_after_sync();
+                if (good) {
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks) {
+                        const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
+                        mma_bf16(tO, smem_desc(sPh + ks * 256, 128, kSboP), b, id, (inter || ks > 0) ? 1u : 0u);
+                        mma_bf16(tO, smem_desc(sPl + ks * 256, 128, kSboP), b, id, 1u);
+                    }
+                }
+            }
+            if (!good) {
+                mma_fail = 1;
+                atomicOr(err, kErrPrefillPipe);
+            }
+            mma_commit(&mb_o);  // tracks every MMA issued, also on the error path
+        }
+    } else {
+        // ------------------------------------------------ operands and epilogue
+        const int row = (warp & 3) * 32 + lane;
+        const int half = warp >> 2;
+        const bool valid = row < nv;
         const int64_t tok = (int64_t)bh * N + t0 + row;
-        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0, k0 = q0, k1 = q0;
+
+        // q, k rows (K-major [128][16]); half of [v | 1 | 0] (MN-major [K=128][80])
+        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;
         if (valid) {
             const uint4* qr = reinterpret_cast<const uint4*>(q + tok * kD);
-            const uint4* kr = reinterpret_cast<const uint4*>(k + tok * kD);
             q0 = __ldg(qr);
             q1 = __ldg(qr + 1);
-            k0 = __ldg(kr);
-            k1 = __ldg(kr + 1);
         }
-        *reinterpret_cast<uint4*>(sQ + kmaj(row, 0, kSboQK)) = q0;
-        *reinterpret_cast<uint4*>(sQ + kmaj(row, 1, kSboQK)) = q1;
-        *reinterpret_cast<uint4*>(sK + kmaj(row, 0, kSboQK)) = k0;
-        *reinterpret_cast<uint4*>(sK + kmaj(row, 1, kSboQK)) = k1;
+        const uint4* vr = reinterpret_cast<const uint4*>(v + tok * kDV) + half * 4;
+        uint4 val[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) val[g] = valid ? __ldg(vr + g) : make_uint4(0, 0, 0, 0);
+        if (half == 0) {
+            uint4 k0 = make_uint4(0, 0, 0, 0), k1 = k0;
+            if (valid) {
+                const uint4* kr = reinterpret_cast<const uint4*>(k + tok * kD);
+                k0 = __ldg(kr);
+                k1 = __ldg(kr + 1);
+            }
+            *reinterpret_cast<uint4*>(sQ + kmaj(row, 0, kSboQK)) = q0;
+            *reinterpret_cast<uint4*>(sQ + kmaj(row, 1, kSboQK)) = q1;
+            *reinterpret_cast<uint4*>(sK + kmaj(row, 0, kSboQK)) = k0;
+            *reinterpret_cast<uint4*>(sK + kmaj(row, 1, kSboQK)) = k1;
+        } else {
+            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 8, kLboV1)) = make_uint4(valid ? 0x3F80u : 0u, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 9, kLboV1)) = make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) *reinterpret_cast<uint4*>(sV1 + mnmaj(row, half * 4 + g, kLboV1)) = val[g];
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&bar_qk);
+
+        bool ok = true;
         if (inter) {
+            // half of Phi_Q for token `row`, while S_<c is in flight
             float x[16];
             const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
@@ -302,149 +411,106 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
                 x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
             }
             const float e1 = n >= 2 ? tau : 0.f, e2 = n >= 3 ? 0.5f * tau * tau : 0.f;
-            phi16_groups(x, valid ? 1.f : 0.f, e1, e2, [&](int g, uint4 hi, uint4 lo) {
+            auto put = [&](int g, uint4 hi, uint4 lo) {
                 *reinterpret_cast<uint4*>(sQh + kmaj(row, g, kSboPhiQ)) = hi;
                 *reinterpret_cast<uint4*>(sQl + kmaj(row, g, kSboPhiQ)) = lo;
-            });
-        }
-    } else {
-        // [v | 1 | 0] (MN-major [K=128 keys][80]) and the carried state S_<c
-        // (MN-major [K=160 features][80], hi and lo)
-        const uint4* vr = reinterpret_cast<const uint4*>(v + ((int64_t)bh * N + t0 + row) * kDV);
+            };
+            if (half == 0) phi16_groups<0, 10>(x, valid ? 1.f : 0.f, e1, e2, put);
+            else phi16_groups<10, 20>(x, valid ? 1.f : 0.f, e1, e2, put);
+            // S_<c from fp32 to hi/lo, MN-major [K=160][80]
+            ok = ptx::mbar_wait(&mb_ld, 0, kWaitPolls);
+            if (ok) {
+                for (int u = tid; u < kFP * 8; u += kThreads) {
+                    const int f = u >> 3, g = u & 7;
+                    float xs[8];
+                    if (f < F) {
+                        const float4 a = reinterpret_cast<const float4*>(sS32 + f * kDV + g * 8)[0];
+                        const float4 b = reinterpret_cast<const float4*>(sS32 + f * kDV + g * 8)[1];
+                        xs[0] = a.x; xs[1] = a.y; xs[2] = a.z; xs[3] = a.w;
+                        xs[4] = b.x; xs[5] = b.y; xs[6] = b.z; xs[7] = b.w;
+                    } else {
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            const uint4 val = valid ? __ldg(vr + g) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, g, kLboV1)) = val;
+                        for (int i = 0; i < 8; ++i) xs[i] = 0.f;
+                    }
+                    uint4 hi, lo;
+                    split8(xs, hi, lo);
+                    *reinterpret_cast<uint4*>(sSh + mnmaj(f, g, kLboS)) = hi;
+                    *reinterpret_cast<uint4*>(sSl + mnmaj(f, g, kLboS)) = lo;
+                }
+                for (int f = tid; f < kFP; f += kThreads) {
+                    float xs[8] = {f < F ? sS32[F * kDV + f] : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    uint4 hi, lo;
+                    split8(xs, hi, lo);
+                    *reinterpret_cast<uint4*>(sSh + mnmaj(f, 8, kLboS)) = hi;
+                    *reinterpret_cast<uint4*>(sSl + mnmaj(f, 8, kLboS)) = lo;
+                    *reinterpret_cast<uint4*>(sSh + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(sSl + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&bar_ops);
+            compute_bar_sync();  // every read of the staged fp32 S precedes the P writes below
         }
-        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 8, kLboV1)) = make_uint4(valid ? 0x3F80u : 0u, 0, 0, 0);
-        *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 9, kLboV1)) = make_uint4(0, 0, 0, 0);
-        if (inter) {
-            const float* Sg = W + ((int64_t)bh * NC + c) * stride;
-            const int u0 = tid - kThreads / 2;
-            for (int u = u0; u < kFP * 8; u += kThreads / 2) {
-                const int f = u >> 3, g = u & 7;
-                float x[8];
-                if (f < F) {
-                    const float4 a = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8));
-                    const float4 b = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8) + 1);
-                    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-                    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-                } else {
+
+        // pairwise weights P = poly(tau q.k) under the causal mask, hi/lo, K-major
+        ok = ptx::mbar_wait(&mb_s, 0, kWaitPolls) && ok;
+        fence_after_sync();
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        {
+            float s0[32], s1[32];
+            tmem_ld32(tA + lane_off + half * 64, s0);
+            tmem_ld32(tA + lane_off + half * 64 + 32, s1);
+            tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) x[i] = 0.f;
+            for (int g = 0; g < 8; ++g) {
+                float p[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int j = g * 8 + e;
+                    const int key = half * 64 + j;
+                    const float sc = j < 32 ? s0[j] : s1[j - 32];
+                    const float xx = tau * sc;
+                    float w = 1.f;
+                    if (n >= 3) w = 1.f + xx * (1.f + 0.5f * xx);
+                    else if (n == 2) w = 1.f + xx;
+                    p[e] = (valid && key <= row) ? w : 0.f;
                 }
                 uint4 hi, lo;
-                split8(x, hi, lo);
-                *reinterpret_cast<uint4*>(sSh + mnmaj(f, g, kLboS)) = hi;
-                *reinterpret_cast<uint4*>(sSl + mnmaj(f, g, kLboS)) = lo;
-            }
-            for (int f = u0; f < kFP; f += kThreads / 2) {
-                float x[8] = {f < F ? __ldg(Sg + (int64_t)F * kDV + f) : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                uint4 hi, lo;
-                split8(x, hi, lo);
-                *reinterpret_cast<uint4*>(sSh + mnmaj(f, 8, kLboS)) = hi;
-                *reinterpret_cast<uint4*>(sSl + mnmaj(f, 8, kLboS)) = lo;
-                *reinterpret_cast<uint4*>(sSh + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(sSl + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                split8(p, hi, lo);
+                const int kg = half * 8 + g;
+                *reinterpret_cast<uint4*>(sPh + kmaj(row, kg, kSboP)) = hi;
+                *reinterpret_cast<uint4*>(sPl + kmaj(row, kg, kSboP)) = lo;
             }
         }
-    }
-    ptx::fence_proxy_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tbase = tslot;
-    const uint32_t tA = tbase;          // scores, columns [0, 128)
-    const uint32_t tO = tbase + 128;    // [numerator | denominator], columns [128, 208)
+        ptx::fence_proxy_async_smem();
+        fence_before_sync();
+        ptx::mbar_arrive(&bar_p);
 
-    if (tid == 0) {
-        mma_bf16(tA, smem_desc(sQ, 128, kSboQK), smem_desc(sK, 128, kSboQK), idesc_bf16(128, 128, 0, 0), 0u);
-        mma_commit(&mb_s);
-        if (inter) {
-            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < kFP / 16; ++ks) {
-                const uint64_t ah = smem_desc(sQh + ks * 256, 128, kSboPhiQ);
-                const uint64_t al = smem_desc(sQl + ks * 256, 128, kSboPhiQ);
-                const uint64_t bh_ = smem_desc(sSh + ks * 2 * kLboS, kLboS, 128);
-                const uint64_t bl_ = smem_desc(sSl + ks * 2 * kLboS, kLboS, 128);
-                mma_bf16(tO, ah, bh_, id, ks > 0 ? 1u : 0u);
-                mma_bf16(tO, ah, bl_, id, 1u);
-                mma_bf16(tO, al, bh_, id, 1u);
-            }
-        }
-    }
-
-    // pairwise weights P = poly(tau q.k) under the causal mask, hi/lo, K-major
-    bool ok = wait_all(&mb_s, 0);
-    fence_after_sync();
-    if (ok) {
-        const uint32_t ta = tA + ((uint32_t)((warp & 3) * 32) << 16) + half * 64;
-        float s0[32], s1[32];
-        tmem_ld32(ta, s0);
-        tmem_ld32(ta + 32, s1);
-        tmem_ld_wait();
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            float p[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int j = g * 8 + e;
-                const int key = half * 64 + j;
-                const float sc = j < 32 ? s0[j] : s1[j - 32];
-                const float x = tau * sc;
-                float w = 1.f;
-                if (n >= 3) w = 1.f + x * (1.f + 0.5f * x);
-                else if (n == 2) w = 1.f + x;
-                p[e] = (valid && key <= row) ? w : 0.f;
-            }
-            uint4 hi, lo;
-            split8(p, hi, lo);
-            const int kg = half * 8 + g;
-            *reinterpret_cast<uint4*>(sPh + kmaj(row, kg, kSboP)) = hi;
-            *reinterpret_cast<uint4*>(sPl + kmaj(row, kg, kSboP)) = lo;
-        }
-    }
-    ptx::fence_proxy_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    if (tid == 0) {
+        // epilogue: o = numerator / denominator
+        const bool done = ptx::mbar_wait(&mb_o, 0, kWaitPolls);
+        fence_after_sync();
+        ok = ok && done && mma_fail == 0;
         if (ok) {
-            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
+            float o[32], dn[16];
+            tmem_ld32(tO + lane_off + half * 32, o);
+            tmem_ld16(tO + lane_off + kDV, dn);
+            tmem_ld_wait();
+            if (valid) {
+                const float den = dn[0];
+                float4* dst = reinterpret_cast<float4*>(out + tok * kDV + half * 32);
 #pragma unroll
-            for (int ks = 0; ks < kC / 16; ++ks) {
-                const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
-                mma_bf16(tO, smem_desc(sPh + ks * 256, 128, kSboP), b, id, (inter || ks > 0) ? 1u : 0u);
-                mma_bf16(tO, smem_desc(sPl + ks * 256, 128, kSboP), b, id, 1u);
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(o[4 * i] / den, o[4 * i + 1] / den, o[4 * i + 2] / den,
+                                         o[4 * i + 3] / den);
             }
+        } else {
+            if (tid == 0) atomicOr(err, kErrPrefillPipe);
+            if (!done) ptx::mbar_wait(&mb_o, 0, kWaitPolls);  // one more bound for MMAs in flight
         }
-        mma_commit(&mb_o);  // tracks every MMA issued so far, also on the error path
-    }
-    const bool done = wait_all(&mb_o, 0);
-    ok = ok && done;
-    fence_after_sync();
-    if (ok) {
-        const uint32_t ta = tO + ((uint32_t)((warp & 3) * 32) << 16);
-        float o[32], dn[16];
-        tmem_ld32(ta + half * 32, o);
-        tmem_ld16(ta + kDV, dn);
-        tmem_ld_wait();
-        if (valid) {
-            const float den = dn[0];
-            float4* dst = reinterpret_cast<float4*>(out + ((int64_t)bh * N + t0 + row) * kDV + half * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(o[4 * i] / den, o[4 * i + 1] / den, o[4 * i + 2] / den, o[4 * i + 3] / den);
-        }
-    } else {
-        if (tid == 0) atomicOr(err, kErrPrefillPipe);
-        // the MMAs in flight get one more bound before TMEM is released
-        if (!done) ptx::mbar_wait(&mb_o, 0, kWaitPolls);
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
         fence_after_sync();
         tmem_dealloc(tbase, 256);
     }
@@ -485,7 +551,7 @@ int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloa
     const int NC = (N + kC - 1) / kC;
     const size_t ws_bytes = (size_t)BH * NC * stride * sizeof(float);
     float* W = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&W), ws_bytes, stream) != cudaSuccess) {
+    if (workspace_alloc(reinterpret_cast<void**>(&W), ws_bytes, stream) != cudaSuccess) {
         cudaGetLastError();
         return TAYLOR_ERR_OUT_OF_MEMORY;
     }
@@ -496,11 +562,11 @@ int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloa
     if (e == cudaSuccess) e = launch_state_scan(W, state_out, BH, NC, stride, F * (dv + 1), stream);
     if (e == cudaSuccess) {
         TA_TIMED(stream, "tc_chunk_out_kernel",
-                 tc_chunk_out_kernel<<<grid, kThreads, kSmemOut, stream>>>(q, k, v, W, out, N, n, tau, (int)F,
+                 tc_chunk_out_kernel<<<grid, kOutThreads, kSmemOut, stream>>>(q, k, v, W, out, N, n, tau, (int)F,
                                                                            stride, NC, err));
         e = cudaGetLastError();
     }
-    const cudaError_t e2 = cudaFreeAsync(W, stream);
+    const cudaError_t e2 = workspace_free(W, stream);
     if (e == cudaSuccess) e = e2;
     if (e == cudaSuccess) return TAYLOR_OK;
     return e == cudaErrorMemoryAllocation ? TAYLOR_ERR_OUT_OF_MEMORY : TAYLOR_ERR_CUDA;

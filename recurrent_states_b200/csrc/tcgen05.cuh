@@ -136,24 +136,23 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 // ---------------------------------------------------------------- bf16 hi/lo split
 
 // x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi): 16 significant bits.
-__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-    hi = __float2bfloat16_rn(x);
-    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+// Two values per conversion instruction; bf16 -> fp32 is a shift.
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
+    const float r0 = x0 - __uint_as_float(hb << 16);
+    const float r1 = x1 - __uint_as_float(hb & 0xffff0000u);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(r0, r1);
+    hi = hb;
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // Packs 8 floats as hi and lo bf16 vectors (16 bytes each).
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        split_bf16(x[2 * i], h0, l0);
-        split_bf16(x[2 * i + 1], h1, l1);
-        h[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-        l[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-    }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
+    split2(x[0], x[1], hi.x, lo.x);
+    split2(x[2], x[3], hi.y, lo.y);
+    split2(x[4], x[5], hi.z, lo.z);
+    split2(x[6], x[7], hi.w, lo.w);
 }
 
 }  // namespace tc

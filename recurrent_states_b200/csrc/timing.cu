@@ -23,7 +23,23 @@ struct Rec {
 
 thread_local bool g_on = false;
 thread_local std::vector<Rec> g_recs;
-thread_local cudaStream_t g_stream = nullptr;
+// Events are created once and reused, so that enabling the timing adds only
+// two event records per launch to the host's enqueue path.
+thread_local std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return e;
+}
 
 }  // namespace
 
@@ -31,13 +47,9 @@ bool enabled() { return g_on; }
 
 void begin(cudaStream_t s, const char* name) {
     if (!g_on) return;
-    Rec r{name, nullptr, nullptr};
-    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) {
-        cudaGetLastError();
-        return;
-    }
+    Rec r{name, take_event(), take_event()};
+    if (!r.start || !r.stop) return;
     cudaEventRecord(r.start, s);
-    g_stream = s;
     g_recs.push_back(r);
 }
 
@@ -53,6 +65,15 @@ extern "C" {
 
 int taylor_attn_timing_enable(int on) {
     ta::timing::g_on = on != 0;
+    // pre-create a pool so the first timed launches do not pay for creation
+    while (on && ta::timing::g_pool.size() < 256) {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            cudaGetLastError();
+            return TAYLOR_ERR_CUDA;
+        }
+        ta::timing::g_pool.push_back(e);
+    }
     return TAYLOR_OK;
 }
 
@@ -79,8 +100,8 @@ int taylor_attn_timing_read(int max_kernels, char* names, int* launches, float* 
         }
         cnt[i] += 1;
         ms[i] += t;
-        cudaEventDestroy(r.start);
-        cudaEventDestroy(r.stop);
+        ta::timing::g_pool.push_back(r.start);
+        ta::timing::g_pool.push_back(r.stop);
     }
     g_recs.clear();
     if (rc != TAYLOR_OK) return rc;

@@ -46,6 +46,7 @@ SIGNATURES = {
     "taylor_attn_prefill_f32_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_prefill_noalloc_scratch_floats": (_I64, []),
     "taylor_attn_device_errors": (_I, [_I, _P]),
+    "taylor_attn_release_workspace": (_I, []),
     "taylor_attn_timing_enable": (_I, [_I]),
     "taylor_attn_timing_read": (_I, [_I, _P, _P, _P]),
 }
@@ -248,6 +249,10 @@ def taylor_attn_state_merge(a, b, d_k: int, d_v: int, n: int, out=None, stream=N
     _check(lib().taylor_attn_state_merge(_ptr(a), _ptr(b), _ptr(out), B, H, d_k, d_v, n, _stream(stream)),
            "taylor_attn_state_merge")
     return out
+
+
+def taylor_attn_release_workspace() -> None:
+    _check(lib().taylor_attn_release_workspace(), "taylor_attn_release_workspace")
 
 
 def taylor_attn_device_errors(clear: bool = True) -> int:
