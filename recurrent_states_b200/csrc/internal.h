@@ -55,7 +55,25 @@ CcPlan plan_prefill_cc(int BH, int N, int d, int dv, int n, int64_t F, int64_t s
 // In place: W[bh][g] <- sum_{g' < g} W[bh][g'] over the first `used` floats
 // of each state; state_out[bh] (if not NULL) <- the total, zero padded.
 cudaError_t launch_state_scan(float* W, float* state_out, int BH, int NG, int64_t stride, int64_t used,
-                              cudaStream_t stream);
+                              cudaStream_t stream, bool pdl = false);
+
+// Launches `kernel` with programmatic stream serialisation when pdl is set,
+// so that it may start while the previous kernel in the stream finishes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 template <typename Tin>
 cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "feature_table.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace ta {
 
@@ -107,11 +108,15 @@ group_state_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, float* 
 // running sum is the state after every group; elements past F*(d_v+1) (the
 // padding, never written by the producers) are written as zeros there.
 constexpr int kScanThreads = 128;
-constexpr int kScanRun = 32;
+constexpr int kScanRun = 16;
 
-__global__ void __launch_bounds__(kScanThreads)
+__global__ void __launch_bounds__(kScanThreads, 4)
 scan_kernel(float* __restrict__ W, float* __restrict__ state_out, int NG, int64_t stride,
             int64_t used) {
+    // the group states come from the previous kernel; the next one may start
+    // its independent work as soon as this grid is resident
+    ptx::pdl_wait_primary();
+    ptx::pdl_launch_dependents();
     const int bh = blockIdx.y;
     const int64_t e4 = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
     const int64_t s4 = stride / 4;
@@ -363,10 +368,12 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
 }
 
 cudaError_t launch_state_scan(float* W, float* state_out, int BH, int NG, int64_t stride, int64_t used,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, bool pdl) {
     const dim3 g((unsigned)((stride / 4 + kScanThreads - 1) / kScanThreads), BH);
-    TA_TIMED(stream, "scan_kernel", scan_kernel<<<g, kScanThreads, 0, stream>>>(W, state_out, NG, stride, used));
-    return cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    TA_TIMED(stream, "scan_kernel",
+             e = launch_maybe_pdl(scan_kernel, g, dim3(kScanThreads), 0, stream, pdl, W, state_out, NG, stride, used));
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template cudaError_t launch_prefill_cc<float>(const float*, const float*, const float*, float*, float*,

@@ -29,6 +29,7 @@
 #include "feature_table.cuh"
 #include "internal.h"
 #include "prefill_tc.h"
+#include "phase.cuh"
 #include "ptx.cuh"
 #include "tcgen05.cuh"
 
@@ -150,6 +151,7 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
     float* sOut = reinterpret_cast<float*>(sm + kOffBh);  // reused once the MMAs are done
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    TA_PHASE(0, 0, tid == 0);
     const int c = blockIdx.x, bh = blockIdx.y;
     const int64_t t0 = (int64_t)c * kC;
     const int nv = (int)min64(kC, (int64_t)N - t0);
@@ -200,6 +202,8 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = tslot;
+    TA_PHASE(0, 1, tid == 0);
+    ptx::pdl_launch_dependents();
 
     if (tid == 0) {
         const uint32_t id = idesc_bf16(128, kFP, 1, 1);
@@ -213,6 +217,7 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
     }
     const bool ok = wait_all(&mb, 0);
     fence_after_sync();
+    TA_PHASE(0, 2, tid == 0);
     const uint32_t bytes = (uint32_t)(((int64_t)F * (kDV + 1) * 4 + 15) / 16 * 16);
     if (ok) {
         // warps 0,1 (+4,5) hold S_v columns 0..63 on their lanes; warp 2 lane 0
@@ -222,19 +227,26 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
             const int col = wq * 32 + lane;
             const uint32_t ta = tbase + ((uint32_t)(wq * 32) << 16);
             const int fb = half * 80;
+            float r[5][16];
 #pragma unroll
-            for (int part = 0; part < 5; ++part) {
-                float r[16];
-                tmem_ld16(ta + fb + part * 16, r);
-                tmem_ld_wait();
+            for (int part = 0; part < 5; ++part) tmem_ld16(ta + fb + part * 16, r[part]);
+            tmem_ld_wait();
+            if (col < kDV) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int f = fb + part * 16 + i;
-                    if (f < F) {
-                        if (col < kDV) sOut[f * kDV + col] = r[i];
-                        else if (col == kDV) sOut[F * kDV + f] = r[i];
+                for (int part = 0; part < 5; ++part)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int f = fb + part * 16 + i;
+                        if (f < F) sOut[f * kDV + col] = r[part][i];
                     }
-                }
+            } else if (col == kDV) {
+#pragma unroll
+                for (int part = 0; part < 5; ++part)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int f = fb + part * 16 + i;
+                        if (f < F) sOut[F * kDV + f] = r[part][i];
+                    }
             }
         }
         if (tid < 4) sOut[F * (kDV + 1) + tid] = 0.f;  // tail of the last 16-byte unit
@@ -245,11 +257,13 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
     if (!ok) ptx::mbar_wait(&mb, 0, kWaitPolls);
     fence_before_sync();
     __syncthreads();
+    TA_PHASE(0, 3, tid == 0);
     if (ok && tid == 0) {
         ptx::bulk_s2g(W + ((int64_t)bh * NC + c) * stride, sOut, bytes);
         ptx::bulk_commit();
         ptx::bulk_wait_read_all();
     }
+    TA_PHASE(0, 4, tid == 0);
     if (warp == 0) {
         fence_after_sync();
         tmem_dealloc(tbase, 256);
@@ -257,21 +271,20 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
 }
 
 // ---------------------------------------------------------------- 3. chunk outputs
-// Warps 0-7 stage operands, build Phi_Q, S_<c and P, and run the epilogue;
+// Warps 0-7 stage operands, build Phi_Q, P and S_<c, and run the epilogue;
 // warp 8 allocates TMEM and issues every MMA, driven by mbarriers that the
-// other warps arrive on, so no warp waits for the MMA issue itself.
+// other warps arrive on.  Everything that does not depend on the carried
+// state (the pairwise part and Phi_Q) comes first, so that with programmatic
+// dependent launch it overlaps the scan that produces S_<c.
 constexpr int kOutThreads = kThreads + 32;
-
-__device__ __forceinline__ void compute_bar_sync() {
-    asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");
-}
+constexpr int kSUnits = kFP * 8 / kThreads;  // 8-column units of S_v per thread (5)
 
 __global__ void __launch_bounds__(kOutThreads, 1)
 tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                     const float* __restrict__ W, float* __restrict__ out, int N, int n, float tau, int F,
                     int64_t stride, int NC, unsigned int* __restrict__ err) {
     extern __shared__ __align__(1024) uint8_t sm[];
-    __shared__ __align__(8) uint64_t mb_ld, mb_s, mb_o, bar_qk, bar_ops, bar_p;
+    __shared__ __align__(8) uint64_t mb_s, mb_o, bar_qk, bar_p, bar_ops;
     __shared__ uint32_t tslot;
     __shared__ int mma_fail;
     uint8_t* sQ = sm + kOffQ;
@@ -283,24 +296,21 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     uint8_t* sQl = sm + kOffQl;
     uint8_t* sSh = sm + kOffSh;
     uint8_t* sSl = sm + kOffSl;
-    // the carried state arrives as fp32 in the P buffers, which are free
-    // until the pairwise weights are written
-    const float* sS32 = reinterpret_cast<const float*>(sPh);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, bh = blockIdx.y;
     const int64_t t0 = (int64_t)c * kC;
     const int nv = (int)min64(kC, (int64_t)N - t0);
     const bool inter = c > 0;
-    const uint32_t sbytes = (uint32_t)(((int64_t)F * (kDV + 1) * 4 + 15) / 16 * 16);
+    TA_PHASE(1, 0, tid == 0);
+    TA_PHASE(2, warp, lane == 0);
 
     if (tid == 0) {
-        ptx::mbar_init(&mb_ld, 1);
         ptx::mbar_init(&mb_s, 1);
         ptx::mbar_init(&mb_o, 1);
         ptx::mbar_init(&bar_qk, kThreads);
-        ptx::mbar_init(&bar_ops, kThreads);
         ptx::mbar_init(&bar_p, kThreads);
+        ptx::mbar_init(&bar_ops, kThreads);
         mma_fail = 0;
         ptx::fence_mbar_init();
     }
@@ -314,23 +324,34 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     const uint32_t tbase = tslot;
     const uint32_t tA = tbase;          // scores, columns [0, 128)
     const uint32_t tO = tbase + 128;    // [numerator | denominator], columns [128, 208)
+    TA_PHASE(1, 1, tid == 0);
 
     if (warp == 8) {
         // ------------------------------------------------ MMA issue (one thread)
         if (lane == 0) {
-            if (inter) {
-                ptx::mbar_arrive_expect_tx(&mb_ld, sbytes);
-                ptx::bulk_g2s(sPh, W + ((int64_t)bh * NC + c) * stride, sbytes, &mb_ld);
-            }
+            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
             bool good = ptx::mbar_wait(&bar_qk, 0, kWaitPolls);
             fence_after_sync();
             if (good)
                 mma_bf16(tA, smem_desc(sQ, 128, kSboQK), smem_desc(sK, 128, kSboQK), idesc_bf16(128, 128, 0, 0), 0u);
             mma_commit(&mb_s);
-            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
-            if (inter && good) {
+            if (good) {
+                good = ptx::mbar_wait(&bar_p, 0, kWaitPolls);
+                fence_after_sync();
+                TA_PHASE(1, 11, true);
+                if (good) {
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks) {
+                        const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
+                        mma_bf16(tO, smem_desc(sPh + ks * 256, 128, kSboP), b, id, ks > 0 ? 1u : 0u);
+                        mma_bf16(tO, smem_desc(sPl + ks * 256, 128, kSboP), b, id, 1u);
+                    }
+                }
+            }
+            if (good && inter) {
                 good = ptx::mbar_wait(&bar_ops, 0, kWaitPolls);
                 fence_after_sync();
+                TA_PHASE(1, 12, true);
                 if (good) {
 #pragma unroll
                     for (int ks = 0; ks < kFP / 16; ++ks) {
@@ -338,21 +359,9 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
                         const uint64_t al = smem_desc(sQl + ks * 256, 128, kSboPhiQ);
                         const uint64_t bh_ = smem_desc(sSh + ks * 2 * kLboS, kLboS, 128);
                         const uint64_t bl_ = smem_desc(sSl + ks * 2 * kLboS, kLboS, 128);
-                        mma_bf16(tO, ah, bh_, id, ks > 0 ? 1u : 0u);
+                        mma_bf16(tO, ah, bh_, id, 1u);
                         mma_bf16(tO, ah, bl_, id, 1u);
                         mma_bf16(tO, al, bh_, id, 1u);
-                    }
-                }
-            }
-            if (good) {
-                good = ptx::mbar_wait(&bar_p, 0, kWaitPolls);
-                fence_after_sync();
-                if (good) {
-#pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks) {
-                        const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
-                        mma_bf16(tO, smem_desc(sPh + ks * 256, 128, kSboP), b, id, (inter || ks > 0) ? 1u : 0u);
-                        mma_bf16(tO, smem_desc(sPl + ks * 256, 128, kSboP), b, id, 1u);
                     }
                 }
             }
@@ -361,6 +370,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
                 atomicOr(err, kErrPrefillPipe);
             }
             mma_commit(&mb_o);  // tracks every MMA issued, also on the error path
+            TA_PHASE(1, 13, true);
         }
     } else {
         // ------------------------------------------------ operands and epilogue
@@ -399,10 +409,10 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
         for (int g = 0; g < 4; ++g) *reinterpret_cast<uint4*>(sV1 + mnmaj(row, half * 4 + g, kLboV1)) = val[g];
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&bar_qk);
+        TA_PHASE(1, 2, tid == 0);
 
-        bool ok = true;
+        // half of Phi_Q for token `row` while the scores are computed
         if (inter) {
-            // half of Phi_Q for token `row`, while S_<c is in flight
             float x[16];
             const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
@@ -417,44 +427,13 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
             };
             if (half == 0) phi16_groups<0, 10>(x, valid ? 1.f : 0.f, e1, e2, put);
             else phi16_groups<10, 20>(x, valid ? 1.f : 0.f, e1, e2, put);
-            // S_<c from fp32 to hi/lo, MN-major [K=160][80]
-            ok = ptx::mbar_wait(&mb_ld, 0, kWaitPolls);
-            if (ok) {
-                for (int u = tid; u < kFP * 8; u += kThreads) {
-                    const int f = u >> 3, g = u & 7;
-                    float xs[8];
-                    if (f < F) {
-                        const float4 a = reinterpret_cast<const float4*>(sS32 + f * kDV + g * 8)[0];
-                        const float4 b = reinterpret_cast<const float4*>(sS32 + f * kDV + g * 8)[1];
-                        xs[0] = a.x; xs[1] = a.y; xs[2] = a.z; xs[3] = a.w;
-                        xs[4] = b.x; xs[5] = b.y; xs[6] = b.z; xs[7] = b.w;
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) xs[i] = 0.f;
-                    }
-                    uint4 hi, lo;
-                    split8(xs, hi, lo);
-                    *reinterpret_cast<uint4*>(sSh + mnmaj(f, g, kLboS)) = hi;
-                    *reinterpret_cast<uint4*>(sSl + mnmaj(f, g, kLboS)) = lo;
-                }
-                for (int f = tid; f < kFP; f += kThreads) {
-                    float xs[8] = {f < F ? sS32[F * kDV + f] : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    uint4 hi, lo;
-                    split8(xs, hi, lo);
-                    *reinterpret_cast<uint4*>(sSh + mnmaj(f, 8, kLboS)) = hi;
-                    *reinterpret_cast<uint4*>(sSl + mnmaj(f, 8, kLboS)) = lo;
-                    *reinterpret_cast<uint4*>(sSh + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(sSl + mnmaj(f, 9, kLboS)) = make_uint4(0, 0, 0, 0);
-                }
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(&bar_ops);
-            compute_bar_sync();  // every read of the staged fp32 S precedes the P writes below
         }
+        TA_PHASE(1, 3, tid == 0);
 
         // pairwise weights P = poly(tau q.k) under the causal mask, hi/lo, K-major
-        ok = ptx::mbar_wait(&mb_s, 0, kWaitPolls) && ok;
+        bool ok = ptx::mbar_wait(&mb_s, 0, kWaitPolls);
         fence_after_sync();
+        TA_PHASE(1, 4, tid == 0);
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         {
             float s0[32], s1[32];
@@ -485,10 +464,52 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
         ptx::fence_proxy_async_smem();
         fence_before_sync();
         ptx::mbar_arrive(&bar_p);
+        TA_PHASE(1, 5, tid == 0);
 
-        // epilogue: o = numerator / denominator
+        // the carried state S_<c: produced by the previous grid
+        if (inter) {
+            ptx::pdl_wait_primary();
+            TA_PHASE(1, 6, tid == 0);
+            const float* Sg = W + ((int64_t)bh * NC + c) * stride;
+            float4 sa[kSUnits], sb[kSUnits];
+#pragma unroll
+            for (int i = 0; i < kSUnits; ++i) {
+                const int u = tid + i * kThreads, f = u >> 3, g = u & 7;
+                if (f < F) {
+                    sa[i] = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8));
+                    sb[i] = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8) + 1);
+                } else {
+                    sa[i] = sb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            const float zf = (tid < kFP && tid < F) ? __ldg(Sg + (int64_t)F * kDV + tid) : 0.f;
+#pragma unroll
+            for (int i = 0; i < kSUnits; ++i) {
+                const int u = tid + i * kThreads, f = u >> 3, g = u & 7;
+                const float xs[8] = {sa[i].x, sa[i].y, sa[i].z, sa[i].w, sb[i].x, sb[i].y, sb[i].z, sb[i].w};
+                uint4 hi, lo;
+                split8(xs, hi, lo);
+                *reinterpret_cast<uint4*>(sSh + mnmaj(f, g, kLboS)) = hi;
+                *reinterpret_cast<uint4*>(sSl + mnmaj(f, g, kLboS)) = lo;
+            }
+            if (tid < kFP) {
+                const float xs[8] = {zf, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                uint4 hi, lo;
+                split8(xs, hi, lo);
+                *reinterpret_cast<uint4*>(sSh + mnmaj(tid, 8, kLboS)) = hi;
+                *reinterpret_cast<uint4*>(sSl + mnmaj(tid, 8, kLboS)) = lo;
+                *reinterpret_cast<uint4*>(sSh + mnmaj(tid, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(sSl + mnmaj(tid, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&bar_ops);
+            TA_PHASE(1, 7, tid == 0);
+        }
+
+        // epilogue: o = numerator * (1 / denominator)
         const bool done = ptx::mbar_wait(&mb_o, 0, kWaitPolls);
         fence_after_sync();
+        TA_PHASE(1, 8, tid == 0);
         ok = ok && done && mma_fail == 0;
         if (ok) {
             float o[32], dn[16];
@@ -496,17 +517,17 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
             tmem_ld16(tO + lane_off + kDV, dn);
             tmem_ld_wait();
             if (valid) {
-                const float den = dn[0];
+                const float r = __frcp_rn(dn[0]);
                 float4* dst = reinterpret_cast<float4*>(out + tok * kDV + half * 32);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    dst[i] = make_float4(o[4 * i] / den, o[4 * i + 1] / den, o[4 * i + 2] / den,
-                                         o[4 * i + 3] / den);
+                    dst[i] = make_float4(o[4 * i] * r, o[4 * i + 1] * r, o[4 * i + 2] * r, o[4 * i + 3] * r);
             }
         } else {
             if (tid == 0) atomicOr(err, kErrPrefillPipe);
             if (!done) ptx::mbar_wait(&mb_o, 0, kWaitPolls);  // one more bound for MMAs in flight
         }
+        TA_PHASE(1, 9, tid == 0);
     }
     fence_before_sync();
     __syncthreads();
@@ -514,6 +535,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
         fence_after_sync();
         tmem_dealloc(tbase, 256);
     }
+    TA_PHASE(1, 14, tid == 0);
 }
 
 constexpr int kMaxDevices = 64;
@@ -559,12 +581,12 @@ int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloa
     TA_TIMED(stream, "tc_chunk_state_kernel",
              tc_chunk_state_kernel<<<grid, kThreads, kSmemState, stream>>>(k, v, W, N, n, (int)F, stride, NC, err));
     e = cudaGetLastError();
-    if (e == cudaSuccess) e = launch_state_scan(W, state_out, BH, NC, stride, F * (dv + 1), stream);
+    if (e == cudaSuccess) e = launch_state_scan(W, state_out, BH, NC, stride, F * (dv + 1), stream, true);
     if (e == cudaSuccess) {
         TA_TIMED(stream, "tc_chunk_out_kernel",
-                 tc_chunk_out_kernel<<<grid, kOutThreads, kSmemOut, stream>>>(q, k, v, W, out, N, n, tau, (int)F,
-                                                                           stride, NC, err));
-        e = cudaGetLastError();
+                 e = launch_maybe_pdl(tc_chunk_out_kernel, grid, dim3(kOutThreads), kSmemOut, stream, true, q, k, v,
+                                      W, out, N, n, tau, (int)F, stride, NC, err));
+        if (e == cudaSuccess) e = cudaGetLastError();
     }
     const cudaError_t e2 = workspace_free(W, stream);
     if (e == cudaSuccess) e = e2;
