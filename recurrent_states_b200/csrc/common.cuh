@@ -134,6 +134,9 @@ __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p) {
     return __bfloat162float(*p);
 }
 
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+
 // sum_{m<n} x^m/m! by Horner: 1 + x(1 + x/2(1 + x/3(...))).
 __device__ __forceinline__ float taylor_kernel(float x, int n) {
     float w = 1.0f;

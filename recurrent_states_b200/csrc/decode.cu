@@ -5,16 +5,16 @@
 // The step is bound by HBM: each head's fp32 state (F*(d_v+1) floats) is read
 // once and written once.  One CTA per head.
 //
-// Main path (d_v in {16, 32, 64, 128}, state <= 110 KB): one thread issues a
-// single bulk (TMA) copy of the head's state into shared memory, completing
-// on an mbarrier, while the block evaluates phi(q), phi(k) from the static
-// feature table.  The block then updates the state in shared memory with
-// 128-bit accesses (each thread owns one 16-byte column group of the rows it
-// visits), accumulates the read-out, and one thread streams the state back
-// with a bulk store.  No state element passes through registers for longer
-// than one update, so occupancy is set by shared memory (5 CTAs per SM at
-// d_k 16, d_v 64, n 3) and every CTA's whole state is in flight at once.
-// The read-out sum over rows is a warp-shuffle plus shared-memory reduction.
+// Main path (d_v in {16, 32, 64, 128}, state <= 110 KB, F <= 1024): at entry
+// one thread issues bulk (TMA) copies of the head's state into shared memory,
+// completing on an mbarrier, while every thread loads the new token and its
+// feature descriptors, so the three latencies overlap.  After phi(q), phi(k)
+// are evaluated and the state has landed, each thread updates the rows it
+// owns (one 16-byte column group per row, 128-bit shared loads) and writes
+// them straight back to HBM with 128-bit stores that nothing waits for.  No
+// state element stays in registers for longer than one update, so occupancy
+// is set by shared memory (5 CTAs per SM at d_k 16, d_v 64, n 3).  The
+// read-out sum over rows is a warp-shuffle plus shared-memory reduction.
 //
 // Fallback path (other d_v or larger states): the same arithmetic with
 // register-staged 128-bit loads and stores, one feature tile at a time.
@@ -23,6 +23,7 @@
 #include "common.cuh"
 #include "feature_table.cuh"
 #include "internal.h"
+#include "phase.cuh"
 #include "ptx.cuh"
 
 namespace ta {
@@ -33,6 +34,13 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr uint32_t kWaitPolls = 1u << 22;  // bound on mbarrier polls (seconds of wall time)
 constexpr int kTmaMaxBytes = 110 * 1024;
+constexpr int kTmaMaxFeatures = 1024;     // feature descriptors held in registers: 4 per thread
+constexpr int kDescPerThread = kTmaMaxFeatures / 256;
+#ifndef TA_DECODE_LOAD_PIECES
+#define TA_DECODE_LOAD_PIECES 1
+#endif
+constexpr int kLoadPieces = TA_DECODE_LOAD_PIECES;     // bulk copies per state load
+constexpr int kMaxDevices = 64;
 
 template <typename Tin, int DV4>
 __global__ void __launch_bounds__(kThreads, 5)
@@ -55,41 +63,71 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     const int bh = blockIdx.x;
     const int tid = threadIdx.x;
     float* gS = state + (int64_t)bh * stride;
+    TA_PHASE(3, 0, tid == 0);
 
+    // Everything this head needs is requested at once: the state (bulk copy,
+    // one thread), the new token and this thread's feature descriptors
+    // (plain loads), so their latencies overlap instead of adding up.
     if (tid == 0) {
         ptx::mbar_init(&bar, 1);
         ptx::fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
         ptx::mbar_arrive_expect_tx(&bar, bytes);
-        ptx::bulk_g2s(S, gS, bytes, &bar);
+        const uint32_t piece = ((bytes + kLoadPieces - 1) / kLoadPieces + 15u) & ~15u;
+        for (uint32_t o = 0; o < bytes; o += piece) {
+            const uint32_t sz = bytes - o < piece ? bytes - o : piece;
+            ptx::bulk_g2s(reinterpret_cast<unsigned char*>(S) + o, reinterpret_cast<const unsigned char*>(gS) + o, sz,
+                          &bar);
+        }
     }
-    // while the state streams in: the new token and the feature map
-    if (tid < d) {
-        xq[tid] = ldf(q + (int64_t)bh * d + tid);
-        xk[tid] = ldf(k + (int64_t)bh * d + tid);
-    }
-    if (tid < DV) vv[tid] = ldf(v + (int64_t)bh * DV + tid);
-    if (tid < n) qc[tid] = query_coeff(tid, tau);
-    __syncthreads();
     const PackedFeat* tab = feat_table(d, n);
-    for (int f = tid; f < F; f += kThreads) {
-        pk[f] = eval_desc(get_desc(tab, d, n, f, tau, qc, false), xk);
-        pq[f] = eval_desc(get_desc(tab, d, n, f, tau, qc, true), xq);
+    PackedFeat pf[kDescPerThread];
+#pragma unroll
+    for (int j = 0; j < kDescPerThread; ++j) {
+        const int f = tid + j * kThreads;
+        if (tab && f < F) pf[j] = tab[f];
     }
+    float aq = 0.f, ak = 0.f, av = 0.f;
+    if (tid < d) {
+        aq = ldf(q + (int64_t)bh * d + tid);
+        ak = ldf(k + (int64_t)bh * d + tid);
+    }
+    if (tid < DV) av = ldf(v + (int64_t)bh * DV + tid);
+    if (tid < d) {
+        xq[tid] = aq;
+        xk[tid] = ak;
+    }
+    if (tid < DV) vv[tid] = av;
+    if (tid < n) qc[tid] = query_coeff(tid, tau);
+    TA_PHASE(3, 1, tid == 0);
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kDescPerThread; ++j) {
+        const int f = tid + j * kThreads;
+        if (f < F) {
+            const FeatDesc dk = tab ? desc_from_packed(pf[j], qc, false) : make_desc(d, n, f, tau, false);
+            const FeatDesc dq = tab ? desc_from_packed(pf[j], qc, true) : make_desc(d, n, f, tau, true);
+            pk[f] = eval_desc(dk, xk);
+            pq[f] = eval_desc(dq, xq);
+        }
+    }
+    TA_PHASE(3, 2, tid == 0);
     // every thread observes the copy's completion itself; the block agrees
     // on the outcome so that a timeout leaves as one
     const bool landed = ptx::mbar_wait(&bar, 0, kWaitPolls);
+    TA_PHASE(3, 7, tid == 0);
     if (!__syncthreads_and(landed)) {
         if (tid == 0) atomicOr(err, kErrDecodeLoad);
         if (!landed) ptx::mbar_wait(&bar, 0, kWaitPolls);  // one more bound for the copy in flight
         return;
     }
 
+    TA_PHASE(3, 3, tid == 0);
+    // each updated row leaves straight from registers: a warp stores 512
+    // contiguous bytes per instruction, and nothing waits for the stores
     const int cg = tid % DV4, rs = tid / DV4;
     const float4 v4 = reinterpret_cast<const float4*>(vv)[cg];
-    float4* S4 = reinterpret_cast<float4*>(S);
+    const float4* S4 = reinterpret_cast<const float4*>(S);
+    float4* G4 = reinterpret_cast<float4*>(gS);
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int r = rs; r < F; r += RS) {
@@ -99,25 +137,21 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
         s.y = fmaf(a, v4.y, s.y);
         s.z = fmaf(a, v4.z, s.z);
         s.w = fmaf(a, v4.w, s.w);
-        S4[r * DV4 + cg] = s;
+        G4[r * DV4 + cg] = s;
         y.x = fmaf(b, s.x, y.x);
         y.y = fmaf(b, s.y, y.y);
         y.z = fmaf(b, s.z, y.z);
         y.w = fmaf(b, s.w, y.w);
     }
     float yz = 0.f;
-    float* Z = S + F * DV;
+    const float* Z = S + F * DV;
+    float* GZ = gS + (int64_t)F * DV;
     for (int f = tid; f < F; f += kThreads) {
         const float z = Z[f] + pk[f];
-        Z[f] = z;
+        GZ[f] = z;
         yz = fmaf(pq[f], z, yz);
     }
-    ptx::fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        ptx::bulk_s2g(gS, S, bytes);
-        ptx::bulk_commit();
-    }
+    TA_PHASE(3, 4, tid == 0);
 
     // read-out: lanes sharing a column group sit DV4 apart inside a warp
 #pragma unroll
@@ -144,7 +178,8 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
         }
         out[(int64_t)bh * DV + tid] = acc / den;
     }
-    if (tid == 0) ptx::bulk_wait_read_all();
+    TA_PHASE(3, 5, tid == 0);
+    TA_PHASE(3, 6, tid == 0);
 }
 
 constexpr int kFeatTile = 1024;  // features whose phi(q), phi(k) sit in smem at once
@@ -242,8 +277,6 @@ decode_generic_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
     }
 }
 
-constexpr int kMaxDevices = 64;
-
 template <typename Tin, int DV4>
 cudaError_t launch_tma(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
                        int n, float tau, int F, int64_t stride, uint32_t bytes, size_t dyn,
@@ -276,7 +309,8 @@ cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state
     const uint32_t bytes = (uint32_t)((used_bytes + 15) / 16 * 16);
     const size_t dyn = ((bytes + 127u) & ~127u) + 2 * (size_t)((F + 3) & ~3) * 4;
     unsigned int* err = device_error_word();
-    const bool tma_ok = err != nullptr && used_bytes <= kTmaMaxBytes && dyn <= (size_t)kTmaMaxBytes + 8192;
+    const bool tma_ok = err != nullptr && used_bytes <= kTmaMaxBytes && dyn <= (size_t)kTmaMaxBytes + 8192 &&
+                        F <= kTmaMaxFeatures;
     if (tma_ok) {
         switch (dv) {
             case 16: return launch_tma<Tin, 4>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn, err, stream);
