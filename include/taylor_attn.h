@@ -114,6 +114,25 @@ TAYLOR_API int taylor_attn_prefill_f32(const float* q, const float* k, const flo
                             float* state_out, int B, int H, int N, int d_k, int d_v, int n,
                             float tau, cudaStream_t stream);
 
+/* Causal prefill that continues a sequence from a carried state: tokens
+ * 0..N-1 here are positions P..P+N-1 of a sequence whose first P tokens
+ * produced state_in [B][H][stride] (by a prefill, decodes or merges).  Each
+ * output attends to the carried prefix through state_in and to the new
+ * tokens as taylor_attn_prefill does; state_out (may be NULL, may alias
+ * state_in) receives state_in plus the new tokens' state (abstract: states
+ * are additive across chunks, so prefill can resume from a chunk boundary).
+ * q, k, v bf16; workspace and errors as taylor_attn_prefill. */
+TAYLOR_API int taylor_attn_prefill_from_state(const void* q, const void* k, const void* v,
+                                              const float* state_in, float* out, float* state_out,
+                                              int B, int H, int N, int d_k, int d_v, int n, float tau,
+                                              cudaStream_t stream);
+
+/* taylor_attn_prefill_from_state with fp32 q, k, v (CUDA-core fp32 path). */
+TAYLOR_API int taylor_attn_prefill_from_state_f32(const float* q, const float* k, const float* v,
+                                                  const float* state_in, float* out, float* state_out,
+                                                  int B, int H, int N, int d_k, int d_v, int n,
+                                                  float tau, cudaStream_t stream);
+
 /* Returns the prefill workspace cached in the current device's pool to the
  * driver (synchronises the device first). */
 TAYLOR_API int taylor_attn_release_workspace(void);
@@ -166,8 +185,14 @@ TAYLOR_API int64_t taylor_attn_prefill_noalloc_scratch_floats(void);
  * for the current device (a synchronous device-to-host copy that waits for
  * all prior work), stores it in *flags, clears it when clear != 0, and
  * returns TAYLOR_ERR_TIMEOUT if any bit was set, else TAYLOR_OK.
- * Bits: 1 = decode state load, 2 = decode state store, 4 = prefill pipeline. */
+ * Bits: 1 = decode state load, 2 = decode state store, 4 = prefill pipeline,
+ * 8 = taylor_attn_selftest_bounded_wait. */
 TAYLOR_API int taylor_attn_device_errors(int clear, unsigned int* flags);
+
+/* Exercises the timeout path on the device: one block waits on an mbarrier
+ * that nothing arrives on, gives up after `polls` polls (1 .. 2^20), sets bit
+ * 8 of the error word and returns; the context stays usable. */
+TAYLOR_API int taylor_attn_selftest_bounded_wait(unsigned int polls, cudaStream_t stream);
 
 /* Opt-in kernel timing, for benchmarks.  With on != 0, every kernel this
  * library launches from the calling host thread is bracketed by two CUDA

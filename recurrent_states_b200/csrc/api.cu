@@ -43,9 +43,9 @@ int num_sms() {
 }
 
 template <typename Tin>
-int prefill_impl(const Tin* q, const Tin* k, const Tin* v, float* out, float* state_out, int B,
-                 int H, int N, int d_k, int d_v, int n, float tau, cudaStream_t stream,
-                 bool allow_tc) {
+int prefill_impl(const Tin* q, const Tin* k, const Tin* v, const float* state_in, float* out,
+                 float* state_out, int B, int H, int N, int d_k, int d_v, int n, float tau,
+                 cudaStream_t stream, bool allow_tc) {
     if (B < 0 || H < 0 || N < 0) return TAYLOR_ERR_INVALID_ARG;
     int rc = check_dims(d_k, d_v, n);
     if (rc != TAYLOR_OK) return rc;
@@ -57,23 +57,26 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, float* out, float* st
     const int64_t F = ta::num_features(d_k, n);
     const int64_t stride = stride_of(d_k, d_v, n);
     if (state_out && !aligned16(state_out)) return TAYLOR_ERR_MISALIGNED;
+    if (state_in && !aligned16(state_in)) return TAYLOR_ERR_MISALIGNED;
     if (N == 0) {
-        if (state_out)
-            return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)BH * stride * sizeof(float), stream));
-        return TAYLOR_OK;
+        if (!state_out) return TAYLOR_OK;
+        const size_t bytes = (size_t)BH * stride * sizeof(float);
+        if (!state_in) return cuda_status(cudaMemsetAsync(state_out, 0, bytes, stream));
+        if (state_in == state_out) return TAYLOR_OK;
+        return cuda_status(cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, stream));
     }
     if (!q || !k || !v || !out) return TAYLOR_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TAYLOR_ERR_MISALIGNED;
 
     if (allow_tc) {
-        const int tc = ta::tc::try_prefill(q, k, v, out, state_out, (int)BH, N, d_k, d_v, n, tau, F,
+        const int tc = ta::tc::try_prefill(q, k, v, out, state_in, state_out, (int)BH, N, d_k, d_v, n, tau, F,
                                            stride, stream);
         if (tc != ta::tc::kNotApplicable) return tc;
     }
 
     const ta::CcPlan plan = ta::plan_prefill_cc((int)BH, N, d_k, d_v, n, F, stride);
     float* ws = nullptr;
-    const bool need_ws = plan.NG > 1 || state_out != nullptr;
+    const bool need_ws = plan.NG > 1 || state_out != nullptr || state_in != nullptr;
     if (need_ws) {
         cudaError_t e = ta::workspace_alloc(reinterpret_cast<void**>(&ws), plan.ws_bytes, stream);
         if (e != cudaSuccess) {
@@ -81,8 +84,8 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, float* out, float* st
             return TAYLOR_ERR_OUT_OF_MEMORY;
         }
     }
-    cudaError_t e = ta::launch_prefill_cc(q, k, v, out, state_out, ws, plan, (int)BH, N, d_k, d_v,
-                                          n, tau, F, stride, stream);
+    cudaError_t e = ta::launch_prefill_cc(q, k, v, out, state_in, state_out, ws, plan, (int)BH, N, d_k,
+                                          d_v, n, tau, F, stride, stream);
     if (ws) {
         cudaError_t e2 = ta::workspace_free(ws, stream);
         if (e == cudaSuccess) e = e2;
@@ -167,13 +170,29 @@ int taylor_attn_prefill(const void* q, const void* k, const void* v, float* out,
                         int B, int H, int N, int d_k, int d_v, int n, float tau, cudaStream_t stream) {
     using bf = __nv_bfloat16;
     return prefill_impl(static_cast<const bf*>(q), static_cast<const bf*>(k), static_cast<const bf*>(v),
-                        out, state_out, B, H, N, d_k, d_v, n, tau, stream, true);
+                        nullptr, out, state_out, B, H, N, d_k, d_v, n, tau, stream, true);
+}
+
+int taylor_attn_prefill_from_state(const void* q, const void* k, const void* v, const float* state_in,
+                                   float* out, float* state_out, int B, int H, int N, int d_k, int d_v,
+                                   int n, float tau, cudaStream_t stream) {
+    using bf = __nv_bfloat16;
+    if (!state_in && B > 0 && H > 0) return TAYLOR_ERR_INVALID_ARG;
+    return prefill_impl(static_cast<const bf*>(q), static_cast<const bf*>(k), static_cast<const bf*>(v),
+                        state_in, out, state_out, B, H, N, d_k, d_v, n, tau, stream, true);
+}
+
+int taylor_attn_prefill_from_state_f32(const float* q, const float* k, const float* v, const float* state_in,
+                                       float* out, float* state_out, int B, int H, int N, int d_k, int d_v,
+                                       int n, float tau, cudaStream_t stream) {
+    if (!state_in && B > 0 && H > 0) return TAYLOR_ERR_INVALID_ARG;
+    return prefill_impl(q, k, v, state_in, out, state_out, B, H, N, d_k, d_v, n, tau, stream, false);
 }
 
 int taylor_attn_prefill_f32(const float* q, const float* k, const float* v, float* out,
                             float* state_out, int B, int H, int N, int d_k, int d_v, int n, float tau,
                             cudaStream_t stream) {
-    return prefill_impl(q, k, v, out, state_out, B, H, N, d_k, d_v, n, tau, stream, false);
+    return prefill_impl(q, k, v, nullptr, out, state_out, B, H, N, d_k, d_v, n, tau, stream, false);
 }
 
 int taylor_attn_decode(const void* q, const void* k, const void* v, float* state_inout, float* out,

@@ -6,6 +6,7 @@
 
 #include "../../include/taylor_attn.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace {
 
@@ -37,6 +38,31 @@ unsigned int* device_error_word() {
 }
 
 }  // namespace ta
+
+namespace {
+
+// Waits on an mbarrier that nothing ever arrives on: the bounded wait must run
+// out, set its bit and return.
+__global__ void selftest_wait_kernel(unsigned int polls, unsigned int* err) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        ta::ptx::mbar_init(&bar, 1);
+        ta::ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    const bool done = ta::ptx::mbar_wait(&bar, 0, polls);
+    if (!done && threadIdx.x == 0) atomicOr(err, ta::kErrSelfTest);
+}
+
+}  // namespace
+
+extern "C" int taylor_attn_selftest_bounded_wait(unsigned int polls, cudaStream_t stream) {
+    if (polls == 0 || polls > (1u << 20)) return TAYLOR_ERR_INVALID_ARG;
+    unsigned int* err = ta::device_error_word();
+    if (!err) return TAYLOR_ERR_CUDA;
+    selftest_wait_kernel<<<1, 32, 0, stream>>>(polls, err);
+    return cudaGetLastError() == cudaSuccess ? TAYLOR_OK : TAYLOR_ERR_CUDA;
+}
 
 extern "C" int taylor_attn_device_errors(int clear, unsigned int* flags) {
     if (!flags) return TAYLOR_ERR_INVALID_ARG;

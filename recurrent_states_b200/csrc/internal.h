@@ -31,6 +31,7 @@ unsigned int* device_error_word();
 constexpr unsigned int kErrDecodeLoad = 1u;
 constexpr unsigned int kErrDecodeStore = 2u;
 constexpr unsigned int kErrPrefillPipe = 4u;
+constexpr unsigned int kErrSelfTest = 8u;
 
 template <typename Tin>
 cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state, float* out,
@@ -52,10 +53,11 @@ struct CcPlan {
 };
 CcPlan plan_prefill_cc(int BH, int N, int d, int dv, int n, int64_t F, int64_t stride);
 
-// In place: W[bh][g] <- sum_{g' < g} W[bh][g'] over the first `used` floats
-// of each state; state_out[bh] (if not NULL) <- the total, zero padded.
-cudaError_t launch_state_scan(float* W, float* state_out, int BH, int NG, int64_t stride, int64_t used,
-                              cudaStream_t stream, bool pdl = false);
+// In place: W[bh][g] <- state_in[bh] + sum_{g' < g} W[bh][g'] over the first
+// `used` floats of each state (state_in may be NULL: zero); state_out[bh]
+// (if not NULL) <- the total, zero padded.
+cudaError_t launch_state_scan(float* W, const float* state_in, float* state_out, int BH, int NG, int64_t stride,
+                              int64_t used, cudaStream_t stream, bool pdl = false);
 
 // Launches `kernel` with programmatic stream serialisation when pdl is set,
 // so that it may start while the previous kernel in the stream finishes.
@@ -77,8 +79,8 @@ cudaError_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 template <typename Tin>
 cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
-                              float* state_out, float* workspace, const CcPlan& plan, int BH,
-                              int N, int d, int dv, int n, float tau, int64_t F, int64_t stride,
-                              cudaStream_t stream);
+                              const float* state_in, float* state_out, float* workspace,
+                              const CcPlan& plan, int BH, int N, int d, int dv, int n, float tau,
+                              int64_t F, int64_t stride, cudaStream_t stream);
 
 }  // namespace ta

@@ -111,8 +111,8 @@ constexpr int kScanThreads = 128;
 constexpr int kScanRun = 16;
 
 __global__ void __launch_bounds__(kScanThreads, 4)
-scan_kernel(float* __restrict__ W, float* __restrict__ state_out, int NG, int64_t stride,
-            int64_t used) {
+scan_kernel(float* __restrict__ W, const float* __restrict__ state_in, float* __restrict__ state_out, int NG,
+            int64_t stride, int64_t used) {
     // the group states come from the previous kernel; the next one may start
     // its independent work as soon as this grid is resident
     ptx::pdl_wait_primary();
@@ -122,7 +122,17 @@ scan_kernel(float* __restrict__ W, float* __restrict__ state_out, int NG, int64_
     const int64_t s4 = stride / 4;
     if (e4 >= s4) return;
     float4* base = reinterpret_cast<float4*>(W + (int64_t)bh * NG * stride) + e4;
+    // the carried state the sequence continues from (zero for a fresh one);
+    // its padding is masked so that garbage there cannot leak into sums
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (state_in) {
+        run = reinterpret_cast<const float4*>(state_in + (int64_t)bh * stride)[e4];
+        const int64_t e = e4 * 4;
+        if (e + 0 >= used) run.x = 0.f;
+        if (e + 1 >= used) run.y = 0.f;
+        if (e + 2 >= used) run.z = 0.f;
+        if (e + 3 >= used) run.w = 0.f;
+    }
     for (int g0 = 0; g0 < NG; g0 += kScanRun) {
         float4 x[kScanRun];
 #pragma unroll
@@ -178,7 +188,7 @@ template <typename Tin>
 __global__ void __launch_bounds__(kThreads)
 chunk_out_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                  const float* __restrict__ W, float* __restrict__ out, int N, int d, int dv, int n,
-                 float tau, int G, int NG, int F, int64_t stride) {
+                 float tau, int G, int NG, int F, int64_t stride, int carried) {
     extern __shared__ float4 sm4[];
     float* sm = reinterpret_cast<float*>(sm4);
     const OutSmem L = out_smem_layout(d);
@@ -252,8 +262,9 @@ chunk_out_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             }
         }
 
-        // across groups, through the exclusive prefix state S_<g
-        if (g > 0) {
+        // across groups, through the exclusive prefix state S_<g (which holds
+        // the carried-in state when the sequence continues one)
+        if (g > 0 || carried) {
             const float* Sg = W + ((int64_t)bh * NG + g) * stride;
             for (int f0 = 0; f0 < F; f0 += kFTC) {
                 const int nf = min(kFTC, F - f0);
@@ -320,13 +331,13 @@ CcPlan plan_prefill_cc(int BH, int N, int d, int dv, int n, int64_t F, int64_t s
 
 template <typename Tin>
 cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
-                              float* state_out, float* W, const CcPlan& plan, int BH, int N,
-                              int d, int dv, int n, float tau, int64_t F, int64_t stride,
+                              const float* state_in, float* state_out, float* W, const CcPlan& plan,
+                              int BH, int N, int d, int dv, int n, float tau, int64_t F, int64_t stride,
                               cudaStream_t stream) {
     if (BH == 0 || N == 0) return cudaSuccess;
     cudaError_t e;
-    // a single group with no state requested needs neither A nor B
-    const bool need_states = plan.NG > 1 || state_out != nullptr;
+    // a single group with no state in or out needs neither A nor B
+    const bool need_states = plan.NG > 1 || state_out != nullptr || state_in != nullptr;
     if (need_states) {
     // A
     const int dv4 = dv / 4;
@@ -353,7 +364,7 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
     // B
     const dim3 gB((unsigned)((stride / 4 + kScanThreads - 1) / kScanThreads), BH);
     TA_TIMED(stream, "cc_scan_kernel",
-             scan_kernel<<<gB, kScanThreads, 0, stream>>>(W, state_out, plan.NG, stride, F * (dv + 1)));
+             scan_kernel<<<gB, kScanThreads, 0, stream>>>(W, state_in, state_out, plan.NG, stride, F * (dv + 1)));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // C
@@ -363,25 +374,26 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
     const dim3 gC((unsigned)((N + kC - 1) / kC), BH);
     TA_TIMED(stream, "cc_chunk_out_kernel",
              fc<<<gC, kThreads, L.total, stream>>>(q, k, v, W, out, N, d, dv, n, tau, plan.G, plan.NG,
-                                                   (int)F, stride));
+                                                   (int)F, stride, state_in != nullptr ? 1 : 0));
     return cudaGetLastError();
 }
 
-cudaError_t launch_state_scan(float* W, float* state_out, int BH, int NG, int64_t stride, int64_t used,
-                              cudaStream_t stream, bool pdl) {
+cudaError_t launch_state_scan(float* W, const float* state_in, float* state_out, int BH, int NG, int64_t stride,
+                              int64_t used, cudaStream_t stream, bool pdl) {
     const dim3 g((unsigned)((stride / 4 + kScanThreads - 1) / kScanThreads), BH);
     cudaError_t e = cudaSuccess;
     TA_TIMED(stream, "scan_kernel",
-             e = launch_maybe_pdl(scan_kernel, g, dim3(kScanThreads), 0, stream, pdl, W, state_out, NG, stride, used));
+             e = launch_maybe_pdl(scan_kernel, g, dim3(kScanThreads), 0, stream, pdl, W, state_in, state_out, NG,
+                                  stride, used));
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template cudaError_t launch_prefill_cc<float>(const float*, const float*, const float*, float*, float*,
-                                              float*, const CcPlan&, int, int, int, int, int, float,
+template cudaError_t launch_prefill_cc<float>(const float*, const float*, const float*, float*, const float*,
+                                              float*, float*, const CcPlan&, int, int, int, int, int, float,
                                               int64_t, int64_t, cudaStream_t);
 template cudaError_t launch_prefill_cc<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
-                                                      const __nv_bfloat16*, float*, float*, float*,
-                                                      const CcPlan&, int, int, int, int, int, float,
+                                                      const __nv_bfloat16*, float*, const float*, float*,
+                                                      float*, const CcPlan&, int, int, int, int, int, float,
                                                       int64_t, int64_t, cudaStream_t);
 
 }  // namespace ta

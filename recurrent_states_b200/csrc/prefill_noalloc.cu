@@ -92,7 +92,7 @@ extern "C" int taylor_attn_prefill_f32_noalloc(const float* q, const float* k, c
         cudaGetLastError();
         return TAYLOR_ERR_CUDA;
     }
-    const cudaError_t e = ta::launch_prefill_cc(q, k, v, out, state_out, scratch, plan, (int)BH, N, d_k,
-                                                d_v, n, tau, F, stride, stream);
+    const cudaError_t e = ta::launch_prefill_cc(q, k, v, out, nullptr, state_out, scratch, plan, (int)BH, N,
+                                                d_k, d_v, n, tau, F, stride, stream);
     return e == cudaSuccess ? TAYLOR_OK : TAYLOR_ERR_CUDA;
 }

@@ -282,7 +282,7 @@ constexpr int kSUnits = kFP * 8 / kThreads;  // 8-column units of S_v per thread
 __global__ void __launch_bounds__(kOutThreads, 1)
 tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                     const float* __restrict__ W, float* __restrict__ out, int N, int n, float tau, int F,
-                    int64_t stride, int NC, unsigned int* __restrict__ err) {
+                    int64_t stride, int NC, int carried, unsigned int* __restrict__ err) {
     extern __shared__ __align__(1024) uint8_t sm[];
     __shared__ __align__(8) uint64_t mb_s, mb_o, bar_qk, bar_p, bar_ops;
     __shared__ uint32_t tslot;
@@ -301,7 +301,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     const int c = blockIdx.x, bh = blockIdx.y;
     const int64_t t0 = (int64_t)c * kC;
     const int nv = (int)min64(kC, (int64_t)N - t0);
-    const bool inter = c > 0;
+    const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
     TA_PHASE(1, 0, tid == 0);
     TA_PHASE(2, warp, lane == 0);
 
@@ -554,8 +554,8 @@ cudaError_t set_smem_once(const void* fn, int bytes, std::once_flag* once, cudaE
 }  // namespace
 
 int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, float* out,
-                float* state_out, int BH, int N, int d, int dv, int n, float tau, int64_t F, int64_t stride,
-                cudaStream_t stream) {
+                const float* state_in, float* state_out, int BH, int N, int d, int dv, int n, float tau, int64_t F,
+                int64_t stride, cudaStream_t stream) {
     if (d != kD || dv != kDV || n > 3 || N <= 0 || BH <= 0) return kNotApplicable;
     unsigned int* err = device_error_word();
     if (!err) return TAYLOR_ERR_CUDA;
@@ -581,11 +581,11 @@ int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloa
     TA_TIMED(stream, "tc_chunk_state_kernel",
              tc_chunk_state_kernel<<<grid, kThreads, kSmemState, stream>>>(k, v, W, N, n, (int)F, stride, NC, err));
     e = cudaGetLastError();
-    if (e == cudaSuccess) e = launch_state_scan(W, state_out, BH, NC, stride, F * (dv + 1), stream, true);
+    if (e == cudaSuccess) e = launch_state_scan(W, state_in, state_out, BH, NC, stride, F * (dv + 1), stream, true);
     if (e == cudaSuccess) {
         TA_TIMED(stream, "tc_chunk_out_kernel",
                  e = launch_maybe_pdl(tc_chunk_out_kernel, grid, dim3(kOutThreads), kSmemOut, stream, true, q, k, v,
-                                      W, out, N, n, tau, (int)F, stride, NC, err));
+                                      W, out, N, n, tau, (int)F, stride, NC, state_in != nullptr ? 1 : 0, err));
         if (e == cudaSuccess) e = cudaGetLastError();
     }
     const cudaError_t e2 = workspace_free(W, stream);

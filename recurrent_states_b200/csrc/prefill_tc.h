@@ -13,12 +13,12 @@ namespace tc {
 constexpr int kNotApplicable = 1;
 
 int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, float* out,
-                float* state_out, int BH, int N, int d, int dv, int n, float tau, int64_t F,
-                int64_t stride, cudaStream_t stream);
+                const float* state_in, float* state_out, int BH, int N, int d, int dv, int n, float tau,
+                int64_t F, int64_t stride, cudaStream_t stream);
 
 // fp32 inputs never take the tensor-core path.
-inline int try_prefill(const float*, const float*, const float*, float*, float*, int, int, int, int,
-                       int, float, int64_t, int64_t, cudaStream_t) {
+inline int try_prefill(const float*, const float*, const float*, float*, const float*, float*, int, int, int,
+                       int, int, float, int64_t, int64_t, cudaStream_t) {
     return kNotApplicable;
 }
 

@@ -40,6 +40,8 @@ SIGNATURES = {
     "taylor_attn_feature_map": (_I, [_P, _P, _I64, _I, _I, _F, _I, _P]),
     "taylor_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_prefill_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "taylor_attn_prefill_from_state": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "taylor_attn_prefill_from_state_f32": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_decode_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_state_merge": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
@@ -47,6 +49,7 @@ SIGNATURES = {
     "taylor_attn_prefill_noalloc_scratch_floats": (_I64, []),
     "taylor_attn_device_errors": (_I, [_I, _P]),
     "taylor_attn_release_workspace": (_I, []),
+    "taylor_attn_selftest_bounded_wait": (_I, [ctypes.c_uint, _P]),
     "taylor_attn_timing_enable": (_I, [_I]),
     "taylor_attn_timing_read": (_I, [_I, _P, _P, _P]),
 }
@@ -193,6 +196,44 @@ def taylor_attn_prefill_f32(q, k, v, n: int, tau: float, out=None, state_out=Non
     return _prefill("taylor_attn_prefill_f32", q, k, v, n, tau, out, state_out, stream)
 
 
+def _prefill_from_state(name, q, k, v, state_in, n, tau, out, state_out, stream):
+    dtype = torch.bfloat16 if name == "taylor_attn_prefill_from_state" else torch.float32
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, H, N, d_k = q.shape
+    d_v = v.shape[-1]
+    stride = taylor_attn_state_stride(d_k, d_v, n)
+    _need(q, "q", dtype)
+    _need(k, "k", dtype, q.device, (B, H, N, d_k))
+    _need(v, "v", dtype, q.device, (B, H, N, d_v))
+    _need(state_in, "state_in", torch.float32, q.device, (B, H, stride))
+    if out is None:
+        out = torch.empty((B, H, N, d_v), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, q.device, (B, H, N, d_v))
+    if state_out is True:
+        state_out = torch.empty((B, H, stride), dtype=torch.float32, device=q.device)
+    if state_out is not None:
+        _need(state_out, "state_out", torch.float32, q.device, (B, H, stride))
+    rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(state_in), _ptr(out), _ptr(state_out), B, H, N,
+                              d_k, d_v, n, float(tau), _stream(stream))
+    _check(rc, name)
+    return out, state_out
+
+
+def taylor_attn_prefill_from_state(q, k, v, state_in, n: int, tau: float, out=None, state_out=None,
+                                   stream=None):
+    """Prefill continuing from a carried state [B, H, stride]; bf16 q, k, v.
+    ``state_out=True`` allocates the final state; it may also be ``state_in``."""
+    return _prefill_from_state("taylor_attn_prefill_from_state", q, k, v, state_in, n, tau, out, state_out,
+                               stream)
+
+
+def taylor_attn_prefill_from_state_f32(q, k, v, state_in, n: int, tau: float, out=None, state_out=None,
+                                       stream=None):
+    return _prefill_from_state("taylor_attn_prefill_from_state_f32", q, k, v, state_in, n, tau, out, state_out,
+                               stream)
+
+
 def taylor_attn_prefill_f32_noalloc(q, k, v, n: int, tau: float, out=None, state_out=None, stream=None):
     """taylor_attn_prefill_f32 without any device allocation inside the call:
     its scratch is a fixed array in the library (see the header).  The caller
@@ -253,6 +294,11 @@ def taylor_attn_state_merge(a, b, d_k: int, d_v: int, n: int, out=None, stream=N
 
 def taylor_attn_release_workspace() -> None:
     _check(lib().taylor_attn_release_workspace(), "taylor_attn_release_workspace")
+
+
+def taylor_attn_selftest_bounded_wait(polls: int = 1000, stream=None) -> None:
+    _check(lib().taylor_attn_selftest_bounded_wait(int(polls), _stream(stream)),
+           "taylor_attn_selftest_bounded_wait")
 
 
 def taylor_attn_device_errors(clear: bool = True) -> int:

@@ -262,6 +262,59 @@ def test_merge_and_split_prefill():
     assert torch.equal(sa2, merged)
 
 
+# ------------------------------------------------------------------ prefill from a carried state
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d,dv,n,N,cut", [(16, 64, 3, 1000, 384), (16, 64, 3, 700, 77), (16, 64, 3, 300, 1),
+                                          (16, 16, 3, 500, 256), (64, 64, 3, 600, 130), (16, 64, 5, 400, 200),
+                                          (7, 12, 2, 200, 33)])
+def test_prefill_from_state_continues_the_sequence(dtype, d, dv, n, N, cut):
+    """Prefill of the tail from the head's state equals the oracle's recursion
+    over the whole sequence (outputs of the tail, final state)."""
+    tau = 2.0
+    q, k, v = synth.qkv(2, 2, N, d, dv, seed=N + cut + n, dtype=dtype)
+    prefill = TA.taylor_attn_prefill if dtype == "bf16" else TA.taylor_attn_prefill_f32
+    cont = TA.taylor_attn_prefill_from_state if dtype == "bf16" else TA.taylor_attn_prefill_from_state_f32
+    h = lambda t: t[:, :, :cut].contiguous().to(DEV)  # noqa: E731
+    t_ = lambda t: t[:, :, cut:].contiguous().to(DEV)  # noqa: E731
+    _, st_head = prefill(h(q), h(k), h(v), n, tau, state_out=True)
+    out_tail, st = cont(t_(q), t_(k), t_(v), st_head, n, tau, state_out=True)
+    torch.cuda.synchronize()
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    assert row_scaled_max_err(f64(out_tail), ref_out[:, :, cut:]) <= TOL[dtype]
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL[dtype]
+    # in place: state_out aliasing state_in
+    st2 = st_head.clone()
+    cont(t_(q), t_(k), t_(v), st2, n, tau, state_out=st2)
+    torch.cuda.synchronize()
+    assert torch.equal(st2, st)
+
+
+def test_prefill_from_state_with_no_new_tokens_copies_the_state():
+    st = torch.randn((1, 2, TA.taylor_attn_state_stride(16, 64, 3)), device=DEV)
+    e = torch.empty((1, 2, 0, 16), dtype=torch.bfloat16, device=DEV)
+    ev = torch.empty((1, 2, 0, 64), dtype=torch.bfloat16, device=DEV)
+    _, st2 = TA.taylor_attn_prefill_from_state(e, e, ev, st, 3, 2.0, state_out=True)
+    torch.cuda.synchronize()
+    assert torch.equal(st2, st)
+
+
 def test_no_device_timeouts_recorded():
     """Every bounded wait in the runs above completed: the error word is clear."""
     assert TA.taylor_attn_device_errors(clear=True) == 0
+
+
+def test_bounded_wait_times_out_cleanly():
+    """A wait that nothing satisfies runs out, reports through the error word,
+    and leaves the context usable for the next call."""
+    assert TA.taylor_attn_device_errors(clear=True) == 0
+    TA.taylor_attn_selftest_bounded_wait(1000)
+    torch.cuda.synchronize()
+    flags = TA.taylor_attn_device_errors(clear=True)
+    assert flags == 8
+    assert TA.taylor_attn_device_errors(clear=True) == 0
+    # the device still computes correctly afterwards
+    q, k, v = synth.qkv(1, 1, 130, 16, 64, seed=3)
+    out, _ = _prefill("bf16", q, k, v, 3, 2.0, state=False)
+    ref, _ = C.recurrent(f64(q), f64(k), f64(v), 3, 2.0)
+    assert row_scaled_max_err(f64(out), ref) <= TOL["bf16"]
