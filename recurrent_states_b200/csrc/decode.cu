@@ -34,8 +34,13 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr uint32_t kWaitPolls = 1u << 22;  // bound on mbarrier polls (seconds of wall time)
 constexpr int kTmaMaxBytes = 110 * 1024;
-constexpr int kTmaMaxFeatures = 1024;     // feature descriptors held in registers: 4 per thread
-constexpr int kDescPerThread = kTmaMaxFeatures / 256;
+#ifndef TA_DECODE_THREADS
+#define TA_DECODE_THREADS 256
+#endif
+constexpr int kDecThreads = TA_DECODE_THREADS;   // threads of the main decode kernel
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kTmaMaxFeatures = 1024;
+constexpr int kDescPerThread = (kTmaMaxFeatures + kDecThreads - 1) / kDecThreads;
 #ifndef TA_DECODE_LOAD_PIECES
 #define TA_DECODE_LOAD_PIECES 1
 #endif
@@ -43,16 +48,16 @@ constexpr int kLoadPieces = TA_DECODE_LOAD_PIECES;     // bulk copies per state 
 constexpr int kMaxDevices = 64;
 
 template <typename Tin, int DV4>
-__global__ void __launch_bounds__(kThreads, 5)
+__global__ void __launch_bounds__(kDecThreads, kDecThreads == 256 ? 5 : 4)
 decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                   float* __restrict__ state, float* __restrict__ out, int d, int n, float tau, int F,
                   int64_t stride, uint32_t bytes, unsigned int* __restrict__ err) {
     constexpr int DV = DV4 * 4;
-    constexpr int RS = kThreads / DV4;  // row sets
+    constexpr int RS = kDecThreads / DV4;  // row sets
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ float xq[kMaxDk], xk[kMaxDk], vv[DV], qc[kMaxN];
-    __shared__ float4 red[kWarps][DV4];
-    __shared__ float zr[kWarps];
+    __shared__ float4 red[kDecWarps][DV4];
+    __shared__ float zr[kDecWarps];
     __shared__ __align__(8) uint64_t bar;
 
     float* S = reinterpret_cast<float*>(dsm);
@@ -83,7 +88,7 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     PackedFeat pf[kDescPerThread];
 #pragma unroll
     for (int j = 0; j < kDescPerThread; ++j) {
-        const int f = tid + j * kThreads;
+        const int f = tid + j * kDecThreads;
         if (tab && f < F) pf[j] = tab[f];
     }
     float aq = 0.f, ak = 0.f, av = 0.f;
@@ -102,7 +107,7 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < kDescPerThread; ++j) {
-        const int f = tid + j * kThreads;
+        const int f = tid + j * kDecThreads;
         if (f < F) {
             const FeatDesc dk = tab ? desc_from_packed(pf[j], qc, false) : make_desc(d, n, f, tau, false);
             const FeatDesc dq = tab ? desc_from_packed(pf[j], qc, true) : make_desc(d, n, f, tau, true);
@@ -146,7 +151,7 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     float yz = 0.f;
     const float* Z = S + F * DV;
     float* GZ = gS + (int64_t)F * DV;
-    for (int f = tid; f < F; f += kThreads) {
+    for (int f = tid; f < F; f += kDecThreads) {
         const float z = Z[f] + pk[f];
         GZ[f] = z;
         yz = fmaf(pq[f], z, yz);
@@ -171,7 +176,7 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
         const int g = tid >> 2, c = tid & 3;
         float acc = 0.f, den = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < kDecWarps; ++w) {
             const float4 t = red[w][g];
             acc += c == 0 ? t.x : c == 1 ? t.y : c == 2 ? t.z : t.w;
             den += zr[w];
@@ -295,7 +300,7 @@ cudaError_t launch_tma(const Tin* q, const Tin* k, const Tin* v, float* state, f
         if (set_err[dev] != cudaSuccess) return set_err[dev];
     }
     TA_TIMED(stream, "decode_tma_kernel",
-             fn<<<BH, kThreads, dyn, stream>>>(q, k, v, state, out, d, n, tau, F, stride, bytes, err));
+             fn<<<BH, kDecThreads, dyn, stream>>>(q, k, v, state, out, d, n, tau, F, stride, bytes, err));
     return cudaGetLastError();
 }
 

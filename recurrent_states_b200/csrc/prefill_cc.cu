@@ -102,45 +102,79 @@ group_state_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, float* 
 }
 
 // ---------------------------------------------------------------- B
-// Exclusive scan over the NG group states of a head, in place.  Each thread
-// owns 4 consecutive state elements (one float4 column) of one head and keeps
-// the loads of kScanRun groups in flight before it adds them up.  The final
-// running sum is the state after every group; elements past F*(d_v+1) (the
-// padding, never written by the producers) are written as zeros there.
-constexpr int kScanThreads = 128;
-constexpr int kScanRun = 16;
+// Exclusive scan over the NG group states of a head, in place, starting from
+// a carried-in state (or zero).  A block covers kScanCols float4 columns of
+// one head; its kScanParts warp groups take consecutive quarters of the
+// groups, keep all their loads in flight, and combine the quarters' totals
+// through shared memory.  The total is the state after every group; elements
+// past F*(d_v+1) (padding, never written by the producers) come out as zeros.
+constexpr int kScanCols = 32;                        // float4 columns per block
+constexpr int kScanParts = 4;                        // group quarters per block
+constexpr int kScanThreads = kScanCols * kScanParts; // 128
+constexpr int kScanRun = 8;                          // loads in flight per thread
 
-__global__ void __launch_bounds__(kScanThreads, 4)
+__global__ void __launch_bounds__(kScanThreads, 8)
 scan_kernel(float* __restrict__ W, const float* __restrict__ state_in, float* __restrict__ state_out, int NG,
             int64_t stride, int64_t used) {
     // the group states come from the previous kernel; the next one may start
     // its independent work as soon as this grid is resident
     ptx::pdl_wait_primary();
     ptx::pdl_launch_dependents();
+    __shared__ float4 part_sum[kScanParts][kScanCols];
     const int bh = blockIdx.y;
-    const int64_t e4 = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
+    const int col = threadIdx.x % kScanCols, part = threadIdx.x / kScanCols;
+    const int64_t e4 = (int64_t)blockIdx.x * kScanCols + col;
     const int64_t s4 = stride / 4;
-    if (e4 >= s4) return;
+    const bool live = e4 < s4;
+    const int per = (NG + kScanParts - 1) / kScanParts;
+    const int g_begin = min(NG, part * per), g_end = min(NG, g_begin + per);
     float4* base = reinterpret_cast<float4*>(W + (int64_t)bh * NG * stride) + e4;
-    // the carried state the sequence continues from (zero for a fresh one);
-    // its padding is masked so that garbage there cannot leak into sums
-    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (state_in) {
-        run = reinterpret_cast<const float4*>(state_in + (int64_t)bh * stride)[e4];
-        const int64_t e = e4 * 4;
-        if (e + 0 >= used) run.x = 0.f;
-        if (e + 1 >= used) run.y = 0.f;
-        if (e + 2 >= used) run.z = 0.f;
-        if (e + 3 >= used) run.w = 0.f;
-    }
-    for (int g0 = 0; g0 < NG; g0 += kScanRun) {
+    const int64_t e = e4 * 4;
+    auto mask_tail = [&](float4 r) {
+        if (e + 0 >= used) r.x = 0.f;
+        if (e + 1 >= used) r.y = 0.f;
+        if (e + 2 >= used) r.z = 0.f;
+        if (e + 3 >= used) r.w = 0.f;
+        return r;
+    };
+
+    // pass 1: this quarter's total
+    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g0 = g_begin; g0 < g_end; g0 += kScanRun) {
         float4 x[kScanRun];
 #pragma unroll
         for (int j = 0; j < kScanRun; ++j)
-            if (g0 + j < NG) x[j] = base[(int64_t)(g0 + j) * s4];
+            if (live && g0 + j < g_end) x[j] = base[(int64_t)(g0 + j) * s4];
+#pragma unroll
+        for (int j = 0; j < kScanRun; ++j)
+            if (live && g0 + j < g_end) {
+                tot.x += x[j].x;
+                tot.y += x[j].y;
+                tot.z += x[j].z;
+                tot.w += x[j].w;
+            }
+    }
+    part_sum[part][col] = tot;
+    __syncthreads();
+    // the carried state plus the earlier quarters
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (state_in && live) run = mask_tail(reinterpret_cast<const float4*>(state_in + (int64_t)bh * stride)[e4]);
+    for (int p = 0; p < part; ++p) {
+        const float4 t = part_sum[p][col];
+        run.x += t.x;
+        run.y += t.y;
+        run.z += t.z;
+        run.w += t.w;
+    }
+    // pass 2: exclusive prefixes (these loads hit L2: pass 1 just read them)
+    for (int g0 = g_begin; g0 < g_end; g0 += kScanRun) {
+        float4 x[kScanRun];
+#pragma unroll
+        for (int j = 0; j < kScanRun; ++j)
+            if (live && g0 + j < g_end) x[j] = base[(int64_t)(g0 + j) * s4];
 #pragma unroll
         for (int j = 0; j < kScanRun; ++j) {
-            if (g0 + j < NG) {
+            if (live && g0 + j < g_end) {
                 base[(int64_t)(g0 + j) * s4] = run;
                 run.x += x[j].x;
                 run.y += x[j].y;
@@ -149,15 +183,9 @@ scan_kernel(float* __restrict__ W, const float* __restrict__ state_in, float* __
             }
         }
     }
-    if (state_out) {
-        const int64_t e = e4 * 4;
-        float4 r = run;
-        if (e + 0 >= used) r.x = 0.f;
-        if (e + 1 >= used) r.y = 0.f;
-        if (e + 2 >= used) r.z = 0.f;
-        if (e + 3 >= used) r.w = 0.f;
-        reinterpret_cast<float4*>(state_out + (int64_t)bh * stride)[e4] = r;
-    }
+    // after its own quarter the last part holds the total
+    if (state_out && live && part == kScanParts - 1)
+        reinterpret_cast<float4*>(state_out + (int64_t)bh * stride)[e4] = mask_tail(run);
 }
 
 // ---------------------------------------------------------------- C
@@ -362,7 +390,7 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
 #undef TA_LAUNCH_A
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // B
-    const dim3 gB((unsigned)((stride / 4 + kScanThreads - 1) / kScanThreads), BH);
+    const dim3 gB((unsigned)((stride / 4 + kScanCols - 1) / kScanCols), BH);
     TA_TIMED(stream, "cc_scan_kernel",
              scan_kernel<<<gB, kScanThreads, 0, stream>>>(W, state_in, state_out, plan.NG, stride, F * (dv + 1)));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -380,7 +408,7 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
 
 cudaError_t launch_state_scan(float* W, const float* state_in, float* state_out, int BH, int NG, int64_t stride,
                               int64_t used, cudaStream_t stream, bool pdl) {
-    const dim3 g((unsigned)((stride / 4 + kScanThreads - 1) / kScanThreads), BH);
+    const dim3 g((unsigned)((stride / 4 + kScanCols - 1) / kScanCols), BH);
     cudaError_t e = cudaSuccess;
     TA_TIMED(stream, "scan_kernel",
              e = launch_maybe_pdl(scan_kernel, g, dim3(kScanThreads), 0, stream, pdl, W, state_in, state_out, NG,

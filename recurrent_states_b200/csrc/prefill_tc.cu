@@ -79,12 +79,6 @@ constexpr uint32_t kSmemState = kOffBl + kC * kFP * 2;  // 114,688 bytes: two CT
 
 static_assert(kSmemOut <= 232448 - 256, "chunk_out shared memory");
 
-__device__ __forceinline__ uint32_t kmaj(int r, int kgroup, uint32_t sbo) {
-    return (uint32_t)(r >> 3) * sbo + (uint32_t)kgroup * 128u + (uint32_t)(r & 7) * 16u;
-}
-__device__ __forceinline__ uint32_t mnmaj(int k, int ngroup, uint32_t lbo) {
-    return (uint32_t)ngroup * 128u + (uint32_t)(k >> 3) * lbo + (uint32_t)(k & 7) * 16u;
-}
 
 __device__ __forceinline__ void ld_row16(const bf16* p, float (&x)[16]) {
     const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));

@@ -47,6 +47,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
            | ((uint32_t)(M >> 4) << 24);
 }
 
+// Byte offset of row r, 8-element K group `kgroup` in a K-major operand with
+// LBO = 128 (K groups of a row group contiguous) and row-group stride sbo.
+__device__ __forceinline__ uint32_t kmaj(int r, int kgroup, uint32_t sbo) {
+    return (uint32_t)(r >> 3) * sbo + (uint32_t)kgroup * 128u + (uint32_t)(r & 7) * 16u;
+}
+
+// Byte offset of K row k, 8-element MN group `ngroup` in an MN-major operand
+// with SBO = 128 (MN groups of a K group contiguous) and K-group stride lbo.
+__device__ __forceinline__ uint32_t mnmaj(int k, int ngroup, uint32_t lbo) {
+    return (uint32_t)ngroup * 128u + (uint32_t)(k >> 3) * lbo + (uint32_t)(k & 7) * 16u;
+}
+
 // ---------------------------------------------------------------- TMEM
 
 // Allocates ncols TMEM columns (power of two >= 32); the whole warp calls it.
