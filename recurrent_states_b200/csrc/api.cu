@@ -72,6 +72,9 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, const float* state_in
         const int tc = ta::tc::try_prefill(q, k, v, out, state_in, state_out, (int)BH, N, d_k, d_v, n, tau, F,
                                            stride, stream);
         if (tc != ta::tc::kNotApplicable) return tc;
+        const int tcf = ta::tc::try_prefill_tiled(q, k, v, out, state_in, state_out, (int)BH, N, d_k, d_v, n, tau,
+                                                  F, stride, stream);
+        if (tcf != ta::tc::kNotApplicable) return tcf;
     }
 
     const ta::CcPlan plan = ta::plan_prefill_cc((int)BH, N, d_k, d_v, n, F, stride);

@@ -16,9 +16,19 @@ int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloa
                 const float* state_in, float* state_out, int BH, int N, int d, int dv, int n, float tau,
                 int64_t F, int64_t stride, cudaStream_t stream);
 
+// Feature-tiled variant for d_k in {16, 32, 64}, d_v = 64 and any number of
+// features (tiles of 128 features; prefill_tcf.cu).
+int try_prefill_tiled(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, float* out,
+                      const float* state_in, float* state_out, int BH, int N, int d, int dv, int n, float tau,
+                      int64_t F, int64_t stride, cudaStream_t stream);
+
 // fp32 inputs never take the tensor-core path.
 inline int try_prefill(const float*, const float*, const float*, float*, const float*, float*, int, int, int,
                        int, int, float, int64_t, int64_t, cudaStream_t) {
+    return kNotApplicable;
+}
+inline int try_prefill_tiled(const float*, const float*, const float*, float*, const float*, float*, int, int,
+                             int, int, int, float, int64_t, int64_t, cudaStream_t) {
     return kNotApplicable;
 }
 

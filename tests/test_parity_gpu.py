@@ -56,6 +56,10 @@ CASES = [
     (1, 1, 333, 32, 32, 3),
     (2, 1, 129, 5, 8, 4),
     (1, 1, 77, 64, 256, 2),
+    # several token groups on the feature-tiled tensor-core path
+    (1, 2, 2500, 32, 64, 3),
+    (1, 1, 3000, 16, 64, 4),
+    (1, 1, 2600, 64, 64, 3),
 ]
 
 
@@ -267,7 +271,7 @@ def test_merge_and_split_prefill():
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("d,dv,n,N,cut", [(16, 64, 3, 1000, 384), (16, 64, 3, 700, 77), (16, 64, 3, 300, 1),
                                           (16, 16, 3, 500, 256), (64, 64, 3, 600, 130), (16, 64, 5, 400, 200),
-                                          (7, 12, 2, 200, 33)])
+                                          (32, 64, 3, 2600, 300), (7, 12, 2, 200, 33)])
 def test_prefill_from_state_continues_the_sequence(dtype, d, dv, n, N, cut):
     """Prefill of the tail from the head's state equals the oracle's recursion
     over the whole sequence (outputs of the tail, final state)."""
