@@ -1,0 +1,13 @@
+// Explicit instantiations of the feature-tiled prefill: (d_k 16, n 4), (d_k 16, n run-time).
+#include "prefill_tcf.cuh"
+
+namespace ta {
+namespace tc {
+namespace tcf {
+template int run<16, 4>(const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, float*, const float*, float*, int,
+                           int, int, float, int64_t, int64_t, unsigned int*, cudaStream_t);
+template int run<16, 0>(const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, float*, const float*, float*, int,
+                           int, int, float, int64_t, int64_t, unsigned int*, cudaStream_t);
+}  // namespace tcf
+}  // namespace tc
+}  // namespace ta

@@ -60,6 +60,8 @@ CASES = [
     (1, 2, 2500, 32, 64, 3),
     (1, 1, 3000, 16, 64, 4),
     (1, 1, 2600, 64, 64, 3),
+    (1, 1, 700, 32, 64, 4),   # run-time feature descriptors on the tiled path
+    (1, 1, 500, 64, 64, 2),
 ]
 
 
