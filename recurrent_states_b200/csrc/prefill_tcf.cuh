@@ -10,19 +10,28 @@
 //        dS_g[tile, :] = Phi_K[:, tile]^T (128 x G) . [V|1|0] (G x 80),
 //        accumulated in TMEM over 64-token stages;
 //   2. the exclusive scan over groups (shared with the other paths);
-//   3. tcf_out_kernel (128 queries, head):
+//   3. tcf_pack_kernel: each S_<g cut into 64-feature read-out operand tiles,
+//      split into hi/lo bf16 once per group rather than once per query tile;
+//   4. tcf_out_kernel (128 queries, head):
 //        O = sum over 64-key tiles of the group up to the diagonal of
 //              (poly(tau Q K^T) (.) mask) [V|1|0]
 //          + sum over 64-feature tiles of (c (.) Phi_Q[:, tile]) S_<g[tile, :],
 //        o = O[:, :64] / O[:, 64].
 // Operands produced in fp32 (Phi_K, Phi_Q, P and S_<g) are split into hi/lo
 // bf16 pairs (about 16 significant bits reach the fp32 accumulators); q, k and
-// v are bf16 already.  Both kernels are software pipelined: 16-byte cp.async
-// copies fill a ring of stages, the CUDA cores evaluate features (or P) for
-// one stage while the tensor cores run the MMAs of the previous one, and each
-// stage is handed back through an mbarrier that tcgen05.commit arrives on.
-// Every wait is bounded; a timeout sets a device error bit.
+// v are bf16 already.
+//
+// Both CTA kinds are warp-specialised.  One thread issues TMA tensor loads
+// (q, k, v rows into the K-major / MN-major operand layouts, zero-filled past
+// the sequence), one thread issues every tcgen05.mma, and two warpgroups of
+// CUDA cores evaluate features (or P) for alternate stages, so that the
+// loads, the tensor cores and the feature arithmetic of different stages run
+// at the same time.  Hand-offs are mbarriers: TMA transaction counts, 128
+// arrivals from a warpgroup, or tcgen05.commit.  Every wait is bounded and a
+// failed wait stops the other roles' waits too; a device error bit records it.
 #pragma once
+
+#include <cuda.h>
 
 #include <mutex>
 
@@ -34,6 +43,7 @@
 #include "prefill_tc.h"
 #include "ptx.cuh"
 #include "tcgen05.cuh"
+#include "tmap.h"
 
 namespace ta {
 namespace tc {
@@ -48,25 +58,26 @@ constexpr int kRT = 64;       // features per read-out tile (K of the read-out M
 constexpr int kQ = 128;       // queries per output CTA (M)
 constexpr int kDV = 64;
 constexpr int kNV = 80;       // [V | 1 | 0 ...]
-constexpr int kThreads = 256;
+constexpr int kCompute = 256; // two warpgroups
 constexpr uint32_t kWaitPolls = 1u << 24;
 
-constexpr uint32_t kLboNV = (kNV / 8) * 128;    // K-group stride of an MN-major operand 80 wide
-constexpr uint32_t kLboFT = (kFT / 8) * 128;    // K-group stride of an MN-major operand 128 wide
-constexpr uint32_t kSbo64 = (64 / 8) * 128;     // row-group stride of a K-major operand 64 deep
+constexpr uint32_t kBox = kTok * 16;             // TMA box of 8 elements x 64 rows (1 KB)
+constexpr uint32_t kV1Bytes = (kNV / 8) * kBox;  // [v|1|0]: 10 column groups of one box each
+constexpr uint32_t kPhiBytes = kTok * kFT * 2;   // state-stage Phi_K, hi or lo
+constexpr uint32_t kLboFT = (kFT / 8) * 128;     // its K-group stride
+constexpr uint32_t kPBytes = kQ * kRT * 2;       // P or Phi_Q tile, hi or lo: K-major [128][64]
+constexpr uint32_t kSbo64 = 8 * 128;             // its row-group stride
+constexpr uint32_t kLboNV = (kNV / 8) * 128;     // K-group stride of a packed S tile
+constexpr uint32_t kSHalf = kRT * kNV * 2;       // packed S tile, hi or lo
+constexpr uint32_t kSTile = 2 * kSHalf;          // packed S tile, hi then lo (20 KB)
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
-    return ptx::mbar_wait(bar, parity, kWaitPolls);
+__device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, volatile int* bad) {
+    return ptx::mbar_wait_or_abort(bar, parity, kWaitPolls, bad);
 }
 
-// Orders this thread's shared-memory writes before the tensor cores read them
-// and synchronises the block; true if any thread reports a failure.
-__device__ __forceinline__ bool publish(bool bad) {
-    ptx::fence_proxy_async_smem();
-    fence_before_sync();
-    const bool any = __syncthreads_or(bad) != 0;
-    fence_after_sync();
-    return any;
+__device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
+    const uint32_t a = ptx::smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
 // Eight fp32 values -> hi/lo bf16 chunks stored at two operand addresses.
@@ -77,59 +88,41 @@ __device__ __forceinline__ void store_split8(const float* x, uint8_t* hi_dst, ui
     *reinterpret_cast<uint4*>(lo_dst) = lo;
 }
 
-// `rows` token rows of a [*, D] bf16 tensor into a K-major operand (rows past
-// `valid` >= 1 zero-filled) by 16-byte cp.async.
-template <int D>
-__device__ __forceinline__ void load_rows_kmajor(uint8_t* dst, const bf16* src, int valid, int rows) {
-    constexpr int KC = D / 8;
-    constexpr uint32_t sbo = KC * 128;
-    for (int e = threadIdx.x; e < rows * KC; e += kThreads) {
-        const int r = e / KC, c = e % KC;
-        const int rr = r < valid ? r : valid - 1;
-        ptx::cp_async16(dst + kmaj(r, c, sbo), src + (int64_t)rr * D + c * 8, r < valid ? 16u : 0u);
+// [v | 1 | 0] operand, MN-major [K = 64 tokens][N = 80] with token rows of
+// 16 bytes (K-group stride 128) and one 1 KB box per 8 columns (N-group
+// stride kBox).  TMA fills groups 0..7; group 8 holds the ones column and
+// group 9 zeros, written once.
+__device__ __forceinline__ void init_v1_tail(uint8_t* v1, int tid, int nthreads) {
+    for (int i = tid; i < 2 * kTok; i += nthreads) {
+        const int g = 8 + i / kTok, k = i % kTok;
+        *reinterpret_cast<uint4*>(v1 + g * kBox + k * 16) = make_uint4(g == 8 ? 0x3F80u : 0u, 0, 0, 0);
     }
-}
-
-// [v | 1 | 0] rows of 64 tokens as an MN-major [K = token][N = 80] operand:
-// v by cp.async, the ones column by a plain store (column group 9 stays 0).
-__device__ __forceinline__ void load_v1(uint8_t* dst, const bf16* v, int valid) {
-    for (int e = threadIdx.x; e < kTok * 8; e += kThreads) {
-        const int r = e >> 3, c = e & 7;
-        const int rr = r < valid ? r : valid - 1;
-        ptx::cp_async16(dst + mnmaj(r, c, kLboNV), v + (int64_t)rr * kDV + c * 8, r < valid ? 16u : 0u);
-    }
-    if (threadIdx.x < kTok)
-        *reinterpret_cast<uint4*>(dst + mnmaj(threadIdx.x, 8, kLboNV)) =
-            make_uint4((int)threadIdx.x < valid ? 0x3F80u : 0u, 0, 0, 0);
-}
-
-__device__ __forceinline__ void zero_v1_tail(uint8_t* dst) {
-    if (threadIdx.x < kTok) *reinterpret_cast<uint4*>(dst + mnmaj(threadIdx.x, 9, kLboNV)) = make_uint4(0, 0, 0, 0);
 }
 
 // ---------------------------------------------------------------- 1. group states
-// Stage: Phi_K hi/lo as MN-major [K = 64 tokens][M = 128 features], the
-// [V|1|0] operand, and the k rows (K-major) the features are read from.
 template <int D>
-struct StateSmem {
-    static constexpr uint32_t kPhi = kTok * kFT * 2;
-    static constexpr uint32_t kV1 = kTok * kNV * 2;
-    static constexpr uint32_t kK = kTok * D * 2;
-    static constexpr uint32_t kStage = 2 * kPhi + kV1 + kK;
-    static constexpr int kStages = 3;
-    static constexpr uint32_t kBytes = kStages * kStage;
-    static constexpr int kOutStride = kDV + 4;  // epilogue staging rows: 16-byte aligned, float4 conflict-free
+struct StSm {
+    static constexpr uint32_t kK = kTok * D * 2;  // k rows, K-major, chunk stride kBox
+    static constexpr uint32_t kStage = 2 * kPhiBytes + kV1Bytes + kK;
+    static constexpr int kStages = 4;             // stage b always belongs to warpgroup b & 1
+    static constexpr uint32_t kBytes = kStages * kStage + 1024;
+    static constexpr int kOutStride = kDV + 4;    // epilogue staging rows: 16-byte aligned, float4 conflict-free
     static_assert(kFT * kOutStride * 4 <= kStage, "epilogue staging fits one stage");
 };
+constexpr int kStateThreads = kCompute + 32;
 
 template <int D, int N>
-__global__ void __launch_bounds__(kThreads, 1)
-tcf_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, float* __restrict__ W, int Ntok, int n,
-                 int F, int64_t stride, int G, int NG, unsigned int* __restrict__ err) {
-    using L = StateSmem<D>;
-    extern __shared__ __align__(1024) uint8_t sm[];
-    __shared__ __align__(8) uint64_t bar[L::kStages];
+__global__ void __launch_bounds__(kStateThreads, 1)
+tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                 float* __restrict__ W, int Ntok, int n, int F, int64_t stride, int G, int NG,
+                 unsigned int* __restrict__ err) {
+    using L = StSm<D>;
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t* sm = align1k(sm_raw);
+    __shared__ __align__(8) uint64_t loaded[L::kStages], full[L::kStages], empty[L::kStages];
     __shared__ uint32_t tslot;
+    __shared__ int s_bad;
+    volatile int* bad = &s_bad;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x, ft = blockIdx.y, bh = blockIdx.z;
@@ -138,79 +131,106 @@ tcf_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, float* 
     const int64_t gt0 = (int64_t)g * G;
     const int gn = (int)min64(G, (int64_t)Ntok - gt0);
     const int nsub = (gn + kTok - 1) / kTok;
-    const bf16* kg = k + ((int64_t)bh * Ntok + gt0) * D;
-    const bf16* vg = v + ((int64_t)bh * Ntok + gt0) * kDV;
+    auto stage = [&](int b) { return sm + b * L::kStage; };
 
     if (tid == 0) {
-        for (int i = 0; i < L::kStages; ++i) ptx::mbar_init(&bar[i], 1);
+        for (int i = 0; i < L::kStages; ++i) {
+            ptx::mbar_init(&loaded[i], 1);
+            ptx::mbar_init(&full[i], kCompute / 2);
+            ptx::mbar_init(&empty[i], 1);
+        }
+        s_bad = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0) {
+    if (warp == kCompute / 32) {
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
-    for (int s = 0; s < L::kStages; ++s) zero_v1_tail(sm + s * L::kStage + 2 * L::kPhi);
-    auto load_stage = [&](int s) {
-        uint8_t* st = sm + (s % L::kStages) * L::kStage;
-        const int valid = min(kTok, gn - s * kTok);
-        load_rows_kmajor<D>(st + 2 * L::kPhi + L::kV1, kg + (int64_t)s * kTok * D, valid, kTok);
-        load_v1(st + 2 * L::kPhi, vg + (int64_t)s * kTok * kDV, valid);
-        ptx::cp_async_commit();
-    };
-    load_stage(0);
-    if (nsub > 1) load_stage(1);
+    for (int b = 0; b < L::kStages; ++b) init_v1_tail(stage(b) + 2 * kPhiBytes, tid, kStateThreads);
+    ptx::fence_proxy_async_smem();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tacc = tslot;
 
-    // thread -> token t of the stage, features [32 qf, 32 qf + 32) of the tile
-    const int t = tid & (kTok - 1), qf = tid >> 6;
-    bool bad = false;
-    int issued = 0;  // stages whose MMAs were committed
-    for (int s = 0; s < nsub; ++s) {
-        uint8_t* st = sm + (s % L::kStages) * L::kStage;
-        if (s + 1 < nsub) ptx::cp_async_wait<1>();
-        else ptx::cp_async_wait<0>();
-        __syncthreads();
-        {
-            float o[32];
-            const uint8_t* rowbase = st + 2 * L::kPhi + L::kV1 + kmaj(t, 0, (D / 8) * 128);
-            fe::Eval<D, N, false>::block(ft * 4 + qf, rowbase, nullptr, n, F, 0.f, o);
+    if (warp == kCompute / 32) {
+        if (lane == 0) {
+            // TMA producer and MMA issuer
+            int ld = 0, mm = 0;
+            for (int s = 0; s < nsub && !*bad; ++s) {
+                while (ld < nsub && ld < s + L::kStages) {
+                    const int b = ld % L::kStages;
+                    if (ld >= L::kStages && !waitb(&empty[b], ((ld / L::kStages) - 1) & 1, bad)) break;
+                    uint8_t* st = stage(b);
+                    ptx::mbar_arrive_expect_tx(&loaded[b], (uint32_t)(D / 8 + 8) * kBox);
+                    const int y = (int)(gt0 + (int64_t)ld * kTok);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                store_split8(o + 8 * i, st + mnmaj(t, qf * 4 + i, kLboFT), st + L::kPhi + mnmaj(t, qf * 4 + i, kLboFT));
-        }
-        if (publish(bad)) {
-            bad = true;
-            break;
-        }
-        if (tid == 0) {
-            const uint32_t id = idesc_bf16(kFT, kNV, 1, 1);
+                    for (int c = 0; c < D / 8; ++c)
+                        ptx::tma_load_3d(st + 2 * kPhiBytes + kV1Bytes + c * kBox, &tmk, c * 8, y, bh, &loaded[b]);
 #pragma unroll
-            for (int ks = 0; ks < kTok / 16; ++ks) {
-                const uint64_t b = smem_desc(st + 2 * L::kPhi + ks * 2 * kLboNV, kLboNV, 128);
-                mma_bf16(tacc, smem_desc(st + ks * 2 * kLboFT, kLboFT, 128), b, id, (s > 0 || ks > 0) ? 1u : 0u);
-                mma_bf16(tacc, smem_desc(st + L::kPhi + ks * 2 * kLboFT, kLboFT, 128), b, id, 1u);
+                    for (int c = 0; c < 8; ++c)
+                        ptx::tma_load_3d(st + 2 * kPhiBytes + c * kBox, &tmv, c * 8, y, bh, &loaded[b]);
+                    ++ld;
+                }
+                if (*bad) break;
+                const int b = s % L::kStages;
+                if (!waitb(&full[b], (s / L::kStages) & 1, bad)) break;
+                fence_after_sync();
+                uint8_t* st = stage(b);
+                const uint32_t id = idesc_bf16(kFT, kNV, 1, 1);
+#pragma unroll
+                for (int ks = 0; ks < kTok / 16; ++ks) {
+                    const uint64_t bd = smem_desc(st + 2 * kPhiBytes + ks * 256, 128, kBox);
+                    mma_bf16(tacc, smem_desc(st + ks * 2 * kLboFT, kLboFT, 128), bd, id, (s > 0 || ks > 0) ? 1u : 0u);
+                    mma_bf16(tacc, smem_desc(st + kPhiBytes + ks * 2 * kLboFT, kLboFT, 128), bd, id, 1u);
+                }
+                mma_commit(&empty[b]);
+                mm = s + 1;
             }
-            mma_commit(&bar[s % L::kStages]);
+            // the last commit covers every MMA issued; loads issued but never
+            // consumed (only after a failure) must land before the CTA leaves
+            if (mm > 0 && !ptx::mbar_wait(&empty[(mm - 1) % L::kStages], ((mm - 1) / L::kStages) & 1, kWaitPolls))
+                *bad = 1;
+            for (int li = mm; li < ld; ++li)
+                ptx::mbar_wait(&loaded[li % L::kStages], (li / L::kStages) & 1, kWaitPolls);
         }
-        issued = s + 1;
-        // stage (s + 2) % 3 was last read by the MMAs of stage s - 1
-        if (s >= 1 && !wait_bar(&bar[(s - 1) % L::kStages], ((s - 1) / L::kStages) & 1)) bad = true;
-        if (s + 2 < nsub && !bad) load_stage(s + 2);
+    } else {
+        // warpgroup w evaluates the features of stages w, w + 2, ...:
+        // token t, features [64 h, 64 h + 64) of the tile
+        const int w = warp >> 2, wt = tid & 127, t = wt & (kTok - 1), h = wt >> 6;
+        for (int s = w; s < nsub; s += 2) {
+            const int b = s % L::kStages;
+            if (!waitb(&loaded[b], (s / L::kStages) & 1, bad)) break;
+            uint8_t* st = stage(b);
+            const int valid = min(kTok, gn - s * kTok);
+            const uint8_t* rowbase = st + 2 * kPhiBytes + kV1Bytes + t * 16;
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+                float o[32];
+                fe::Eval<D, N, false, kBox>::block(ft * 4 + h * 2 + sub, rowbase, nullptr, n, F, 0.f, o);
+                if (t >= valid) {  // zero-filled rows past the sequence: phi(0) has a constant feature
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t off = mnmaj(t, h * 8 + sub * 4 + i, kLboFT);
+                    store_split8(o + 8 * i, st + off, st + kPhiBytes + off);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&full[b]);
+        }
     }
-    ptx::cp_async_wait<0>();
-    // MMAs complete in order: the last commit covers them all
-    if (issued > 0 && !wait_bar(&bar[(issued - 1) % L::kStages], ((issued - 1) / L::kStages) & 1)) bad = true;
-    bad = __syncthreads_or(bad) != 0;
+    __syncthreads();
     fence_after_sync();
+    const bool ok = s_bad == 0;
 
     // TMEM lane j holds feature f0 + j: columns 0..63 its S_v row, 64 its z
     float* Wg = W + ((int64_t)bh * NG + g) * stride;
     float* sOut = reinterpret_cast<float*>(sm);
-    const int row = (warp & 3) * 32 + lane, half = warp >> 2;
-    if (!bad) {
+    if (ok && tid < kCompute) {
+        const int row = (warp & 3) * 32 + lane, half = warp >> 2;
         const uint32_t ta = tacc + ((uint32_t)((warp & 3) * 32) << 16);
         float r[32];
         tmem_ld32(ta + half * 32, r);
@@ -221,57 +241,86 @@ tcf_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, float* 
 #pragma unroll
         for (int i = 0; i < 8; ++i) so[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
         if (half == 1 && row < nf) Wg[(int64_t)F * kDV + f0 + row] = zz[0];
-    } else if (tid == 0) {
-        atomicOr(err, kErrPrefillPipe);
     }
+    if (!ok && tid == 0) atomicOr(err, kErrPrefillPipe);
     fence_before_sync();
     __syncthreads();
-    if (!bad) {
+    if (ok) {
         float4* dst = reinterpret_cast<float4*>(Wg + (int64_t)f0 * kDV);
-        for (int e = tid; e < nf * (kDV / 4); e += kThreads) {
+        for (int e = tid; e < nf * (kDV / 4); e += kStateThreads) {
             const int j = e / (kDV / 4), c = e % (kDV / 4);
             dst[e] = *reinterpret_cast<const float4*>(sOut + j * L::kOutStride + c * 4);
         }
     }
-    if (warp == 0) {
+    if (warp == kCompute / 32) {
         fence_after_sync();
         tmem_dealloc(tacc, 128);
     }
 }
 
-// ---------------------------------------------------------------- 3. outputs
+// ---------------------------------------------------------------- 3. read-out operand tiles
+// S_<g (fp32, the library's state layout) -> for each 64-feature tile r:
+// hi then lo bf16 [K = 64 features][N = 80] MN-major (K-group stride 1280 B),
+// column 64 the z entry, columns 65..79 and features past F zero.
+__global__ void __launch_bounds__(256)
+tcf_pack_kernel(const float* __restrict__ W, uint8_t* __restrict__ PK, int F, int64_t stride, int NG, int R,
+                int g0) {
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait_primary();
+    const int r = blockIdx.x, g = g0 + blockIdx.y, bh = blockIdx.z;
+    const float* S = W + ((int64_t)bh * NG + g) * stride;
+    uint8_t* dst = PK + (((int64_t)bh * NG + g) * R + r) * kSTile;
+    for (int u = threadIdx.x; u < kRT * 10; u += 256) {
+        const int gq = u / kRT, j = u % kRT, f = r * kRT + j;
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (f < F) {
+            if (gq < 8) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(S + (int64_t)f * kDV + gq * 8));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(S + (int64_t)f * kDV + gq * 8) + 1);
+                x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+                x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+            } else if (gq == 8) {
+                x[0] = __ldg(S + (int64_t)F * kDV + f);
+            }
+        }
+        const uint32_t off = mnmaj(j, gq, kLboNV);
+        store_split8(x, dst + off, dst + kSHalf + off);
+    }
+}
+
+// ---------------------------------------------------------------- 4. outputs
 template <int D>
-struct OutSmem {
-    static constexpr uint32_t kSboD = (D / 8) * 128;  // row-group stride of K-major rows of D
-    static constexpr uint32_t kQop = kQ * D * 2;      // Q, K-major [128][D]
-    // pairwise: ring of 3 (K tile, [V|1|0]) + 2 x (P hi, P lo)
-    static constexpr uint32_t kKt = kTok * D * 2;
-    static constexpr uint32_t kV1 = kTok * kNV * 2;
-    static constexpr uint32_t kKV = kKt + kV1;
-    static constexpr uint32_t kP = kQ * kTok * 2;     // one of hi/lo, K-major [128][64]
-    static constexpr uint32_t kPbase = 3 * kKV;
-    static constexpr uint32_t kPair = kPbase + 4 * kP;
-    // read-out: 2 x (Phi_Q hi, lo K-major [128][64]; S hi, lo MN-major [64][80]) + fp32 S staging
-    static constexpr uint32_t kA = kQ * kRT * 2;
-    static constexpr uint32_t kB = kRT * kNV * 2;
-    static constexpr uint32_t kRS = 2 * kA + 2 * kB;
-    static constexpr uint32_t kStg = 2 * kRS;              // staging: [64][64] S_v rows then [64] z
-    static constexpr uint32_t kRead = kStg + kRT * kDV * 4 + kRT * 4;
-    static constexpr uint32_t kU = kPair > kRead ? kPair : kRead;
-    static constexpr uint32_t kBytes = kQop + kU;
+struct OutSm {
+    static constexpr uint32_t kQop = kQ * D * 2;  // Q, K-major, chunk stride kQ * 16
+    static constexpr uint32_t kKt = kTok * D * 2; // key tile, K-major, chunk stride kBox
+    static constexpr uint32_t kKV = kKt + kV1Bytes;
+    static constexpr int kKVSlots = 3, kSSlots = 3;
+    static constexpr uint32_t kKVbase = kQop;
+    static constexpr uint32_t kSbase = kKVbase + kKVSlots * kKV;
+    static constexpr uint32_t kPPbase = kSbase + kSSlots * kSTile;
+    static constexpr uint32_t kPP = 2 * kPBytes;  // P or Phi_Q, hi then lo, one per warpgroup
+    static constexpr uint32_t kBytes = kPPbase + 2 * kPP + 1024;
 };
+constexpr int kOutThreads = kCompute + 96;  // + MMA warp, q/k/v producer warp, S producer warp
 
 template <int D, int N>
-__global__ void __launch_bounds__(kThreads, 1)
-tcf_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-               const float* __restrict__ W, float* __restrict__ out, int Ntok, int n, float tau, int F,
-               int64_t stride, int G, int NG, int carried, unsigned int* __restrict__ err) {
-    using L = OutSmem<D>;
-    extern __shared__ __align__(1024) uint8_t sm[];
-    __shared__ __align__(8) uint64_t bar_sc[2], bar_pv[2], bar_ro[2], bar_st;
+__global__ void __launch_bounds__(kOutThreads, 1)
+tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+               const __grid_constant__ CUtensorMap tmv, const uint8_t* __restrict__ PK, float* __restrict__ out,
+               int Ntok, int n, float tau, int F, int G, int NG, int R, int carried,
+               unsigned int* __restrict__ err) {
+    using L = OutSm<D>;
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t* sm = align1k(sm_raw);
+    __shared__ __align__(8) uint64_t q_loaded, kv_loaded[L::kKVSlots], kv_empty[L::kKVSlots], sc_full[2], pp_full[2],
+        pp_free[2], s_loaded[L::kSSlots], s_empty[L::kSSlots], o_done;
     __shared__ uint32_t tslot;
+    __shared__ int s_bad;
+    volatile int* bad = &s_bad;
     uint8_t* sQ = sm;
-    uint8_t* sU = sm + L::kQop;
+    auto kv = [&](int slot) { return sm + L::kKVbase + slot * L::kKV; };
+    auto sS = [&](int slot) { return sm + L::kSbase + slot * kSTile; };
+    auto pp = [&](int w) { return sm + L::kPPbase + w * L::kPP; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qt = blockIdx.x, bh = blockIdx.y;
@@ -279,204 +328,216 @@ tcf_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
     const int nq = (int)min64(kQ, (int64_t)Ntok - q0);
     const int g = (int)(q0 / G);
     const int64_t gs = (int64_t)g * G;
-    const int row = (warp & 3) * 32 + lane, half = warp >> 2;
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int64_t kend = min64(q0 + kQ, (int64_t)Ntok);
     const int T = (int)((kend - gs + kTok - 1) / kTok);  // key tiles, >= 1
-
-    float qc[kMaxN];
-#pragma unroll
-    for (int m = 0; m < kMaxN; ++m) qc[m] = query_coeff(m, tau);
+    const int Rr = (g > 0 || carried) ? R : 0;           // read-out tiles
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&bar_sc[i], 1);
-            ptx::mbar_init(&bar_pv[i], 1);
-            ptx::mbar_init(&bar_ro[i], 1);
+        ptx::mbar_init(&q_loaded, 1);
+        for (int i = 0; i < L::kKVSlots; ++i) {
+            ptx::mbar_init(&kv_loaded[i], 1);
+            ptx::mbar_init(&kv_empty[i], 1);
         }
-        ptx::mbar_init(&bar_st, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&sc_full[i], 1);
+            ptx::mbar_init(&pp_full[i], kCompute / 2);
+            ptx::mbar_init(&pp_free[i], 1);
+        }
+        for (int i = 0; i < L::kSSlots; ++i) {
+            ptx::mbar_init(&s_loaded[i], 1);
+            ptx::mbar_init(&s_empty[i], 1);
+        }
+        ptx::mbar_init(&o_done, 1);
+        s_bad = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0) {
+    if (warp == 8) {
         tmem_alloc(&tslot, 256);
         tmem_relinquish();
     }
-    const bf16* kb = k + (int64_t)bh * Ntok * D;
-    const bf16* vb = v + (int64_t)bh * Ntok * kDV;
-    auto load_tile = [&](int t) {
-        uint8_t* st = sU + (t % 3) * L::kKV;
-        const int64_t k0 = gs + (int64_t)t * kTok;
-        const int valid = (int)min64(kTok, kend - k0);
-        load_rows_kmajor<D>(st, kb + k0 * D, valid, kTok);
-        load_v1(st + L::kKt, vb + k0 * kDV, valid);
-        ptx::cp_async_commit();
-    };
-    for (int s = 0; s < 3; ++s) zero_v1_tail(sU + s * L::kKV + L::kKt);
-    load_rows_kmajor<D>(sQ, q + ((int64_t)bh * Ntok + q0) * D, nq, kQ);
-    load_tile(0);
-    if (T > 1) {
-        load_tile(1);
-        ptx::cp_async_wait<1>();
-    } else {
-        ptx::cp_async_wait<0>();
-    }
-    publish(false);
+    for (int s = 0; s < L::kKVSlots; ++s) init_v1_tail(kv(s) + L::kKt, tid, kOutThreads);
+    ptx::fence_proxy_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
     const uint32_t tS = tslot, tO = tslot + 128;
 
-    auto issue_scores = [&](int t) {
-        const uint8_t* kt = sU + (t % 3) * L::kKV;
-        const uint32_t id = idesc_bf16(kQ, kTok, 0, 0);
+    if (warp == 9) {
+        if (lane == 0) {
+            // q once, then key/value tiles through a ring of three slots
+            ptx::mbar_arrive_expect_tx(&q_loaded, L::kQop);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-            mma_bf16(tS + (t & 1) * kTok, smem_desc(sQ + ks * 256, 128, L::kSboD),
-                     smem_desc(kt + ks * 256, 128, L::kSboD), id, ks > 0 ? 1u : 0u);
-        mma_commit(&bar_sc[t & 1]);
-    };
-    if (tid == 0) issue_scores(0);
-
-    bool bad = false;
-    // ------------------------------------------------ pairwise part, 64-key tiles of this group
-    for (int t = 0; t < T; ++t) {
-        if (!wait_bar(&bar_sc[t & 1], (t >> 1) & 1)) bad = true;
-        fence_after_sync();
-        {
-            float s32[32];
-            tmem_ld32(tS + lane_off + (t & 1) * kTok + half * 32, s32);
-            tmem_ld_wait();
-            const int64_t k0 = gs + (int64_t)t * kTok + half * 32;
-            const int64_t qi = q0 + row;
-            uint8_t* ph = sU + L::kPbase + (t & 1) * 2 * L::kP;
+            for (int c = 0; c < D / 8; ++c) ptx::tma_load_3d(sQ + c * (kQ * 16), &tmq, c * 8, (int)q0, bh, &q_loaded);
+            int ld = 0;
+            for (; ld < T; ++ld) {
+                const int slot = ld % L::kKVSlots;
+                if (ld >= L::kKVSlots && !waitb(&kv_empty[slot], ((ld / L::kKVSlots) - 1) & 1, bad)) break;
+                uint8_t* st = kv(slot);
+                ptx::mbar_arrive_expect_tx(&kv_loaded[slot], (uint32_t)(D / 8 + 8) * kBox);
+                const int y = (int)(gs + (int64_t)ld * kTok);
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                float p[8];
+                for (int c = 0; c < D / 8; ++c) ptx::tma_load_3d(st + c * kBox, &tmk, c * 8, y, bh, &kv_loaded[slot]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x = s32[g8 * 8 + e];
-                    float w;
-                    if constexpr (N > 0) {
-                        w = qc[N - 1];
-#pragma unroll
-                        for (int m = N - 2; m >= 0; --m) w = fmaf(w, x, qc[m]);
-                    } else {
-                        w = qc[n - 1];
-                        for (int m = n - 2; m >= 0; --m) w = fmaf(w, x, qc[m]);
-                    }
-                    const int64_t kj = k0 + g8 * 8 + e;
-                    p[e] = (kj <= qi && kj < kend && row < nq) ? w : 0.f;
-                }
-                const uint32_t off = kmaj(row, half * 4 + g8, kSbo64);
-                store_split8(p, ph + off, ph + L::kP + off);
+                for (int c = 0; c < 8; ++c) ptx::tma_load_3d(st + L::kKt + c * kBox, &tmv, c * 8, y, bh, &kv_loaded[slot]);
             }
+            // every issued copy lands before the CTA can leave
+            ptx::mbar_wait(&q_loaded, 0, kWaitPolls);
+            for (int li = (ld > L::kKVSlots ? ld - L::kKVSlots : 0); li < ld; ++li)
+                ptx::mbar_wait(&kv_loaded[li % L::kKVSlots], (li / L::kKVSlots) & 1, kWaitPolls);
         }
-        if (t + 1 < T) ptx::cp_async_wait<0>();  // key tile t + 1 resident
-        if (publish(bad)) {
-            bad = true;
-            break;
+    } else if (warp == 10) {
+        // waits for the preceding kernels even without a read-out, so that
+        // this grid completes only after they have
+        if (lane == 0) ptx::pdl_wait_primary();
+        if (lane == 0 && Rr > 0) {
+            const uint8_t* src = PK + ((int64_t)bh * NG + g) * R * kSTile;
+            int ld = 0;
+            for (; ld < Rr; ++ld) {
+                const int slot = ld % L::kSSlots;
+                if (ld >= L::kSSlots && !waitb(&s_empty[slot], ((ld / L::kSSlots) - 1) & 1, bad)) break;
+                ptx::mbar_arrive_expect_tx(&s_loaded[slot], kSTile);
+                ptx::bulk_g2s(sS(slot), src + (int64_t)ld * kSTile, kSTile, &s_loaded[slot]);
+            }
+            for (int li = (ld > L::kSSlots ? ld - L::kSSlots : 0); li < ld; ++li)
+                ptx::mbar_wait(&s_loaded[li % L::kSSlots], (li / L::kSSlots) & 1, kWaitPolls);
         }
-        if (tid == 0) {
-            const uint8_t* ph = sU + L::kPbase + (t & 1) * 2 * L::kP;
-            const uint8_t* v1 = sU + (t % 3) * L::kKV + L::kKt;
-            const uint32_t id = idesc_bf16(kQ, kNV, 0, 1);
+    } else if (warp == 8) {
+        if (lane == 0) {
+            // every tcgen05.mma of the CTA, in order
+            constexpr uint32_t kSboQ = 128;
+            auto scores = [&](int t) -> bool {
+                const int slot = t % L::kKVSlots;
+                if (!waitb(&kv_loaded[slot], (t / L::kKVSlots) & 1, bad)) return false;
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(kQ, kTok, 0, 0);
 #pragma unroll
-            for (int ks = 0; ks < kTok / 16; ++ks) {
-                const uint64_t b = smem_desc(v1 + ks * 2 * kLboNV, kLboNV, 128);
-                mma_bf16(tO, smem_desc(ph + ks * 256, 128, kSbo64), b, id, (t > 0 || ks > 0) ? 1u : 0u);
-                mma_bf16(tO, smem_desc(ph + L::kP + ks * 256, 128, kSbo64), b, id, 1u);
-            }
-            mma_commit(&bar_pv[t & 1]);
-            if (t + 1 < T) issue_scores(t + 1);
-        }
-        // ring slot (t + 2) % 3 and P buffer (t + 1) & 1 were last read by PV(t - 1)
-        if (t >= 1 && !wait_bar(&bar_pv[(t - 1) & 1], ((t - 1) >> 1) & 1)) bad = true;
-        if (t + 2 < T && !bad) load_tile(t + 2);
-    }
-    ptx::cp_async_wait<0>();
-    if (!bad && !wait_bar(&bar_pv[(T - 1) & 1], ((T - 1) >> 1) & 1)) bad = true;
-    bad = __syncthreads_or(bad) != 0;
-    fence_after_sync();
-
-    // ------------------------------------------------ read-out through S_<g, 64-feature tiles
-    ptx::pdl_wait_primary();  // the scan over group states has completed
-    const int R = (F + kRT - 1) / kRT;
-    int ro_issued = 0;
-    if (!bad && (g > 0 || carried)) {
-        const float* Sg = W + ((int64_t)bh * NG + g) * stride;
-        float* stg = reinterpret_cast<float*>(sU + L::kStg);
-        float* stg_z = stg + kRT * kDV;
-        auto fetch_s = [&](int r) {  // S_v rows of tile r by one bulk copy, z by plain loads
-            const int fr = r * kRT, nr = min(kRT, F - fr);
-            if (tid == 0) {
-                ptx::mbar_arrive_expect_tx(&bar_st, (uint32_t)nr * kDV * 4u);
-                ptx::bulk_g2s(stg, Sg + (int64_t)fr * kDV, (uint32_t)nr * kDV * 4u, &bar_st);
-            }
-            if (tid < kRT) stg_z[tid] = tid < nr ? __ldg(Sg + (int64_t)F * kDV + fr + tid) : 0.f;
-        };
-        fetch_s(0);
-        for (int r = 0; r < R; ++r) {
-            uint8_t* stA = sU + (r & 1) * L::kRS;  // Phi_Q hi, lo, S hi, lo
-            const int nr = min(kRT, F - r * kRT);
-            {
-                float o[32];
-                fe::Eval<D, N, true>::block(r * 2 + half, sQ + kmaj(row, 0, L::kSboD), qc, n, F, tau, o);
-                if (row >= nq) {
+                for (int ks = 0; ks < D / 16; ++ks)
+                    mma_bf16(tS + (t & 1) * kTok, smem_desc(sQ + ks * 2 * (kQ * 16), kQ * 16, kSboQ),
+                             smem_desc(kv(slot) + ks * 2 * kBox, kBox, kSboQ), id, ks > 0 ? 1u : 0u);
+                mma_commit(&sc_full[t & 1]);
+                return true;
+            };
+            bool go = waitb(&q_loaded, 0, bad);
+            if (go) go = scores(0);
+            if (go && T > 1) go = scores(1);
+            for (int t = 0; t < T && go; ++t) {
+                const int w = t & 1;
+                if (!waitb(&pp_full[w], (t >> 1) & 1, bad)) {
+                    go = false;
+                    break;
+                }
+                fence_after_sync();
+                const uint8_t* p = pp(w);
+                const uint8_t* v1 = kv(t % L::kKVSlots) + L::kKt;
+                const uint32_t id = idesc_bf16(kQ, kNV, 0, 1);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0.f;
+                for (int ks = 0; ks < kTok / 16; ++ks) {
+                    const uint64_t bd = smem_desc(v1 + ks * 256, 128, kBox);
+                    mma_bf16(tO, smem_desc(p + ks * 256, 128, kSbo64), bd, id, (t > 0 || ks > 0) ? 1u : 0u);
+                    mma_bf16(tO, smem_desc(p + kPBytes + ks * 256, 128, kSbo64), bd, id, 1u);
                 }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t off = kmaj(row, half * 4 + i, kSbo64);
-                    store_split8(o + 8 * i, stA + off, stA + L::kA + off);
+                mma_commit(&pp_free[w]);
+                mma_commit(&kv_empty[t % L::kKVSlots]);
+                if (t + 2 < T) go = scores(t + 2);
+            }
+            const int nuse[2] = {(T + 1) / 2, T / 2};
+            for (int r = 0; r < Rr && go; ++r) {
+                const int w = r & 1, u = nuse[w] + (r >> 1);
+                if (!waitb(&pp_full[w], u & 1, bad) || !waitb(&s_loaded[r % L::kSSlots], (r / L::kSSlots) & 1, bad)) {
+                    go = false;
+                    break;
                 }
-            }
-            if (!wait_bar(&bar_st, r & 1)) bad = true;
-            __syncthreads();  // staged z visible
-            for (int u = tid; u < kRT * 10; u += kThreads) {
-                const int j = u / 10, gq = u % 10;
-                float x8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                if (j < nr && !bad) {
-                    if (gq < 8) {
-                        const float4 a = *reinterpret_cast<const float4*>(stg + j * kDV + gq * 8);
-                        const float4 b = *reinterpret_cast<const float4*>(stg + j * kDV + gq * 8 + 4);
-                        x8[0] = a.x; x8[1] = a.y; x8[2] = a.z; x8[3] = a.w;
-                        x8[4] = b.x; x8[5] = b.y; x8[6] = b.z; x8[7] = b.w;
-                    } else if (gq == 8) {
-                        x8[0] = stg_z[j];
-                    }
-                }
-                const uint32_t off = mnmaj(j, gq, kLboNV);
-                store_split8(x8, stA + 2 * L::kA + off, stA + 2 * L::kA + L::kB + off);
-            }
-            if (publish(bad)) {
-                bad = true;
-                break;
-            }
-            if (tid == 0) {
+                fence_after_sync();
+                const uint8_t* a = pp(w);
+                const uint8_t* s = sS(r % L::kSSlots);
                 const uint32_t id = idesc_bf16(kQ, kNV, 0, 1);
 #pragma unroll
                 for (int ks = 0; ks < kRT / 16; ++ks) {
-                    const uint64_t ah = smem_desc(stA + ks * 256, 128, kSbo64);
-                    const uint64_t al = smem_desc(stA + L::kA + ks * 256, 128, kSbo64);
-                    const uint64_t bh_ = smem_desc(stA + 2 * L::kA + ks * 2 * kLboNV, kLboNV, 128);
-                    const uint64_t bl_ = smem_desc(stA + 2 * L::kA + L::kB + ks * 2 * kLboNV, kLboNV, 128);
+                    const uint64_t ah = smem_desc(a + ks * 256, 128, kSbo64);
+                    const uint64_t al = smem_desc(a + kPBytes + ks * 256, 128, kSbo64);
+                    const uint64_t bh_ = smem_desc(s + ks * 2 * kLboNV, kLboNV, 128);
+                    const uint64_t bl_ = smem_desc(s + kSHalf + ks * 2 * kLboNV, kLboNV, 128);
                     mma_bf16(tO, ah, bh_, id, 1u);
                     mma_bf16(tO, ah, bl_, id, 1u);
                     mma_bf16(tO, al, bh_, id, 1u);
                 }
-                mma_commit(&bar_ro[r & 1]);
+                mma_commit(&pp_free[w]);
+                mma_commit(&s_empty[r % L::kSSlots]);
             }
-            ro_issued = r + 1;
-            if (r + 1 < R) fetch_s(r + 1);  // the staging was consumed before the barrier above
-            // stage (r + 1) & 1 was last read by the MMAs of tile r - 1
-            if (r >= 1 && !wait_bar(&bar_ro[(r - 1) & 1], ((r - 1) >> 1) & 1)) bad = true;
+            mma_commit(&o_done);  // covers every MMA issued above
+            if (!ptx::mbar_wait(&o_done, 0, kWaitPolls)) *bad = 1;
         }
-        if (!bad && ro_issued > 0 && !wait_bar(&bar_ro[(ro_issued - 1) & 1], ((ro_issued - 1) >> 1) & 1))
-            bad = true;
+    } else {
+        // warpgroup w: P of key tiles w, w + 2, ..., then Phi_Q of read-out
+        // tiles w, w + 2, ...; thread = query row
+        const int w = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const int64_t qi = q0 + row;
+        float qc[kMaxN];
+#pragma unroll
+        for (int m = 0; m < kMaxN; ++m) qc[m] = query_coeff(m, tau);
+        uint8_t* buf = pp(w);
+        int u = 0;
+        for (int t = w; t < T; t += 2, ++u) {
+            if (!waitb(&sc_full[w], (t >> 1) & 1, bad)) break;
+            fence_after_sync();
+            float s[64];
+            tmem_ld32(tS + lane_off + w * kTok, *reinterpret_cast<float(*)[32]>(s));
+            tmem_ld32(tS + lane_off + w * kTok + 32, *reinterpret_cast<float(*)[32]>(s + 32));
+            tmem_ld_wait();
+            const int64_t k0 = gs + (int64_t)t * kTok;
+            const bool mask = k0 + kTok - 1 > q0 || k0 + kTok > Ntok;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float x = s[j];
+                float p;
+                if constexpr (N > 0) {
+                    p = qc[N - 1];
+#pragma unroll
+                    for (int m = N - 2; m >= 0; --m) p = fmaf(p, x, qc[m]);
+                } else {
+                    p = qc[n - 1];
+                    for (int m = n - 2; m >= 0; --m) p = fmaf(p, x, qc[m]);
+                }
+                if (mask && !(k0 + j <= qi && k0 + j < kend)) p = 0.f;
+                s[j] = p;
+            }
+            fence_before_sync();
+            if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
+#pragma unroll
+            for (int kg = 0; kg < 8; ++kg) {
+                const uint32_t off = kmaj(row, kg, kSbo64);
+                store_split8(s + 8 * kg, buf + off, buf + kPBytes + off);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&pp_full[w]);
+        }
+        if (!*bad) {
+            const uint8_t* rowbase = sQ + row * 16;
+            for (int r = w; r < Rr; r += 2, ++u) {
+                float o[64];
+                fe::Eval<D, N, true, kQ * 16>::block(r * 2, rowbase, qc, n, F, tau,
+                                                       *reinterpret_cast<float(*)[32]>(o));
+                fe::Eval<D, N, true, kQ * 16>::block(r * 2 + 1, rowbase, qc, n, F, tau,
+                                                       *reinterpret_cast<float(*)[32]>(o + 32));
+                if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
+#pragma unroll
+                for (int kg = 0; kg < 8; ++kg) {
+                    const uint32_t off = kmaj(row, kg, kSbo64);
+                    store_split8(o + 8 * kg, buf + off, buf + kPBytes + off);
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(&pp_full[w]);
+            }
+        }
     }
-    bad = __syncthreads_or(bad) != 0;
+    __syncthreads();  // the MMA thread has seen every MMA complete (or a failure)
     fence_after_sync();
-
-    // ------------------------------------------------ epilogue
-    if (!bad) {
+    const bool ok = s_bad == 0;
+    if (ok && tid < kCompute) {
+        const int row = (warp & 3) * 32 + lane, half = warp >> 2;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         float o[32], dn[16];
         tmem_ld32(tO + lane_off + half * 32, o);
         tmem_ld16(tO + lane_off + kDV, dn);
@@ -488,15 +549,11 @@ tcf_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
             for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(o[4 * i] * rcp, o[4 * i + 1] * rcp, o[4 * i + 2] * rcp, o[4 * i + 3] * rcp);
         }
-    } else {
-        if (tid == 0) atomicOr(err, kErrPrefillPipe);
-        // bounded waits for work that may still be in flight
-        wait_bar(&bar_pv[(T - 1) & 1], ((T - 1) >> 1) & 1);
-        if (ro_issued > 0) wait_bar(&bar_ro[(ro_issued - 1) & 1], ((ro_issued - 1) >> 1) & 1);
     }
+    if (!ok && tid == 0) atomicOr(err, kErrPrefillPipe);
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
         fence_after_sync();
         tmem_dealloc(tslot, 256);
     }
@@ -517,12 +574,18 @@ int run(const bf16* q, const bf16* k, const bf16* v, float* out, const float* st
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TAYLOR_ERR_CUDA;
     std::call_once(once[dev], [&]() {
         res[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(tcf_state_kernel<D, N>),
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem<D>::kBytes);
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StSm<D>::kBytes);
         if (res[dev] == cudaSuccess)
             res[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(tcf_out_kernel<D, N>),
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem<D>::kBytes);
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSm<D>::kBytes);
     });
     if (res[dev] != cudaSuccess) return TAYLOR_ERR_CUDA;
+
+    CUtensorMap tmq, tmk, tmv;
+    if (make_tmap_bf16_3d(&tmq, q, D, (uint64_t)Ntok, (uint64_t)BH, 8, kQ) != cudaSuccess ||
+        make_tmap_bf16_3d(&tmk, k, D, (uint64_t)Ntok, (uint64_t)BH, 8, kTok) != cudaSuccess ||
+        make_tmap_bf16_3d(&tmv, v, kDV, (uint64_t)Ntok, (uint64_t)BH, 8, kTok) != cudaSuccess)
+        return kNotApplicable;
 
     // group size: about F tokens (the pairwise work of a query tile then
     // stays below its read-out work), in [128, 2048], no larger than needed
@@ -531,34 +594,45 @@ int run(const bf16* q, const bf16* k, const bf16* v, float* out, const float* st
     while (G > 128 && G / 2 >= Ntok) G /= 2;
     const int NG = (Ntok + G - 1) / G;
     const int NFT = (int)((F + kFT - 1) / kFT);
+    const int R = (int)((F + kRT - 1) / kRT);
     const bool need_ws = NG > 1 || state_in || state_out;
-    float* Wb = nullptr;
+    const int g0 = state_in ? 0 : 1;  // first group whose outputs read a state
+    const bool need_pk = NG > g0;
+    const size_t w_bytes = ((size_t)BH * NG * stride * sizeof(float) + 1023) / 1024 * 1024;
+    const size_t pk_bytes = need_pk ? (size_t)BH * NG * R * kSTile : 0;
+    uint8_t* ws = nullptr;
     if (need_ws) {
-        if (workspace_alloc(reinterpret_cast<void**>(&Wb), (size_t)BH * NG * stride * sizeof(float), stream) !=
-            cudaSuccess) {
+        if (workspace_alloc(reinterpret_cast<void**>(&ws), w_bytes + pk_bytes, stream) != cudaSuccess) {
             cudaGetLastError();
             return TAYLOR_ERR_OUT_OF_MEMORY;
         }
     }
+    float* Wb = reinterpret_cast<float*>(ws);
+    uint8_t* PKb = need_pk ? ws + w_bytes : nullptr;
     cudaError_t e = cudaSuccess;
     if (need_ws) {
         TA_TIMED(stream, "tcf_state_kernel",
-                 tcf_state_kernel<D, N><<<dim3(NG, NFT, BH), kThreads, StateSmem<D>::kBytes, stream>>>(
-                     k, v, Wb, Ntok, n, (int)F, stride, G, NG, err));
+                 tcf_state_kernel<D, N><<<dim3(NG, NFT, BH), kStateThreads, StSm<D>::kBytes, stream>>>(
+                     tmk, tmv, Wb, Ntok, n, (int)F, stride, G, NG, err));
         e = cudaGetLastError();
         if (e == cudaSuccess)
             e = launch_state_scan(Wb, state_in, state_out, BH, NG, stride, F * (kDV + 1), stream, true);
+        if (e == cudaSuccess && need_pk) {
+            TA_TIMED(stream, "tcf_pack_kernel",
+                     e = launch_maybe_pdl(tcf_pack_kernel, dim3(R, NG - g0, BH), dim3(256), 0, stream, true,
+                                          (const float*)Wb, PKb, (int)F, stride, NG, R, g0));
+        }
     }
     if (e == cudaSuccess) {
         const int NQ = (Ntok + kQ - 1) / kQ;
         TA_TIMED(stream, "tcf_out_kernel",
-                 e = launch_maybe_pdl(tcf_out_kernel<D, N>, dim3(NQ, BH), dim3(kThreads), OutSmem<D>::kBytes, stream,
-                                      need_ws, q, k, v, (const float*)Wb, out, Ntok, n, tau, (int)F, stride, G, NG,
+                 e = launch_maybe_pdl(tcf_out_kernel<D, N>, dim3(NQ, BH), dim3(kOutThreads), OutSm<D>::kBytes, stream,
+                                      need_ws, tmq, tmk, tmv, (const uint8_t*)PKb, out, Ntok, n, tau, (int)F, G, NG, R,
                                       state_in != nullptr ? 1 : 0, err));
         if (e == cudaSuccess) e = cudaGetLastError();
     }
-    if (Wb) {
-        const cudaError_t e2 = workspace_free(Wb, stream);
+    if (ws) {
+        const cudaError_t e2 = workspace_free(ws, stream);
         if (e == cudaSuccess) e = e2;
     }
     if (e == cudaSuccess) return TAYLOR_OK;

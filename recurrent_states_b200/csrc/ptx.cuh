@@ -52,6 +52,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     return false;
 }
 
+// Waits for the phase with the given parity, giving up after max_iters
+// polls or as soon as *abort is set (checked every 1024 polls); sets *abort
+// itself on a timeout.  For producer/consumer loops in which one failed wait
+// must not leave the others waiting out their own bounds one after another.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, uint32_t max_iters,
+                                                   volatile int* abort) {
+    for (uint32_t i = 0; i < max_iters; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+// 3-D tiled TMA load (no multicast): box at element coordinates (x, y, z)
+// of the tensor map, completing on an mbarrier.  x * element size must be a
+// multiple of 16 bytes; the destination must be 128-byte aligned.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Global -> shared bulk copy completing on an mbarrier (bytes % 16 == 0,
 // both addresses 16-byte aligned, bytes < 2^20).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

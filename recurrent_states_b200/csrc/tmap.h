@@ -1,0 +1,17 @@
+// Host-side TMA tensor maps (cuTensorMapEncodeTiled, reached through the
+// runtime's driver entry point so that the library does not link libcuda).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ta {
+
+// A bf16 tensor [d2][d1][d0] (d0 innermost, contiguous) with boxes of
+// box0 x box1 x 1 elements, no swizzle, zero fill outside the tensor.
+// Returns cudaErrorInvalidValue when the driver rejects the description.
+cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                              uint32_t box0, uint32_t box1);
+
+}  // namespace ta
