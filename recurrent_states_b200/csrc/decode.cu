@@ -194,10 +194,14 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
 // next head's token are already in flight, so HBM sees a continuous stream
 // instead of one wave of CTAs, a gap, and a partial second wave.
 constexpr int kPersistThreads = 256;
+// Largest shared-memory footprint (two states plus features) that takes the
+// persistent kernel; 0 (the default) keeps every shape on the one-CTA-per-head
+// kernel, which measured faster on the decode workload (64 x 16 heads of
+// 153 x 65 floats).  Two CTAs per SM need at most about 100 KB each.
 #ifndef TA_DECODE_PERSIST_MAX_DYN
-#define TA_DECODE_PERSIST_MAX_DYN (100 * 1024)
+#define TA_DECODE_PERSIST_MAX_DYN 0
 #endif
-constexpr size_t kPersistMaxDyn = TA_DECODE_PERSIST_MAX_DYN;  // two CTAs per SM
+constexpr size_t kPersistMaxDyn = TA_DECODE_PERSIST_MAX_DYN;
 constexpr int kPersistWarps = kPersistThreads / 32;
 constexpr int kPersistDescPerThread = (kTmaMaxFeatures + kPersistThreads - 1) / kPersistThreads;
 
@@ -498,7 +502,7 @@ cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state
     const bool tma_ok = err != nullptr && used_bytes <= kTmaMaxBytes && dyn <= (size_t)kTmaMaxBytes + 8192 &&
                         F <= kTmaMaxFeatures;
     const size_t dyn2 = 2 * (size_t)((bytes + 127u) & ~127u) + 2 * (size_t)((F + 3) & ~3) * 4;
-    if (tma_ok && dyn2 <= kPersistMaxDyn) {
+    if (tma_ok && kPersistMaxDyn > 0 && dyn2 <= kPersistMaxDyn) {
         switch (dv) {
             case 16: return launch_persist<Tin, 4>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn2, err, stream);
             case 32: return launch_persist<Tin, 8>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn2, err, stream);

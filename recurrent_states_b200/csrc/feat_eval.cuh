@@ -1,7 +1,7 @@
 // Evaluation of 32 consecutive packed features of one token inside the
-// tensor-core kernels, from the token's bf16 row held in shared memory in a
-// K-major operand layout: 16-byte chunk c of the row (elements 8c .. 8c+7)
-// at rowbase + c * kCS.
+// tensor-core kernels, from the token's bf16 row held in shared memory as a
+// row of a swizzled K-major operand: 16-byte chunk c of the row (elements
+// 8c .. 8c+7) at rowbase + 16 (c ^ sw).
 //
 // Feature f (degree m, indices i1 <= ... <= im, weight sqrt(m!/alpha!); the
 // packing of arXiv 2610.20637, abstract) is w * x_i1 * ... * x_im, times the
@@ -99,15 +99,15 @@ __device__ __forceinline__ float ct_feature(const uint4 (&ch)[D / 8], const floa
     }
 }
 
-template <uint32_t kMask, int kCS, int C, int NC>
-__device__ __forceinline__ void ct_load_chunk(const uint8_t* rowbase, uint4 (&ch)[NC]) {
-    if constexpr ((kMask >> C) & 1u) ch[C] = *reinterpret_cast<const uint4*>(rowbase + C * kCS);
+template <uint32_t kMask, int C, int NC>
+__device__ __forceinline__ void ct_load_chunk(const uint8_t* rowbase, uint32_t sw, uint4 (&ch)[NC]) {
+    if constexpr ((kMask >> C) & 1u) ch[C] = *reinterpret_cast<const uint4*>(rowbase + ((C ^ sw) << 4));
 }
 
-template <uint32_t kMask, int kCS, int NC, int... C>
-__device__ __forceinline__ void ct_load_chunks(const uint8_t* rowbase, uint4 (&ch)[NC],
+template <uint32_t kMask, int NC, int... C>
+__device__ __forceinline__ void ct_load_chunks(const uint8_t* rowbase, uint32_t sw, uint4 (&ch)[NC],
                                                std::integer_sequence<int, C...>) {
-    (ct_load_chunk<kMask, kCS, C>(rowbase, ch), ...);
+    (ct_load_chunk<kMask, C>(rowbase, sw, ch), ...);
 }
 
 template <int D, int N, bool kQuery, int F0, int... E>
@@ -116,38 +116,38 @@ __device__ __forceinline__ void ct_fill(const uint4 (&ch)[D / 8], const float (&
     ((o[E] = ct_feature<D, N, kQuery, F0 + E>(ch, qc)), ...);
 }
 
-template <int D, int N, bool kQuery, int kCS, int B>
-__device__ __forceinline__ void ct_block(const uint8_t* rowbase, const float (&qc)[N], float (&o)[32]) {
+template <int D, int N, bool kQuery, int B>
+__device__ __forceinline__ void ct_block(const uint8_t* rowbase, uint32_t sw, const float (&qc)[N], float (&o)[32]) {
     constexpr uint32_t kMask = ct_chunk_mask<D>(cx_num_features(D, N), B);
     uint4 ch[D / 8];
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) ch[c] = make_uint4(0, 0, 0, 0);
-    ct_load_chunks<kMask, kCS>(rowbase, ch, std::make_integer_sequence<int, D / 8>{});
+    ct_load_chunks<kMask>(rowbase, sw, ch, std::make_integer_sequence<int, D / 8>{});
     ct_fill<D, N, kQuery, 32 * B>(ch, qc, o, std::make_integer_sequence<int, 32>{});
 }
 
 // Binary dispatch on the run-time block index.
-template <int D, int N, bool kQuery, int kCS, int LO, int HI>
-__device__ __forceinline__ void ct_dispatch(int b, const uint8_t* rowbase, const float (&qc)[N], float (&o)[32]) {
+template <int D, int N, bool kQuery, int LO, int HI>
+__device__ __forceinline__ void ct_dispatch(int b, const uint8_t* rowbase, uint32_t sw, const float (&qc)[N],
+                                            float (&o)[32]) {
     if constexpr (HI - LO == 1) {
-        ct_block<D, N, kQuery, kCS, LO>(rowbase, qc, o);
+        ct_block<D, N, kQuery, LO>(rowbase, sw, qc, o);
     } else {
         constexpr int MID = (LO + HI) / 2;
-        if (b < MID) ct_dispatch<D, N, kQuery, kCS, LO, MID>(b, rowbase, qc, o);
-        else ct_dispatch<D, N, kQuery, kCS, MID, HI>(b, rowbase, qc, o);
+        if (b < MID) ct_dispatch<D, N, kQuery, LO, MID>(b, rowbase, sw, qc, o);
+        else ct_dispatch<D, N, kQuery, MID, HI>(b, rowbase, sw, qc, o);
     }
 }
 
 // ------------------------------------------------------------ run-time path
-template <int kCS>
-__device__ __forceinline__ float rt_x(const uint8_t* rowbase, int i) {
-    const uint16_t h = *reinterpret_cast<const uint16_t*>(rowbase + (i >> 3) * kCS + (i & 7) * 2);
+__device__ __forceinline__ float rt_x(const uint8_t* rowbase, uint32_t sw, int i) {
+    const uint16_t h = *reinterpret_cast<const uint16_t*>(rowbase + ((((uint32_t)i >> 3) ^ sw) << 4) + (i & 7) * 2);
     return __uint_as_float((uint32_t)h << 16);
 }
 
-template <int D, bool kQuery, int kCS>
-__device__ __forceinline__ void rt_block(int b, const uint8_t* rowbase, const float* qc, int n, int F, float tau,
-                                         float (&o)[32]) {
+template <int D, bool kQuery>
+__device__ __forceinline__ void rt_block(int b, const uint8_t* rowbase, uint32_t sw, const float* qc, int n, int F,
+                                         float tau, float (&o)[32]) {
     const PackedFeat* tab = feat_table(D, n);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
@@ -156,7 +156,7 @@ __device__ __forceinline__ void rt_block(int b, const uint8_t* rowbase, const fl
         if (f < F) {
             const FeatDesc fd = get_desc(tab, D, n, f, tau, qc, kQuery);
             c = fd.w;
-            for (int s = 0; s < fd.m; ++s) c *= rt_x<kCS>(rowbase, (fd.packed >> (8 * s)) & 0xff);
+            for (int s = 0; s < fd.m; ++s) c *= rt_x(rowbase, sw, (fd.packed >> (8 * s)) & 0xff);
         }
         o[e] = c;
     }
@@ -166,11 +166,11 @@ __device__ __forceinline__ void rt_block(int b, const uint8_t* rowbase, const fl
 // Features 32b .. 32b+31 of the token at rowbase.  N > 0: compile-time
 // shape (D, N); N == 0: run-time order n (F features).  qc[m] = tau^m/m!
 // (read on the query side only).
-template <int D, int N, bool kQuery, int kCS>
+template <int D, int N, bool kQuery>
 struct Eval {
     static constexpr bool kCompileTime = N > 0;
-    __device__ static __forceinline__ void block(int b, const uint8_t* rowbase, const float* qc, int n, int F,
-                                                 float tau, float (&o)[32]) {
+    __device__ static __forceinline__ void block(int b, const uint8_t* rowbase, uint32_t sw, const float* qc, int n,
+                                                 int F, float tau, float (&o)[32]) {
         if constexpr (N > 0) {
             constexpr int kBlocks = (cx_num_features(D, N) + 31) / 32;
             if (b >= kBlocks) {  // a tile's blocks past the last feature
@@ -181,9 +181,9 @@ struct Eval {
             float q[N];
 #pragma unroll
             for (int m = 0; m < N; ++m) q[m] = kQuery ? qc[m] : 1.f;
-            ct_dispatch<D, N, kQuery, kCS, 0, kBlocks>(b, rowbase, q, o);
+            ct_dispatch<D, N, kQuery, 0, kBlocks>(b, rowbase, sw, q, o);
         } else {
-            rt_block<D, kQuery, kCS>(b, rowbase, qc, n, F, tau, o);
+            rt_block<D, kQuery>(b, rowbase, sw, qc, n, F, tau, o);
         }
     }
 };

@@ -22,8 +22,8 @@
 // v are bf16 already.
 //
 // Both CTA kinds are warp-specialised.  One thread issues TMA tensor loads
-// (q, k, v rows into the K-major / MN-major operand layouts, zero-filled past
-// the sequence), one thread issues every tcgen05.mma, and two warpgroups of
+// (whole q, k, v rows into the swizzled K-major / MN-major operand layouts,
+// zero-filled past the sequence), one thread issues every tcgen05.mma, and two warpgroups of
 // CUDA cores evaluate features (or P) for alternate stages, so that the
 // loads, the tensor cores and the feature arithmetic of different stages run
 // at the same time.  Hand-offs are mbarriers: TMA transaction counts, 128
@@ -61,8 +61,7 @@ constexpr int kNV = 80;       // [V | 1 | 0 ...]
 constexpr int kCompute = 256; // two warpgroups
 constexpr uint32_t kWaitPolls = 1u << 24;
 
-constexpr uint32_t kBox = kTok * 16;             // TMA box of 8 elements x 64 rows (1 KB)
-constexpr uint32_t kV1Bytes = (kNV / 8) * kBox;  // [v|1|0]: 10 column groups of one box each
+constexpr uint32_t kVAtom = kTok * 128;         // 64 token rows of 64 v columns, 128-byte swizzle (8 KB)
 constexpr uint32_t kPhiBytes = kTok * kFT * 2;   // state-stage Phi_K, hi or lo
 constexpr uint32_t kLboFT = (kFT / 8) * 128;     // its K-group stride
 constexpr uint32_t kPBytes = kQ * kRT * 2;       // P or Phi_Q tile, hi or lo: K-major [128][64]
@@ -88,26 +87,44 @@ __device__ __forceinline__ void store_split8(const float* x, uint8_t* hi_dst, ui
     *reinterpret_cast<uint4*>(lo_dst) = lo;
 }
 
-// [v | 1 | 0] operand, MN-major [K = 64 tokens][N = 80] with token rows of
-// 16 bytes (K-group stride 128) and one 1 KB box per 8 columns (N-group
-// stride kBox).  TMA fills groups 0..7; group 8 holds the ones column and
-// group 9 zeros, written once.
-__device__ __forceinline__ void init_v1_tail(uint8_t* v1, int tid, int nthreads) {
-    for (int i = tid; i < 2 * kTok; i += nthreads) {
-        const int g = 8 + i / kTok, k = i % kTok;
-        *reinterpret_cast<uint4*>(v1 + g * kBox + k * 16) = make_uint4(g == 8 ? 0x3F80u : 0u, 0, 0, 0);
+// q and k rows as TMA writes them: K-major operands with D-element rows
+// (32, 64 or 128 bytes) under the matching swizzle.
+template <int D>
+struct RowSw {
+    static constexpr uint32_t kRowBytes = D * 2;
+    static constexpr uint32_t kLayout = D == 64 ? kSwizzle128 : D == 32 ? kSwizzle64 : kSwizzle32;
+    static constexpr uint32_t kSbo = 8 * kRowBytes;
+};
+
+// The [v | 1 | 0] operand is MN-major [K = 64 tokens][N = 80] under the
+// 128-byte swizzle: atom 0 (columns 0..63) is a slot that TMA fills with v
+// rows; atom 1 (columns 64..127, of which the MMA reads 64..79) is one ones
+// atom shared by every slot, reached through the descriptor's LBO: column 64
+// is 1 and the rest 0, in every token row.
+__device__ __forceinline__ void init_ones_atom(uint8_t* atom, int tid, int nthreads) {
+    for (int i = tid; i < kTok * 8; i += nthreads) {
+        const int k = i >> 3, c = i & 7;
+        *reinterpret_cast<uint4*>(atom + k * 128 + ((c ^ (k & 7)) << 4)) = make_uint4(c == 0 ? 0x3F80u : 0u, 0, 0, 0);
     }
 }
 
 // ---------------------------------------------------------------- 1. group states
+// Shared memory: four Phi_K slots (stage s uses slot s % 4 and belongs to
+// warpgroup s & 1), four v slots beside them plus the ones atom, and a
+// separate ring of six k-row slots, released as soon as a warpgroup has read
+// its rows, so that k loads run several stages ahead of the evaluation.
 template <int D>
 struct StSm {
-    static constexpr uint32_t kK = kTok * D * 2;  // k rows, K-major, chunk stride kBox
-    static constexpr uint32_t kStage = 2 * kPhiBytes + kV1Bytes + kK;
-    static constexpr int kStages = 4;             // stage b always belongs to warpgroup b & 1
-    static constexpr uint32_t kBytes = kStages * kStage + 1024;
+    static constexpr int kSlots = 4;
+    static constexpr int kKSlots = 6;
+    static constexpr uint32_t kK = kTok * D * 2;  // k rows, swizzled K-major
+    static constexpr uint32_t kPhiBase = 0;
+    static constexpr uint32_t kV1Base = kSlots * 2 * kPhiBytes;
+    static constexpr uint32_t kOnes = kV1Base + kSlots * kVAtom;
+    static constexpr uint32_t kKBase = kOnes + kVAtom;
+    static constexpr uint32_t kBytes = kKBase + kKSlots * kK + 1024;
     static constexpr int kOutStride = kDV + 4;    // epilogue staging rows: 16-byte aligned, float4 conflict-free
-    static_assert(kFT * kOutStride * 4 <= kStage, "epilogue staging fits one stage");
+    static_assert(kFT * kOutStride * 4 <= kV1Base, "epilogue staging fits the Phi_K slots");
 };
 constexpr int kStateThreads = kCompute + 32;
 
@@ -117,9 +134,10 @@ tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                  float* __restrict__ W, int Ntok, int n, int F, int64_t stride, int G, int NG,
                  unsigned int* __restrict__ err) {
     using L = StSm<D>;
+    constexpr int S4 = L::kSlots, KS = L::kKSlots;
     extern __shared__ uint8_t sm_raw[];
     uint8_t* sm = align1k(sm_raw);
-    __shared__ __align__(8) uint64_t loaded[L::kStages], full[L::kStages], empty[L::kStages];
+    __shared__ __align__(8) uint64_t kload[KS], kfree[KS], vload[S4], full[S4], empty[S4];
     __shared__ uint32_t tslot;
     __shared__ int s_bad;
     volatile int* bad = &s_bad;
@@ -131,11 +149,17 @@ tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const int64_t gt0 = (int64_t)g * G;
     const int gn = (int)min64(G, (int64_t)Ntok - gt0);
     const int nsub = (gn + kTok - 1) / kTok;
-    auto stage = [&](int b) { return sm + b * L::kStage; };
+    auto phi = [&](int b) { return sm + L::kPhiBase + b * 2 * kPhiBytes; };
+    auto v1s = [&](int b) { return sm + L::kV1Base + b * kVAtom; };
+    auto krows = [&](int b) { return sm + L::kKBase + b * L::kK; };
 
     if (tid == 0) {
-        for (int i = 0; i < L::kStages; ++i) {
-            ptx::mbar_init(&loaded[i], 1);
+        for (int i = 0; i < KS; ++i) {
+            ptx::mbar_init(&kload[i], 1);
+            ptx::mbar_init(&kfree[i], kCompute / 2);
+        }
+        for (int i = 0; i < S4; ++i) {
+            ptx::mbar_init(&vload[i], 1);
             ptx::mbar_init(&full[i], kCompute / 2);
             ptx::mbar_init(&empty[i], 1);
         }
@@ -146,7 +170,7 @@ tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
-    for (int b = 0; b < L::kStages; ++b) init_v1_tail(stage(b) + 2 * kPhiBytes, tid, kStateThreads);
+    init_ones_atom(sm + L::kOnes, tid, kStateThreads);
     ptx::fence_proxy_async_smem();
     fence_before_sync();
     __syncthreads();
@@ -155,68 +179,82 @@ tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 
     if (warp == kCompute / 32) {
         if (lane == 0) {
-            // TMA producer and MMA issuer
-            int ld = 0, mm = 0;
-            for (int s = 0; s < nsub && !*bad; ++s) {
-                while (ld < nsub && ld < s + L::kStages) {
-                    const int b = ld % L::kStages;
-                    if (ld >= L::kStages && !waitb(&empty[b], ((ld / L::kStages) - 1) & 1, bad)) break;
-                    uint8_t* st = stage(b);
-                    ptx::mbar_arrive_expect_tx(&loaded[b], (uint32_t)(D / 8 + 8) * kBox);
-                    const int y = (int)(gt0 + (int64_t)ld * kTok);
-#pragma unroll
-                    for (int c = 0; c < D / 8; ++c)
-                        ptx::tma_load_3d(st + 2 * kPhiBytes + kV1Bytes + c * kBox, &tmk, c * 8, y, bh, &loaded[b]);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        ptx::tma_load_3d(st + 2 * kPhiBytes + c * kBox, &tmv, c * 8, y, bh, &loaded[b]);
-                    ++ld;
+            // TMA producer and MMA issuer: issue whatever is ready, in order
+            // within each kind (k loads, v loads, MMAs of a stage)
+            int nk = 0, nv = 0, nm = 0;
+            uint32_t idle = 0;
+            while (nm < nsub) {
+                bool prog = false;
+                if (nk < nsub && (nk < KS || ptx::mbar_test(&kfree[nk % KS], ((nk / KS) - 1) & 1))) {
+                    ptx::mbar_arrive_expect_tx(&kload[nk % KS], L::kK);
+                    ptx::tma_load_3d(krows(nk % KS), &tmk, 0, (int)(gt0 + (int64_t)nk * kTok), bh, &kload[nk % KS]);
+                    ++nk;
+                    prog = true;
                 }
-                if (*bad) break;
-                const int b = s % L::kStages;
-                if (!waitb(&full[b], (s / L::kStages) & 1, bad)) break;
-                fence_after_sync();
-                uint8_t* st = stage(b);
-                const uint32_t id = idesc_bf16(kFT, kNV, 1, 1);
-#pragma unroll
-                for (int ks = 0; ks < kTok / 16; ++ks) {
-                    const uint64_t bd = smem_desc(st + 2 * kPhiBytes + ks * 256, 128, kBox);
-                    mma_bf16(tacc, smem_desc(st + ks * 2 * kLboFT, kLboFT, 128), bd, id, (s > 0 || ks > 0) ? 1u : 0u);
-                    mma_bf16(tacc, smem_desc(st + kPhiBytes + ks * 2 * kLboFT, kLboFT, 128), bd, id, 1u);
+                if (nv < nsub && (nv < S4 || ptx::mbar_test(&empty[nv % S4], ((nv / S4) - 1) & 1))) {
+                    ptx::mbar_arrive_expect_tx(&vload[nv % S4], kVAtom);
+                    ptx::tma_load_3d(v1s(nv % S4), &tmv, 0, (int)(gt0 + (int64_t)nv * kTok), bh, &vload[nv % S4]);
+                    ++nv;
+                    prog = true;
                 }
-                mma_commit(&empty[b]);
-                mm = s + 1;
+                if (nm < nv && ptx::mbar_test(&full[nm % S4], (nm / S4) & 1) &&
+                    ptx::mbar_test(&vload[nm % S4], (nm / S4) & 1)) {
+                    fence_after_sync();
+                    const uint8_t* ph = phi(nm % S4);
+                    const uint8_t* vb = v1s(nm % S4);
+                    const uint32_t lbo = (uint32_t)(L::kOnes - (L::kV1Base + (nm % S4) * kVAtom));
+                    const uint32_t id = idesc_bf16(kFT, kNV, 1, 1);
+#pragma unroll
+                    for (int ks = 0; ks < kTok / 16; ++ks) {
+                        const uint64_t bd = smem_desc_sw(vb + ks * 2048, lbo, 1024, kSwizzle128);
+                        mma_bf16(tacc, smem_desc(ph + ks * 2 * kLboFT, kLboFT, 128), bd, id,
+                                 (nm > 0 || ks > 0) ? 1u : 0u);
+                        mma_bf16(tacc, smem_desc(ph + kPhiBytes + ks * 2 * kLboFT, kLboFT, 128), bd, id, 1u);
+                    }
+                    mma_commit(&empty[nm % S4]);
+                    ++nm;
+                    prog = true;
+                }
+                if (prog) {
+                    idle = 0;
+                } else if (++idle > kWaitPolls || *bad) {
+                    *bad = 1;
+                    break;
+                }
             }
-            // the last commit covers every MMA issued; loads issued but never
+            // the last commit covers every MMA issued; copies issued but never
             // consumed (only after a failure) must land before the CTA leaves
-            if (mm > 0 && !ptx::mbar_wait(&empty[(mm - 1) % L::kStages], ((mm - 1) / L::kStages) & 1, kWaitPolls))
-                *bad = 1;
-            for (int li = mm; li < ld; ++li)
-                ptx::mbar_wait(&loaded[li % L::kStages], (li / L::kStages) & 1, kWaitPolls);
+            if (nm > 0 && !ptx::mbar_wait(&empty[(nm - 1) % S4], ((nm - 1) / S4) & 1, kWaitPolls)) *bad = 1;
+            for (int i = (nk > KS ? nk - KS : 0); i < nk; ++i)
+                ptx::mbar_wait(&kload[i % KS], (i / KS) & 1, kWaitPolls);
+            for (int i = (nv > S4 ? nv - S4 : 0); i < nv; ++i)
+                ptx::mbar_wait(&vload[i % S4], (i / S4) & 1, kWaitPolls);
         }
     } else {
         // warpgroup w evaluates the features of stages w, w + 2, ...:
         // token t, features [64 h, 64 h + 64) of the tile
         const int w = warp >> 2, wt = tid & 127, t = wt & (kTok - 1), h = wt >> 6;
         for (int s = w; s < nsub; s += 2) {
-            const int b = s % L::kStages;
-            if (!waitb(&loaded[b], (s / L::kStages) & 1, bad)) break;
-            uint8_t* st = stage(b);
-            const int valid = min(kTok, gn - s * kTok);
-            const uint8_t* rowbase = st + 2 * kPhiBytes + kV1Bytes + t * 16;
+            const int kb = s % KS, b = s % S4;
+            if (!waitb(&kload[kb], (s / KS) & 1, bad)) break;
+            float o[64];
+            const uint8_t* rowbase = krows(kb) + t * RowSw<D>::kRowBytes;
+            const uint32_t sw = swizzle_of_row(t, RowSw<D>::kRowBytes);
+            fe::Eval<D, N, false>::block(ft * 4 + h * 2, rowbase, sw, nullptr, n, F, 0.f,
+                                         *reinterpret_cast<float(*)[32]>(o));
+            fe::Eval<D, N, false>::block(ft * 4 + h * 2 + 1, rowbase, sw, nullptr, n, F, 0.f,
+                                         *reinterpret_cast<float(*)[32]>(o + 32));
+            ptx::mbar_arrive(&kfree[kb]);
+            if (t >= min(kTok, gn - s * kTok)) {  // zero-filled rows past the sequence: phi(0) has a constant feature
 #pragma unroll
-            for (int sub = 0; sub < 2; ++sub) {
-                float o[32];
-                fe::Eval<D, N, false, kBox>::block(ft * 4 + h * 2 + sub, rowbase, nullptr, n, F, 0.f, o);
-                if (t >= valid) {  // zero-filled rows past the sequence: phi(0) has a constant feature
+                for (int e = 0; e < 64; ++e) o[e] = 0.f;
+            }
+            if (s >= S4 && !waitb(&empty[b], ((s / S4) - 1) & 1, bad)) break;
+            uint8_t* ph = phi(b);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0.f;
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t off = mnmaj(t, h * 8 + sub * 4 + i, kLboFT);
-                    store_split8(o + 8 * i, st + off, st + kPhiBytes + off);
-                }
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t off = mnmaj(t, h * 8 + i, kLboFT);
+                store_split8(o + 8 * i, ph + off, ph + kPhiBytes + off);
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&full[b]);
@@ -291,12 +329,13 @@ tcf_pack_kernel(const float* __restrict__ W, uint8_t* __restrict__ PK, int F, in
 // ---------------------------------------------------------------- 4. outputs
 template <int D>
 struct OutSm {
-    static constexpr uint32_t kQop = kQ * D * 2;  // Q, K-major, chunk stride kQ * 16
-    static constexpr uint32_t kKt = kTok * D * 2; // key tile, K-major, chunk stride kBox
-    static constexpr uint32_t kKV = kKt + kV1Bytes;
-    static constexpr int kKVSlots = 3, kSSlots = 3;
+    static constexpr uint32_t kQop = kQ * D * 2;  // Q, swizzled K-major
+    static constexpr uint32_t kKt = kTok * D * 2; // key tile, swizzled K-major
+    static constexpr uint32_t kKV = kKt + kVAtom;
+    static constexpr int kKVSlots = 4, kSSlots = 3;
     static constexpr uint32_t kKVbase = kQop;
-    static constexpr uint32_t kSbase = kKVbase + kKVSlots * kKV;
+    static constexpr uint32_t kOnes = kKVbase + kKVSlots * kKV;
+    static constexpr uint32_t kSbase = kOnes + kVAtom;
     static constexpr uint32_t kPPbase = kSbase + kSSlots * kSTile;
     static constexpr uint32_t kPP = 2 * kPBytes;  // P or Phi_Q, hi then lo, one per warpgroup
     static constexpr uint32_t kBytes = kPPbase + 2 * kPP + 1024;
@@ -312,8 +351,8 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     using L = OutSm<D>;
     extern __shared__ uint8_t sm_raw[];
     uint8_t* sm = align1k(sm_raw);
-    __shared__ __align__(8) uint64_t q_loaded, kv_loaded[L::kKVSlots], kv_empty[L::kKVSlots], sc_full[2], pp_full[2],
-        pp_free[2], s_loaded[L::kSSlots], s_empty[L::kSSlots], o_done;
+    __shared__ __align__(8) uint64_t q_loaded, kv_loaded[L::kKVSlots], kv_empty[L::kKVSlots], sc_full[2], sc_free[2],
+        pp_full[2], pp_free[2], s_loaded[L::kSSlots], s_empty[L::kSSlots], o_done;
     __shared__ uint32_t tslot;
     __shared__ int s_bad;
     volatile int* bad = &s_bad;
@@ -340,6 +379,7 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&sc_full[i], 1);
+            ptx::mbar_init(&sc_free[i], kCompute / 2);
             ptx::mbar_init(&pp_full[i], kCompute / 2);
             ptx::mbar_init(&pp_free[i], 1);
         }
@@ -355,7 +395,7 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         tmem_alloc(&tslot, 256);
         tmem_relinquish();
     }
-    for (int s = 0; s < L::kKVSlots; ++s) init_v1_tail(kv(s) + L::kKt, tid, kOutThreads);
+    init_ones_atom(sm + L::kOnes, tid, kOutThreads);
     ptx::fence_proxy_async_smem();
     fence_before_sync();
     __syncthreads();
@@ -366,19 +406,16 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         if (lane == 0) {
             // q once, then key/value tiles through a ring of three slots
             ptx::mbar_arrive_expect_tx(&q_loaded, L::kQop);
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c) ptx::tma_load_3d(sQ + c * (kQ * 16), &tmq, c * 8, (int)q0, bh, &q_loaded);
+            ptx::tma_load_3d(sQ, &tmq, 0, (int)q0, bh, &q_loaded);
             int ld = 0;
             for (; ld < T; ++ld) {
                 const int slot = ld % L::kKVSlots;
                 if (ld >= L::kKVSlots && !waitb(&kv_empty[slot], ((ld / L::kKVSlots) - 1) & 1, bad)) break;
                 uint8_t* st = kv(slot);
-                ptx::mbar_arrive_expect_tx(&kv_loaded[slot], (uint32_t)(D / 8 + 8) * kBox);
+                ptx::mbar_arrive_expect_tx(&kv_loaded[slot], L::kKV);
                 const int y = (int)(gs + (int64_t)ld * kTok);
-#pragma unroll
-                for (int c = 0; c < D / 8; ++c) ptx::tma_load_3d(st + c * kBox, &tmk, c * 8, y, bh, &kv_loaded[slot]);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) ptx::tma_load_3d(st + L::kKt + c * kBox, &tmv, c * 8, y, bh, &kv_loaded[slot]);
+                ptx::tma_load_3d(st, &tmk, 0, y, bh, &kv_loaded[slot]);
+                ptx::tma_load_3d(st + L::kKt, &tmv, 0, y, bh, &kv_loaded[slot]);
             }
             // every issued copy lands before the CTA can leave
             ptx::mbar_wait(&q_loaded, 0, kWaitPolls);
@@ -404,7 +441,7 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     } else if (warp == 8) {
         if (lane == 0) {
             // every tcgen05.mma of the CTA, in order
-            constexpr uint32_t kSboQ = 128;
+            using RS = RowSw<D>;
             auto scores = [&](int t) -> bool {
                 const int slot = t % L::kKVSlots;
                 if (!waitb(&kv_loaded[slot], (t / L::kKVSlots) & 1, bad)) return false;
@@ -412,8 +449,8 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 const uint32_t id = idesc_bf16(kQ, kTok, 0, 0);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    mma_bf16(tS + (t & 1) * kTok, smem_desc(sQ + ks * 2 * (kQ * 16), kQ * 16, kSboQ),
-                             smem_desc(kv(slot) + ks * 2 * kBox, kBox, kSboQ), id, ks > 0 ? 1u : 0u);
+                    mma_bf16(tS + (t & 1) * kTok, smem_desc_sw(sQ + ks * 32, 16, RS::kSbo, RS::kLayout),
+                             smem_desc_sw(kv(slot) + ks * 32, 16, RS::kSbo, RS::kLayout), id, ks > 0 ? 1u : 0u);
                 mma_commit(&sc_full[t & 1]);
                 return true;
             };
@@ -422,23 +459,38 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             if (go && T > 1) go = scores(1);
             for (int t = 0; t < T && go; ++t) {
                 const int w = t & 1;
-                if (!waitb(&pp_full[w], (t >> 1) & 1, bad)) {
+                // scores of tile t + 2 go ahead of PV(t) when its warpgroup has
+                // read the scores of tile t and the key tile is resident (they
+                // write different TMEM, so the order does not change results)
+                bool early = false;
+                if (t + 2 < T) {
+                    if (!waitb(&sc_free[w], (t >> 1) & 1, bad)) {
+                        go = false;
+                        break;
+                    }
+                    if (ptx::mbar_test(&kv_loaded[(t + 2) % L::kKVSlots], ((t + 2) / L::kKVSlots) & 1)) {
+                        go = scores(t + 2);
+                        early = true;
+                    }
+                }
+                if (!go || !waitb(&pp_full[w], (t >> 1) & 1, bad)) {
                     go = false;
                     break;
                 }
                 fence_after_sync();
                 const uint8_t* p = pp(w);
                 const uint8_t* v1 = kv(t % L::kKVSlots) + L::kKt;
+                const uint32_t lbo = (uint32_t)(L::kOnes - (L::kKVbase + (t % L::kKVSlots) * L::kKV + L::kKt));
                 const uint32_t id = idesc_bf16(kQ, kNV, 0, 1);
 #pragma unroll
                 for (int ks = 0; ks < kTok / 16; ++ks) {
-                    const uint64_t bd = smem_desc(v1 + ks * 256, 128, kBox);
+                    const uint64_t bd = smem_desc_sw(v1 + ks * 2048, lbo, 1024, kSwizzle128);
                     mma_bf16(tO, smem_desc(p + ks * 256, 128, kSbo64), bd, id, (t > 0 || ks > 0) ? 1u : 0u);
                     mma_bf16(tO, smem_desc(p + kPBytes + ks * 256, 128, kSbo64), bd, id, 1u);
                 }
                 mma_commit(&pp_free[w]);
                 mma_commit(&kv_empty[t % L::kKVSlots]);
-                if (t + 2 < T) go = scores(t + 2);
+                if (t + 2 < T && !early) go = scores(t + 2);
             }
             const int nuse[2] = {(T + 1) / 2, T / 2};
             for (int r = 0; r < Rr && go; ++r) {
@@ -486,6 +538,8 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             tmem_ld32(tS + lane_off + w * kTok, *reinterpret_cast<float(*)[32]>(s));
             tmem_ld32(tS + lane_off + w * kTok + 32, *reinterpret_cast<float(*)[32]>(s + 32));
             tmem_ld_wait();
+            fence_before_sync();
+            ptx::mbar_arrive(&sc_free[w]);
             const int64_t k0 = gs + (int64_t)t * kTok;
             const bool mask = k0 + kTok - 1 > q0 || k0 + kTok > Ntok;
 #pragma unroll
@@ -503,7 +557,6 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 if (mask && !(k0 + j <= qi && k0 + j < kend)) p = 0.f;
                 s[j] = p;
             }
-            fence_before_sync();
             if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
 #pragma unroll
             for (int kg = 0; kg < 8; ++kg) {
@@ -514,13 +567,13 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             ptx::mbar_arrive(&pp_full[w]);
         }
         if (!*bad) {
-            const uint8_t* rowbase = sQ + row * 16;
+            const uint8_t* rowbase = sQ + row * RowSw<D>::kRowBytes;
+            const uint32_t sw = swizzle_of_row(row, RowSw<D>::kRowBytes);
             for (int r = w; r < Rr; r += 2, ++u) {
                 float o[64];
-                fe::Eval<D, N, true, kQ * 16>::block(r * 2, rowbase, qc, n, F, tau,
-                                                       *reinterpret_cast<float(*)[32]>(o));
-                fe::Eval<D, N, true, kQ * 16>::block(r * 2 + 1, rowbase, qc, n, F, tau,
-                                                       *reinterpret_cast<float(*)[32]>(o + 32));
+                fe::Eval<D, N, true>::block(r * 2, rowbase, sw, qc, n, F, tau, *reinterpret_cast<float(*)[32]>(o));
+                fe::Eval<D, N, true>::block(r * 2 + 1, rowbase, sw, qc, n, F, tau,
+                                            *reinterpret_cast<float(*)[32]>(o + 32));
                 if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
 #pragma unroll
                 for (int kg = 0; kg < 8; ++kg) {
@@ -582,9 +635,9 @@ int run(const bf16* q, const bf16* k, const bf16* v, float* out, const float* st
     if (res[dev] != cudaSuccess) return TAYLOR_ERR_CUDA;
 
     CUtensorMap tmq, tmk, tmv;
-    if (make_tmap_bf16_3d(&tmq, q, D, (uint64_t)Ntok, (uint64_t)BH, 8, kQ) != cudaSuccess ||
-        make_tmap_bf16_3d(&tmk, k, D, (uint64_t)Ntok, (uint64_t)BH, 8, kTok) != cudaSuccess ||
-        make_tmap_bf16_3d(&tmv, v, kDV, (uint64_t)Ntok, (uint64_t)BH, 8, kTok) != cudaSuccess)
+    if (make_tmap_bf16_3d(&tmq, q, D, (uint64_t)Ntok, (uint64_t)BH, D, kQ, D * 2) != cudaSuccess ||
+        make_tmap_bf16_3d(&tmk, k, D, (uint64_t)Ntok, (uint64_t)BH, D, kTok, D * 2) != cudaSuccess ||
+        make_tmap_bf16_3d(&tmv, v, kDV, (uint64_t)Ntok, (uint64_t)BH, kDV, kTok, 128) != cudaSuccess)
         return kNotApplicable;
 
     // group size: about F tokens (the pairwise work of a query tile then

@@ -35,6 +35,24 @@ __device__ __forceinline__ uint64_t smem_desc(const void* start, uint32_t lbo_by
     return d;
 }
 
+// Swizzled layouts (the forms TMA writes with CU_TENSOR_MAP_SWIZZLE_*):
+// rows of 32, 64 or 128 bytes whose 16-byte chunks are XOR-permuted by
+// address bits 7.. (chunk c of row r lands at chunk c ^ sw(r)); the atom
+// base must be 1024-byte aligned.  K-major: LBO is unused, SBO = 8 rows.
+// MN-major (128 B): LBO = stride between 64-element atoms along MN, SBO =
+// stride between groups of 8 K rows.
+enum : uint32_t { kSwizzleNone = 0, kSwizzle128 = 2, kSwizzle64 = 4, kSwizzle32 = 6 };
+
+__device__ __forceinline__ uint64_t smem_desc_sw(const void* start, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                                 uint32_t layout) {
+    return smem_desc(start, lbo_bytes, sbo_bytes) | ((uint64_t)layout << 61);
+}
+
+// Chunk permutation of row r in a swizzled layout with row_bytes-wide rows.
+__host__ __device__ constexpr uint32_t swizzle_of_row(uint32_t r, uint32_t row_bytes) {
+    return ((r * row_bytes) >> 7) & (row_bytes / 16 - 1);
+}
+
 // Instruction descriptor for kind::f16: bf16 A and B, fp32 accumulator,
 // M x N tile, each operand K-major (0) or MN-major (1).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
