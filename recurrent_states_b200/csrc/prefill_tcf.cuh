@@ -26,8 +26,13 @@
 // zero-filled past the sequence), one thread issues every tcgen05.mma, and two warpgroups of
 // CUDA cores evaluate features (or P) for alternate stages, so that the
 // loads, the tensor cores and the feature arithmetic of different stages run
-// at the same time.  Hand-offs are mbarriers: TMA transaction counts, 128
-// arrivals from a warpgroup, or tcgen05.commit.  Every wait is bounded and a
+// at the same time.  In the output kernel the operands the CUDA cores produce
+// (P and Phi_Q, hi/lo) go to TMEM with tcgen05.st and the MMAs read them from
+// there (A in TMEM, B in shared memory), which keeps the tensor cores' shared
+// memory reads to the B operand: with N = 80 an MMA reading A from shared
+// memory as well would need more bytes per cycle than shared memory gives.
+// Hand-offs are mbarriers: TMA transaction counts, 128 arrivals from a
+// warpgroup, or tcgen05.commit.  Every wait is bounded and a
 // failed wait stops the other roles' waits too; a device error bit records it.
 #pragma once
 
@@ -40,6 +45,7 @@
 #include "feat_eval.cuh"
 #include "feature_table.cuh"
 #include "internal.h"
+#include "phase.cuh"
 #include "prefill_tc.h"
 #include "ptx.cuh"
 #include "tcgen05.cuh"
@@ -64,11 +70,8 @@ constexpr uint32_t kWaitPolls = 1u << 24;
 constexpr uint32_t kVAtom = kTok * 128;         // 64 token rows of 64 v columns, 128-byte swizzle (8 KB)
 constexpr uint32_t kPhiBytes = kTok * kFT * 2;   // state-stage Phi_K, hi or lo
 constexpr uint32_t kLboFT = (kFT / 8) * 128;     // its K-group stride
-constexpr uint32_t kPBytes = kQ * kRT * 2;       // P or Phi_Q tile, hi or lo: K-major [128][64]
-constexpr uint32_t kSbo64 = 8 * 128;             // its row-group stride
-constexpr uint32_t kLboNV = (kNV / 8) * 128;     // K-group stride of a packed S tile
-constexpr uint32_t kSHalf = kRT * kNV * 2;       // packed S tile, hi or lo
-constexpr uint32_t kSTile = 2 * kSHalf;          // packed S tile, hi then lo (20 KB)
+constexpr uint32_t kLboS = (2 * kNV / 8) * 128;  // K-group stride of a packed S tile
+constexpr uint32_t kSTile = kRT * 2 * kNV * 2;   // packed S tile [64 features][hi 80 | lo 80] (20 KB)
 
 __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, volatile int* bad) {
     return ptx::mbar_wait_or_abort(bar, parity, kWaitPolls, bad);
@@ -77,6 +80,13 @@ __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, volatile i
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
     const uint32_t a = ptx::smem_u32(p);
     return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// 64 fp32 values -> hi/lo bf16 pairs, K order, as 32 + 32 words of a TMEM
+// A-operand row.
+__device__ __forceinline__ void split64_words(const float* x, uint32_t (&hi)[32], uint32_t (&lo)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) split2(x[2 * i], x[2 * i + 1], hi[i], lo[i]);
 }
 
 // Eight fp32 values -> hi/lo bf16 chunks stored at two operand addresses.
@@ -201,15 +211,15 @@ tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     ptx::mbar_test(&vload[nm % S4], (nm / S4) & 1)) {
                     fence_after_sync();
                     const uint8_t* ph = phi(nm % S4);
-                    const uint8_t* vb = v1s(nm % S4);
                     const uint32_t lbo = (uint32_t)(L::kOnes - (L::kV1Base + (nm % S4) * kVAtom));
+                    const uint64_t ahd = smem_desc(ph, kLboFT, 128), ald = smem_desc(ph + kPhiBytes, kLboFT, 128);
+                    const uint64_t bd = smem_desc_sw(v1s(nm % S4), lbo, 1024, kSwizzle128);
                     const uint32_t id = idesc_bf16(kFT, kNV, 1, 1);
+                    // descriptors advance by constants: 2 K groups of Phi_K, 16 token rows of v
 #pragma unroll
                     for (int ks = 0; ks < kTok / 16; ++ks) {
-                        const uint64_t bd = smem_desc_sw(vb + ks * 2048, lbo, 1024, kSwizzle128);
-                        mma_bf16(tacc, smem_desc(ph + ks * 2 * kLboFT, kLboFT, 128), bd, id,
-                                 (nm > 0 || ks > 0) ? 1u : 0u);
-                        mma_bf16(tacc, smem_desc(ph + kPhiBytes + ks * 2 * kLboFT, kLboFT, 128), bd, id, 1u);
+                        mma_bf16(tacc, ahd + (2 * kLboFT / 16) * ks, bd + 128 * ks, id, (nm > 0 || ks > 0) ? 1u : 0u);
+                        mma_bf16(tacc, ald + (2 * kLboFT / 16) * ks, bd + 128 * ks, id, 1u);
                     }
                     mma_commit(&empty[nm % S4]);
                     ++nm;
@@ -297,9 +307,9 @@ tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 }
 
 // ---------------------------------------------------------------- 3. read-out operand tiles
-// S_<g (fp32, the library's state layout) -> for each 64-feature tile r:
-// hi then lo bf16 [K = 64 features][N = 80] MN-major (K-group stride 1280 B),
-// column 64 the z entry, columns 65..79 and features past F zero.
+// S_<g (fp32, the library's state layout) -> for each 64-feature tile r one
+// MN-major bf16 operand [K = 64 features][N = 160]: columns 0..79 the hi
+// parts, 80..159 the lo parts, of [S_v row | z | 0 ...]; features past F zero.
 __global__ void __launch_bounds__(256)
 tcf_pack_kernel(const float* __restrict__ W, uint8_t* __restrict__ PK, int F, int64_t stride, int NG, int R,
                 int g0) {
@@ -321,8 +331,7 @@ tcf_pack_kernel(const float* __restrict__ W, uint8_t* __restrict__ PK, int F, in
                 x[0] = __ldg(S + (int64_t)F * kDV + f);
             }
         }
-        const uint32_t off = mnmaj(j, gq, kLboNV);
-        store_split8(x, dst + off, dst + kSHalf + off);
+        store_split8(x, dst + mnmaj(j, gq, kLboS), dst + mnmaj(j, 10 + gq, kLboS));
     }
 }
 
@@ -332,15 +341,19 @@ struct OutSm {
     static constexpr uint32_t kQop = kQ * D * 2;  // Q, swizzled K-major
     static constexpr uint32_t kKt = kTok * D * 2; // key tile, swizzled K-major
     static constexpr uint32_t kKV = kKt + kVAtom;
-    static constexpr int kKVSlots = 4, kSSlots = 3;
+    static constexpr int kKVSlots = 4, kSSlots = 4;
     static constexpr uint32_t kKVbase = kQop;
     static constexpr uint32_t kOnes = kKVbase + kKVSlots * kKV;
     static constexpr uint32_t kSbase = kOnes + kVAtom;
-    static constexpr uint32_t kPPbase = kSbase + kSSlots * kSTile;
-    static constexpr uint32_t kPP = 2 * kPBytes;  // P or Phi_Q, hi then lo, one per warpgroup
-    static constexpr uint32_t kBytes = kPPbase + 2 * kPP + 1024;
+    static constexpr uint32_t kBytes = kSbase + kSSlots * kSTile + 1024;
 };
-constexpr int kOutThreads = kCompute + 96;  // + MMA warp, q/k/v producer warp, S producer warp
+// two warpgroups of eight warps (two per TMEM lane quadrant, each taking half
+// of a tile's columns), then the hi-operand PV/read-out MMA warp, the q/k/v
+// and S producer warps, and the warp that issues the scores MMAs and the
+// lo-operand PV/read-out MMAs
+constexpr int kOutCompute = 512;
+constexpr int kOutThreads = kOutCompute + 128;
+constexpr int kWMma = kOutCompute / 32, kWLoad = kWMma + 1, kWSLoad = kWMma + 2, kWMma2 = kWMma + 3;
 
 template <int D, int N>
 __global__ void __launch_bounds__(kOutThreads, 1)
@@ -352,14 +365,13 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     extern __shared__ uint8_t sm_raw[];
     uint8_t* sm = align1k(sm_raw);
     __shared__ __align__(8) uint64_t q_loaded, kv_loaded[L::kKVSlots], kv_empty[L::kKVSlots], sc_full[2], sc_free[2],
-        pp_full[2], pp_free[2], s_loaded[L::kSSlots], s_empty[L::kSSlots], o_done;
+        pp_full[2], pp_free[2], s_loaded[L::kSSlots], s_empty[L::kSSlots], o_done[2];
     __shared__ uint32_t tslot;
     __shared__ int s_bad;
     volatile int* bad = &s_bad;
     uint8_t* sQ = sm;
     auto kv = [&](int slot) { return sm + L::kKVbase + slot * L::kKV; };
     auto sS = [&](int slot) { return sm + L::kSbase + slot * kSTile; };
-    auto pp = [&](int w) { return sm + L::kPPbase + w * L::kPP; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qt = blockIdx.x, bh = blockIdx.y;
@@ -370,29 +382,32 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     const int64_t kend = min64(q0 + kQ, (int64_t)Ntok);
     const int T = (int)((kend - gs + kTok - 1) / kTok);  // key tiles, >= 1
     const int Rr = (g > 0 || carried) ? R : 0;           // read-out tiles
+    TA_PHASE_VARS(ph_start);
+    TA_PHASE_T0(ph_start);
 
     if (tid == 0) {
         ptx::mbar_init(&q_loaded, 1);
         for (int i = 0; i < L::kKVSlots; ++i) {
             ptx::mbar_init(&kv_loaded[i], 1);
-            ptx::mbar_init(&kv_empty[i], 1);
+            ptx::mbar_init(&kv_empty[i], 2);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&sc_full[i], 1);
-            ptx::mbar_init(&sc_free[i], kCompute / 2);
-            ptx::mbar_init(&pp_full[i], kCompute / 2);
-            ptx::mbar_init(&pp_free[i], 1);
+            ptx::mbar_init(&sc_free[i], kOutCompute / 2);
+            ptx::mbar_init(&pp_full[i], kOutCompute / 2);
+            ptx::mbar_init(&pp_free[i], 2);
         }
         for (int i = 0; i < L::kSSlots; ++i) {
             ptx::mbar_init(&s_loaded[i], 1);
-            ptx::mbar_init(&s_empty[i], 1);
+            ptx::mbar_init(&s_empty[i], 2);
         }
-        ptx::mbar_init(&o_done, 1);
+        ptx::mbar_init(&o_done[0], 1);
+        ptx::mbar_init(&o_done[1], 1);
         s_bad = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 8) {
-        tmem_alloc(&tslot, 256);
+    if (warp == kWMma) {
+        tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
     init_ones_atom(sm + L::kOnes, tid, kOutThreads);
@@ -400,9 +415,15 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    const uint32_t tS = tslot, tO = tslot + 128;
+    // TMEM (all 512 columns): scores of two key tiles (0..127); O_hi in
+    // 128..287, whose columns 0..79 take P_hi [V|1] + Phi_Q,hi S_hi and 80..159
+    // Phi_Q,hi S_lo; O_lo in 288..367 takes P_lo [V|1] + Phi_Q,lo S_hi; per
+    // warpgroup one A operand (P or Phi_Q, hi in 32 columns then lo in 32) at
+    // 384 + 64 w.  O = O_hi[0:80] + O_hi[80:160] + O_lo.
+    const uint32_t tS = tslot, tO = tslot + 128, tO2 = tslot + 288;
+    auto tA = [&](int w) { return tslot + 384u + 64u * (uint32_t)w; };
 
-    if (warp == 9) {
+    if (warp == kWLoad) {
         if (lane == 0) {
             // q once, then key/value tiles through a ring of three slots
             ptx::mbar_arrive_expect_tx(&q_loaded, L::kQop);
@@ -422,7 +443,7 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             for (int li = (ld > L::kKVSlots ? ld - L::kKVSlots : 0); li < ld; ++li)
                 ptx::mbar_wait(&kv_loaded[li % L::kKVSlots], (li / L::kKVSlots) & 1, kWaitPolls);
         }
-    } else if (warp == 10) {
+    } else if (warp == kWSLoad) {
         // waits for the preceding kernels even without a read-out, so that
         // this grid completes only after they have
         if (lane == 0) ptx::pdl_wait_primary();
@@ -438,112 +459,143 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             for (int li = (ld > L::kSSlots ? ld - L::kSSlots : 0); li < ld; ++li)
                 ptx::mbar_wait(&s_loaded[li % L::kSSlots], (li / L::kSSlots) & 1, kWaitPolls);
         }
-    } else if (warp == 8) {
+    } else if (warp == kWMma || warp == kWMma2) {
         if (lane == 0) {
-            // every tcgen05.mma of the CTA, in order
+            // PV and read-out MMAs, in order: role 0 multiplies the hi halves
+            // of P / Phi_Q into O_hi, role 1 the lo halves into O_lo
+            const int role = warp == kWMma ? 0 : 1;
+            const uint32_t dst = role == 0 ? tO : tO2;
+            TA_PHASE_VARS(m_t, m_ppfull = 0, m_sl = 0, m_issue = 0);
+            const uint32_t id80 = idesc_bf16(kQ, kNV, 0, 1);
+            const uint32_t idro = idesc_bf16(kQ, role == 0 ? 2 * kNV : kNV, 0, 1);
+            // role 1 also issues the scores S_t = Q K_t^T into TMEM buffer t & 1
             using RS = RowSw<D>;
+            const uint64_t qd = smem_desc_sw(sQ, 16, RS::kSbo, RS::kLayout);
+            const uint32_t ids = idesc_bf16(kQ, kTok, 0, 0);
             auto scores = [&](int t) -> bool {
                 const int slot = t % L::kKVSlots;
                 if (!waitb(&kv_loaded[slot], (t / L::kKVSlots) & 1, bad)) return false;
                 fence_after_sync();
-                const uint32_t id = idesc_bf16(kQ, kTok, 0, 0);
+                const uint64_t kd = smem_desc_sw(kv(slot), 16, RS::kSbo, RS::kLayout);
+                const uint32_t d = tS + (uint32_t)((t & 1) * kTok);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    mma_bf16(tS + (t & 1) * kTok, smem_desc_sw(sQ + ks * 32, 16, RS::kSbo, RS::kLayout),
-                             smem_desc_sw(kv(slot) + ks * 32, 16, RS::kSbo, RS::kLayout), id, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < D / 16; ++ks) mma_bf16(d, qd + 2 * ks, kd + 2 * ks, ids, ks > 0 ? 1u : 0u);
                 mma_commit(&sc_full[t & 1]);
                 return true;
             };
-            bool go = waitb(&q_loaded, 0, bad);
-            if (go) go = scores(0);
-            if (go && T > 1) go = scores(1);
+            bool go = true;
+            if (role == 1) {
+                go = waitb(&q_loaded, 0, bad);
+                if (go) go = scores(0);
+                if (go && T > 1) go = scores(1);
+            }
             for (int t = 0; t < T && go; ++t) {
-                const int w = t & 1;
-                // scores of tile t + 2 go ahead of PV(t) when its warpgroup has
-                // read the scores of tile t and the key tile is resident (they
-                // write different TMEM, so the order does not change results)
+                const int w = t & 1, slot = t % L::kKVSlots;
+                // scores of tile t + 2 go ahead of PV(t) once the warpgroup has
+                // read the scores of tile t, if the key tile is already resident
                 bool early = false;
-                if (t + 2 < T) {
+                if (role == 1 && t + 2 < T) {
                     if (!waitb(&sc_free[w], (t >> 1) & 1, bad)) {
                         go = false;
                         break;
                     }
                     if (ptx::mbar_test(&kv_loaded[(t + 2) % L::kKVSlots], ((t + 2) / L::kKVSlots) & 1)) {
-                        go = scores(t + 2);
+                        if (!scores(t + 2)) {
+                            go = false;
+                            break;
+                        }
                         early = true;
                     }
                 }
-                if (!go || !waitb(&pp_full[w], (t >> 1) & 1, bad)) {
+                TA_PHASE_T0(m_t);
+                if (!waitb(&pp_full[w], (t >> 1) & 1, bad)) {
                     go = false;
                     break;
                 }
+                TA_PHASE_ACC(m_ppfull, m_t);
+                TA_PHASE_T0(m_t);
                 fence_after_sync();
-                const uint8_t* p = pp(w);
-                const uint8_t* v1 = kv(t % L::kKVSlots) + L::kKt;
-                const uint32_t lbo = (uint32_t)(L::kOnes - (L::kKVbase + (t % L::kKVSlots) * L::kKV + L::kKt));
-                const uint32_t id = idesc_bf16(kQ, kNV, 0, 1);
+                const uint32_t a = tA(w) + 32u * role;
+                const uint32_t lbo = (uint32_t)(L::kOnes - (L::kKVbase + slot * L::kKV + L::kKt));
+                const uint64_t vd = smem_desc_sw(kv(slot) + L::kKt, lbo, 1024, kSwizzle128);
 #pragma unroll
-                for (int ks = 0; ks < kTok / 16; ++ks) {
-                    const uint64_t bd = smem_desc_sw(v1 + ks * 2048, lbo, 1024, kSwizzle128);
-                    mma_bf16(tO, smem_desc(p + ks * 256, 128, kSbo64), bd, id, (t > 0 || ks > 0) ? 1u : 0u);
-                    mma_bf16(tO, smem_desc(p + kPBytes + ks * 256, 128, kSbo64), bd, id, 1u);
-                }
+                for (int ks = 0; ks < kTok / 16; ++ks)
+                    mma_bf16_ts(dst, a + ks * 8, vd + 128 * ks, id80, (t > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(&pp_free[w]);
-                mma_commit(&kv_empty[t % L::kKVSlots]);
-                if (t + 2 < T && !early) go = scores(t + 2);
+                mma_commit(&kv_empty[slot]);  // scores(t) completed before P(t) existed
+                TA_PHASE_ACC(m_issue, m_t);
+                if (role == 1 && t + 2 < T && !early && !scores(t + 2)) go = false;
             }
             const int nuse[2] = {(T + 1) / 2, T / 2};
             for (int r = 0; r < Rr && go; ++r) {
-                const int w = r & 1, u = nuse[w] + (r >> 1);
-                if (!waitb(&pp_full[w], u & 1, bad) || !waitb(&s_loaded[r % L::kSSlots], (r / L::kSSlots) & 1, bad)) {
+                const int w = r & 1, u = nuse[w] + (r >> 1), slot = r % L::kSSlots;
+                TA_PHASE_T0(m_t);
+                if (!waitb(&pp_full[w], u & 1, bad)) {
                     go = false;
                     break;
                 }
-                fence_after_sync();
-                const uint8_t* a = pp(w);
-                const uint8_t* s = sS(r % L::kSSlots);
-                const uint32_t id = idesc_bf16(kQ, kNV, 0, 1);
-#pragma unroll
-                for (int ks = 0; ks < kRT / 16; ++ks) {
-                    const uint64_t ah = smem_desc(a + ks * 256, 128, kSbo64);
-                    const uint64_t al = smem_desc(a + kPBytes + ks * 256, 128, kSbo64);
-                    const uint64_t bh_ = smem_desc(s + ks * 2 * kLboNV, kLboNV, 128);
-                    const uint64_t bl_ = smem_desc(s + kSHalf + ks * 2 * kLboNV, kLboNV, 128);
-                    mma_bf16(tO, ah, bh_, id, 1u);
-                    mma_bf16(tO, ah, bl_, id, 1u);
-                    mma_bf16(tO, al, bh_, id, 1u);
+                TA_PHASE_ACC(m_ppfull, m_t);
+                TA_PHASE_T0(m_t);
+                if (!waitb(&s_loaded[slot], (r / L::kSSlots) & 1, bad)) {
+                    go = false;
+                    break;
                 }
+                TA_PHASE_ACC(m_sl, m_t);
+                TA_PHASE_T0(m_t);
+                fence_after_sync();
+                const uint32_t a = tA(w) + 32u * role;
+                const uint64_t sd = smem_desc(sS(slot), kLboS, 128);
+#pragma unroll
+                for (int ks = 0; ks < kRT / 16; ++ks) mma_bf16_ts(dst, a + ks * 8, sd + (2 * kLboS / 16) * ks, idro, 1u);
                 mma_commit(&pp_free[w]);
-                mma_commit(&s_empty[r % L::kSSlots]);
+                mma_commit(&s_empty[slot]);
+                TA_PHASE_ACC(m_issue, m_t);
             }
-            mma_commit(&o_done);  // covers every MMA issued above
-            if (!ptx::mbar_wait(&o_done, 0, kWaitPolls)) *bad = 1;
+            mma_commit(&o_done[role]);  // covers every MMA this thread issued
+            if (!ptx::mbar_wait(&o_done[role], 0, kWaitPolls)) *bad = 1;
+            TA_PHASE_PUT(0, 1, role == 0, m_ppfull);
+            TA_PHASE_PUT(0, 4, role == 0, m_sl);
+            TA_PHASE_PUT(0, 5, role == 0, m_issue);
         }
     } else {
         // warpgroup w: P of key tiles w, w + 2, ..., then Phi_Q of read-out
-        // tiles w, w + 2, ...; thread = query row
-        const int w = warp >> 2;
+        // tiles w, w + 2, ...; thread = query row, half hh of the tile's 64
+        // columns (keys or features)
+        const int w = warp >> 3, hh = (warp >> 2) & 1;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const int64_t qi = q0 + row;
         float qc[kMaxN];
 #pragma unroll
         for (int m = 0; m < kMaxN; ++m) qc[m] = query_coeff(m, tau);
-        uint8_t* buf = pp(w);
+        const uint32_t a_hi = tA(w) + lane_off + 16 * hh, a_lo = a_hi + 32;
+        if (w == 0 && hh == 0) {  // O columns 80..159 start at zero (the MMAs into them accumulate)
+            uint32_t z[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) z[i] = 0;
+            tmem_st32(tO + lane_off + 80, z);
+            tmem_st32(tO + lane_off + 112, z);
+            tmem_st16(tO + lane_off + 144, *reinterpret_cast<uint32_t(*)[16]>(z));
+            tmem_st_wait();
+            fence_before_sync();
+        }
         int u = 0;
+        TA_PHASE_VARS(w_t, w_sc = 0, w_p = 0, w_pf = 0, w_st = 0, w_phi = 0, w_pf2 = 0);
         for (int t = w; t < T; t += 2, ++u) {
+            TA_PHASE_T0(w_t);
             if (!waitb(&sc_full[w], (t >> 1) & 1, bad)) break;
+            TA_PHASE_ACC(w_sc, w_t);
+            TA_PHASE_T0(w_t);
             fence_after_sync();
-            float s[64];
-            tmem_ld32(tS + lane_off + w * kTok, *reinterpret_cast<float(*)[32]>(s));
-            tmem_ld32(tS + lane_off + w * kTok + 32, *reinterpret_cast<float(*)[32]>(s + 32));
+            float s[32];
+            tmem_ld32(tS + lane_off + w * kTok + 32 * hh, s);
             tmem_ld_wait();
             fence_before_sync();
             ptx::mbar_arrive(&sc_free[w]);
-            const int64_t k0 = gs + (int64_t)t * kTok;
-            const bool mask = k0 + kTok - 1 > q0 || k0 + kTok > Ntok;
+            const int64_t k0 = gs + (int64_t)t * kTok + 32 * hh;
+            const bool mask = k0 + 31 > q0 || k0 + 32 > Ntok;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
+            for (int j = 0; j < 32; ++j) {
                 const float x = s[j];
                 float p;
                 if constexpr (N > 0) {
@@ -557,58 +609,90 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 if (mask && !(k0 + j <= qi && k0 + j < kend)) p = 0.f;
                 s[j] = p;
             }
-            if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
+            uint32_t hi[16], lo[16];
 #pragma unroll
-            for (int kg = 0; kg < 8; ++kg) {
-                const uint32_t off = kmaj(row, kg, kSbo64);
-                store_split8(s + 8 * kg, buf + off, buf + kPBytes + off);
-            }
-            ptx::fence_proxy_async_smem();
+            for (int i = 0; i < 16; ++i) split2(s[2 * i], s[2 * i + 1], hi[i], lo[i]);
+            TA_PHASE_ACC(w_p, w_t);
+            TA_PHASE_T0(w_t);
+            if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
+            TA_PHASE_ACC(w_pf, w_t);
+            TA_PHASE_T0(w_t);
+            fence_after_sync();
+            tmem_st16(a_hi, hi);
+            tmem_st16(a_lo, lo);
+            tmem_st_wait();
+            fence_before_sync();
             ptx::mbar_arrive(&pp_full[w]);
+            TA_PHASE_ACC(w_st, w_t);
         }
         if (!*bad) {
             const uint8_t* rowbase = sQ + row * RowSw<D>::kRowBytes;
             const uint32_t sw = swizzle_of_row(row, RowSw<D>::kRowBytes);
             for (int r = w; r < Rr; r += 2, ++u) {
-                float o[64];
-                fe::Eval<D, N, true>::block(r * 2, rowbase, sw, qc, n, F, tau, *reinterpret_cast<float(*)[32]>(o));
-                fe::Eval<D, N, true>::block(r * 2 + 1, rowbase, sw, qc, n, F, tau,
-                                            *reinterpret_cast<float(*)[32]>(o + 32));
-                if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
+                float o[32];
+                TA_PHASE_T0(w_t);
+                fe::Eval<D, N, true>::block(r * 2 + hh, rowbase, sw, qc, n, F, tau, o);
+                uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int kg = 0; kg < 8; ++kg) {
-                    const uint32_t off = kmaj(row, kg, kSbo64);
-                    store_split8(o + 8 * kg, buf + off, buf + kPBytes + off);
-                }
-                ptx::fence_proxy_async_smem();
+                for (int i = 0; i < 16; ++i) split2(o[2 * i], o[2 * i + 1], hi[i], lo[i]);
+                TA_PHASE_ACC(w_phi, w_t);
+                TA_PHASE_T0(w_t);
+                if (u > 0 && !waitb(&pp_free[w], (u - 1) & 1, bad)) break;
+                TA_PHASE_ACC(w_pf2, w_t);
+                TA_PHASE_T0(w_t);
+                fence_after_sync();
+                tmem_st16(a_hi, hi);
+                tmem_st16(a_lo, lo);
+                tmem_st_wait();
+                fence_before_sync();
                 ptx::mbar_arrive(&pp_full[w]);
+                TA_PHASE_ACC(w_st, w_t);
             }
         }
+        TA_PHASE_PUT(0, 6, tid == 0, w_sc);
+        TA_PHASE_PUT(0, 7, tid == 0, w_p);
+        TA_PHASE_PUT(0, 8, tid == 0, w_pf);
+        TA_PHASE_PUT(0, 9, tid == 0, w_st);
+        TA_PHASE_PUT(0, 10, tid == 0, w_phi);
+        TA_PHASE_PUT(0, 11, tid == 0, w_pf2);
     }
     __syncthreads();  // the MMA thread has seen every MMA complete (or a failure)
+    TA_PHASE_PUT(0, 12, tid == 0, (unsigned long long)T);
+    TA_PHASE_PUT(0, 13, tid == 0, (unsigned long long)Rr);
+    TA_PHASE_VARS(ph_end);
+    TA_PHASE_T0(ph_end);
+    TA_PHASE_PUT(0, 0, tid == 0, ph_end - ph_start);
     fence_after_sync();
     const bool ok = s_bad == 0;
-    if (ok && tid < kCompute) {
-        const int row = (warp & 3) * 32 + lane, half = warp >> 2;
+    if (ok && tid < kOutCompute) {
+        // warp (quadrant q, column block cb): rows 32 q .., output columns 16 cb ..
+        const int row = (warp & 3) * 32 + lane, cb = warp >> 2;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        float o[32], dn[16];
-        tmem_ld32(tO + lane_off + half * 32, o);
-        tmem_ld16(tO + lane_off + kDV, dn);
+        float o[16], o2[16];
+        tmem_ld16(tO + lane_off + 16 * cb, o);
+        tmem_ld16(tO + lane_off + kNV + 16 * cb, o2);
+        const float d1 = tmem_ld1(tO + lane_off + kDV), d2 = tmem_ld1(tO + lane_off + kNV + kDV);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] += o2[i];
+        tmem_ld16(tO2 + lane_off + 16 * cb, o2);
+        const float d3 = tmem_ld1(tO2 + lane_off + kDV);
         tmem_ld_wait();
         if (row < nq) {
-            const float rcp = __frcp_rn(dn[0]);
-            float4* dst = reinterpret_cast<float4*>(out + ((int64_t)bh * Ntok + q0 + row) * kDV + half * 32);
+            const float rcp = __frcp_rn(d1 + d2 + d3);
+            float4* dst = reinterpret_cast<float4*>(out + ((int64_t)bh * Ntok + q0 + row) * kDV + 16 * cb);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(o[4 * i] * rcp, o[4 * i + 1] * rcp, o[4 * i + 2] * rcp, o[4 * i + 3] * rcp);
+            for (int i = 0; i < 16; ++i) o[i] = (o[i] + o2[i]) * rcp;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
     }
     if (!ok && tid == 0) atomicOr(err, kErrPrefillPipe);
     fence_before_sync();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kWMma) {
         fence_after_sync();
-        tmem_dealloc(tslot, 256);
+        tmem_dealloc(tslot, 512);
     }
 }
 
