@@ -279,6 +279,42 @@ def run_ours(args, world, rank, local):
     dec_warm_us = warm_ev[0].elapsed_time(warm_ev[1]) * 1e3 / dsteps
     dec_us_max = allmax(dec_us, world, dev)
 
+    # ---- batched multi-token decode: T new tokens per head per call, in place
+    multi = {}
+    for T in (4, 16):
+        def unit_t(shape):
+            x = torch.randn(shape, device=dev, generator=g, dtype=torch.float32)
+            return (x / x.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        mtoks = [(unit_t((dB, dH, T, dw["d_k"])), unit_t((dB, dH, T, dw["d_k"])),
+                  torch.randn((dB, dH, T, dw["d_v"]), device=dev, generator=g).to(torch.bfloat16))
+                 for _ in range(dsteps)]
+        mout = torch.empty((dB, dH, T, dw["d_v"]), dtype=torch.float32, device=dev)
+        for s_ in range(3):
+            flush_l2()
+            TA.taylor_attn_prefill_from_state(*mtoks[s_], dstate, dw["n"], dw["tau"], out=mout, state_out=dstate)
+        torch.cuda.synchronize()
+        TA.taylor_attn_timing_read()
+        TA.taylor_attn_timing_enable(True)
+        m_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(dsteps)]
+        for s_ in range(dsteps):
+            flush_l2()
+            m_ev[s_][0].record(stream)
+            TA.taylor_attn_prefill_from_state(*mtoks[s_], dstate, dw["n"], dw["tau"], out=mout, state_out=dstate)
+            m_ev[s_][1].record(stream)
+        torch.cuda.synchronize()
+        TA.taylor_attn_timing_enable(False)
+        mk = TA.taylor_attn_timing_read()
+        m_us = statistics.mean(a.elapsed_time(b) for a, b in m_ev) * 1e3
+        mk_name, (mk_launch, mk_ms) = max(mk.items(), key=lambda kv: kv[1][1])
+        mk_us = mk_ms / mk_launch * 1e3
+        Fd = TA.taylor_attn_num_features(dw["d_k"], dw["n"])
+        m_bytes = dB * dH * (2 * Fd * (dw["d_v"] + 1) * 4 + T * ((2 * dw["d_k"] + dw["d_v"]) * 2 + dw["d_v"] * 4))
+        multi[str(T)] = {"us_per_call": round(m_us, 3), "kernel": mk_name, "kernel_us": round(mk_us, 3),
+                         "Mtok_s": round(dB * dH * T / (m_us * 1e-6) / 1e6, 2),
+                         "hbm_frac": round(m_bytes / (mk_us * 1e-6) / 1e9 / hbm_peak, 4),
+                         "algorithmic_bytes_per_launch": m_bytes}
+        del mtoks, mout
+
     # ---- large-head prefill (F = 2,145): the contraction-bound configuration
     lw = LARGE
     lB, lH, lN, ld, ldv, ln = lw["B"], lw["H"], lw["N"], lw["d_k"], lw["d_v"], lw["n"]
@@ -393,6 +429,11 @@ def run_ours(args, world, rank, local):
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(dbytes / (dec_kernel_us * 1e-6) / 1e9 / hbm_peak, 4),
                              "algorithmic_bytes_per_launch": dbytes, "traffic": None},
+            },
+            "multi_token_decode": {
+                "workload": "B=64 H=16 d_k=16 d_v=64 n=3, T new tokens per head per call against the carried "
+                            "states (taylor_attn_prefill_from_state in place), L2 flushed before each call",
+                "by_tokens_per_call": multi,
             },
             "large_head_prefill": {
                 "workload": "causal prefill B=4 H=16 N=32768 d_k=64 d_v=64 n=3 (F=2145) tau=2, bf16 q/k/v, "

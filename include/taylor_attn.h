@@ -121,7 +121,10 @@ TAYLOR_API int taylor_attn_prefill_f32(const float* q, const float* k, const flo
  * tokens as taylor_attn_prefill does; state_out (may be NULL, may alias
  * state_in) receives state_in plus the new tokens' state (abstract: states
  * are additive across chunks, so prefill can resume from a chunk boundary).
- * q, k, v bf16; workspace and errors as taylor_attn_prefill. */
+ * q, k, v bf16; workspace and errors as taylor_attn_prefill.  With N <= 16,
+ * d_v in {16, 32, 64, 128} and at most 1,024 features this is batched
+ * multi-token decode: one kernel reads and writes each head's state once
+ * and allocates no workspace. */
 TAYLOR_API int taylor_attn_prefill_from_state(const void* q, const void* k, const void* v,
                                               const float* state_in, float* out, float* state_out,
                                               int B, int H, int N, int d_k, int d_v, int n, float tau,

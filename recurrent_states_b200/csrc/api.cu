@@ -68,6 +68,12 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, const float* state_in
     if (!q || !k || !v || !out) return TAYLOR_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TAYLOR_ERR_MISALIGNED;
 
+    if (state_in != nullptr && N <= 16) {
+        // a few new tokens against a carried state: one pass over the state
+        const cudaError_t e = ta::launch_decode_multi(q, k, v, state_in, state_out, out, (int)BH, N, d_k, d_v, n,
+                                                      tau, F, stride, stream);
+        if (e != cudaErrorNotSupported) return cuda_status(e);
+    }
     if (allow_tc) {
         const int tc = ta::tc::try_prefill(q, k, v, out, state_in, state_out, (int)BH, N, d_k, d_v, n, tau, F,
                                            stride, stream);

@@ -38,6 +38,14 @@ cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state
                           int BH, int d, int dv, int n, float tau, int64_t F, int64_t stride,
                           cudaStream_t stream);
 
+// Batched multi-token decode: T (1..16) new tokens per head against
+// state_in, outputs for all of them and (if state_out) the updated state;
+// cudaErrorNotSupported when the shape is outside the kernel's range.
+template <typename Tin>
+cudaError_t launch_decode_multi(const Tin* q, const Tin* k, const Tin* v, const float* state_in, float* state_out,
+                                float* out, int BH, int T, int d, int dv, int n, float tau, int64_t F, int64_t stride,
+                                cudaStream_t stream);
+
 cudaError_t launch_merge(const float* a, const float* b, float* out, int64_t count, int num_sms,
                          cudaStream_t stream);
 

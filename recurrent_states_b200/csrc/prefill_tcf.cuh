@@ -625,6 +625,10 @@ tcf_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             ptx::mbar_arrive(&pp_full[w]);
             TA_PHASE_ACC(w_st, w_t);
         }
+        // q must be resident before Phi_Q is read from it: a warpgroup
+        // without key tiles (T == 1) reaches this point before any scores
+        // MMA, hence before anything else has waited for the q load
+        if (Rr > 0 && !waitb(&q_loaded, 0, bad)) *bad = 1;
         if (!*bad) {
             const uint8_t* rowbase = sQ + row * RowSw<D>::kRowBytes;
             const uint32_t sw = swizzle_of_row(row, RowSw<D>::kRowBytes);

@@ -273,7 +273,12 @@ def test_merge_and_split_prefill():
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("d,dv,n,N,cut", [(16, 64, 3, 1000, 384), (16, 64, 3, 700, 77), (16, 64, 3, 300, 1),
                                           (16, 16, 3, 500, 256), (64, 64, 3, 600, 130), (16, 64, 5, 400, 200),
-                                          (32, 64, 3, 2600, 300), (7, 12, 2, 200, 33)])
+                                          (32, 64, 3, 2600, 300), (7, 12, 2, 200, 33),
+                                          # a few new tokens: the multi-token decode kernel
+                                          (16, 64, 3, 300, 292), (16, 64, 3, 300, 299), (16, 16, 3, 200, 184),
+                                          (32, 64, 3, 300, 290), (16, 128, 3, 100, 88),
+                                          # tails shorter than one key tile on the feature-tiled path
+                                          (64, 64, 3, 300, 280), (16, 64, 4, 300, 250), (16, 64, 5, 300, 240)])
 def test_prefill_from_state_continues_the_sequence(dtype, d, dv, n, N, cut):
     """Prefill of the tail from the head's state equals the oracle's recursion
     over the whole sequence (outputs of the tail, final state)."""
@@ -294,6 +299,29 @@ def test_prefill_from_state_continues_the_sequence(dtype, d, dv, n, N, cut):
     cont(t_(q), t_(k), t_(v), st2, n, tau, state_out=st2)
     torch.cuda.synchronize()
     assert torch.equal(st2, st)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_multi_token_decode_blocks_follow_the_recursion(dtype):
+    """Blocks of 1..16 new tokens, each fed in place through prefill from
+    state, give the oracle's outputs for those tokens and its final state."""
+    d, dv, n, tau = 16, 64, 3, 2.0
+    blocks = [1, 4, 16, 7, 16, 2]
+    prefix = 256
+    N = prefix + sum(blocks)
+    q, k, v = synth.qkv(2, 3, N, d, dv, seed=77, dtype=dtype)
+    prefill = TA.taylor_attn_prefill if dtype == "bf16" else TA.taylor_attn_prefill_f32
+    cont = TA.taylor_attn_prefill_from_state if dtype == "bf16" else TA.taylor_attn_prefill_from_state_f32
+    sl = lambda t, a, b: t[:, :, a:b].contiguous().to(DEV)  # noqa: E731
+    _, st = prefill(sl(q, 0, prefix), sl(k, 0, prefix), sl(v, 0, prefix), n, tau, state_out=True)
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    t0 = prefix
+    for T in blocks:
+        o, _ = cont(sl(q, t0, t0 + T), sl(k, t0, t0 + T), sl(v, t0, t0 + T), st, n, tau, state_out=st)
+        torch.cuda.synchronize()
+        assert row_scaled_max_err(f64(o), ref_out[:, :, t0:t0 + T]) <= TOL[dtype]
+        t0 += T
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL[dtype]
 
 
 def test_prefill_from_state_with_no_new_tokens_copies_the_state():
