@@ -501,6 +501,10 @@ cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state
     unsigned int* err = device_error_word();
     const bool tma_ok = err != nullptr && used_bytes <= kTmaMaxBytes && dyn <= (size_t)kTmaMaxBytes + 8192 &&
                         F <= kTmaMaxFeatures;
+    if (err != nullptr) {  // many heads of a small state: the persistent warp-specialised kernel
+        const cudaError_t e = launch_decode_ws(q, k, v, state, out, BH, d, dv, n, tau, F, stride, stream);
+        if (e != cudaErrorNotSupported) return e;
+    }
     const size_t dyn2 = 2 * (size_t)((bytes + 127u) & ~127u) + 2 * (size_t)((F + 3) & ~3) * 4;
     if (tma_ok && kPersistMaxDyn > 0 && dyn2 <= kPersistMaxDyn) {
         switch (dv) {

@@ -1,0 +1,228 @@
+// Persistent, warp-specialised decode step for d_v = 64 and states of at most
+// 256 features (the decode workload: d_k 16, n 3, 153 x 65 floats per head).
+// Same arithmetic as the one-CTA-per-head kernel in decode.cu (the pages'
+// constant-cost decode, arXiv 2610.20637, abstract):
+//   S += phi(k) [v | 1]^T,  y = (c (.) phi(q))^T S,  o = y[0:64] / y[64].
+//
+// One CTA per SM walks the heads blockIdx.x, blockIdx.x + gridDim.x, ...
+// One producer thread keeps a ring of state buffers in shared memory full:
+// for each head a bulk copy of its state and of its new token (q, k, v)
+// completing on the buffer's mbarrier, issued as soon as the buffer is free,
+// so several heads' loads per SM are always in flight.  Four consumer
+// warpgroups take the heads in turn; a warpgroup evaluates phi(k), phi(q) for
+// its head, updates the rows (one 16-byte column group per thread per row,
+// stored straight to HBM), reduces the read-out and writes o, synchronising
+// only its own 128 threads (named barriers), then hands the buffer back.
+#include <mutex>
+
+#include "common.cuh"
+#include "feature_table.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace ta {
+
+namespace {
+
+constexpr int kDV = 64, kDV4 = 16;
+constexpr int kWG = 4;                      // consumer warpgroups
+constexpr int kWGThreads = 128;
+constexpr int kThreadsWS = kWG * kWGThreads + 32;
+constexpr int kMaxF = 256;
+constexpr int kMaxBuf = 6;
+constexpr uint32_t kWaitPolls = 1u << 22;
+constexpr size_t kMaxDynWS = 218 * 1024;  // with the static arrays, within the 227 KB per CTA
+constexpr int kMaxDevices = 64;
+
+struct WGArea {                 // per consumer warpgroup
+    float pk[kMaxF], pq[kMaxF];
+    float4 red[4][kDV4];
+    float zr[4];
+    int fail;                   // written only before a warpgroup barrier, read after it
+};
+
+__device__ __forceinline__ void wg_sync(int wg) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + wg), "r"(kWGThreads) : "memory");
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreadsWS, 1)
+decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                 float* __restrict__ state, float* __restrict__ out, int BH, int d, int n, float tau, int F,
+                 int64_t stride, uint32_t bytes, uint32_t buf_bytes, int nbuf, unsigned int* __restrict__ err) {
+    extern __shared__ __align__(128) unsigned char dsm[];
+    __shared__ __align__(8) uint64_t full[kMaxBuf], empty[kMaxBuf];
+    __shared__ FeatDesc dk_s[kMaxF], dq_s[kMaxF];
+    __shared__ float qc[kMaxN];
+    __shared__ int s_bad;
+    WGArea* wga = reinterpret_cast<WGArea*>(dsm + (size_t)nbuf * buf_bytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nheads = BH > (int)blockIdx.x ? (BH - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const uint32_t tok_in = (uint32_t)(d * sizeof(Tin)), tok_v = (uint32_t)(kDV * sizeof(Tin));
+    // token area of a buffer: q, k, v rows right after the state, 16-byte aligned
+    const uint32_t offq = (bytes + 15u) & ~15u, offk = offq + ((tok_in + 15u) & ~15u),
+                   offv = offk + ((tok_in + 15u) & ~15u);
+
+    if (tid == 0) {
+        for (int i = 0; i < nbuf; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], 1);
+        }
+        s_bad = 0;
+        ptx::fence_mbar_init();
+    }
+    if (tid < n) qc[tid] = query_coeff(tid, tau);
+    if (tid < kWG) wga[tid].fail = 0;
+    __syncthreads();
+    {
+        const PackedFeat* tab = feat_table(d, n);
+        for (int f = tid; f < F; f += kThreadsWS) {
+            dk_s[f] = tab ? desc_from_packed(tab[f], qc, false) : make_desc(d, n, f, tau, false);
+            dq_s[f] = tab ? desc_from_packed(tab[f], qc, true) : make_desc(d, n, f, tau, true);
+        }
+    }
+    __syncthreads();
+
+    if (warp == kWG * kWGThreads / 32) {
+        if (lane == 0) {
+            int i = 0;
+            for (; i < nheads; ++i) {
+                const int b = i % nbuf;
+                if (i >= nbuf && !ptx::mbar_wait_or_abort(&empty[b], ((i / nbuf) - 1) & 1, kWaitPolls, &s_bad)) break;
+                const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+                unsigned char* buf = dsm + (size_t)b * buf_bytes;
+                ptx::mbar_arrive_expect_tx(&full[b], bytes + 2 * tok_in + tok_v);
+                ptx::bulk_g2s(buf, state + h * stride, bytes, &full[b]);
+                ptx::bulk_g2s(buf + offq, q + h * d, tok_in, &full[b]);
+                ptx::bulk_g2s(buf + offk, k + h * d, tok_in, &full[b]);
+                ptx::bulk_g2s(buf + offv, v + h * kDV, tok_v, &full[b]);
+            }
+            // copies that no warpgroup consumed (only after a failure) land before the CTA leaves
+            for (int j = (i > nbuf ? i - nbuf : 0); j < i; ++j)
+                ptx::mbar_wait(&full[j % nbuf], (j / nbuf) & 1, kWaitPolls);
+        }
+    } else {
+        const int wg = warp >> 2, t = tid & (kWGThreads - 1), wl = (warp & 3);
+        WGArea& A = wga[wg];
+        const int cg = t % kDV4, rs = t / kDV4;  // 8 row sets
+        for (int i = wg; i < nheads; i += kWG) {
+            const int b = i % nbuf;
+            if (!ptx::mbar_wait_or_abort(&full[b], (i / nbuf) & 1, kWaitPolls, &s_bad)) A.fail = 1;
+            wg_sync(wg);
+            if (A.fail) break;  // the same value for all 128 threads: set only before this barrier
+            const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+            const unsigned char* buf = dsm + (size_t)b * buf_bytes;
+            const Tin* xq = reinterpret_cast<const Tin*>(buf + offq);
+            const Tin* xk = reinterpret_cast<const Tin*>(buf + offk);
+            const Tin* vv = reinterpret_cast<const Tin*>(buf + offv);
+            for (int f = t; f < F; f += kWGThreads) {
+                const FeatDesc fk = dk_s[f], fq = dq_s[f];
+                float pk = fk.w, pq = fq.w;
+                for (int s = 0; s < fk.m; ++s) pk *= to_float(xk[(fk.packed >> (8 * s)) & 0xff]);
+                for (int s = 0; s < fq.m; ++s) pq *= to_float(xq[(fq.packed >> (8 * s)) & 0xff]);
+                A.pk[f] = pk;
+                A.pq[f] = pq;
+            }
+            const float4 v4 = make_float4(to_float(vv[4 * cg]), to_float(vv[4 * cg + 1]), to_float(vv[4 * cg + 2]),
+                                          to_float(vv[4 * cg + 3]));
+            wg_sync(wg);
+            const float4* S4 = reinterpret_cast<const float4*>(buf);
+            float4* G4 = reinterpret_cast<float4*>(state + h * stride);
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int r = rs; r < F; r += kWGThreads / kDV4) {
+                const float a = A.pk[r], c = A.pq[r];
+                float4 s = S4[r * kDV4 + cg];
+                s.x = fmaf(a, v4.x, s.x);
+                s.y = fmaf(a, v4.y, s.y);
+                s.z = fmaf(a, v4.z, s.z);
+                s.w = fmaf(a, v4.w, s.w);
+                G4[r * kDV4 + cg] = s;
+                y.x = fmaf(c, s.x, y.x);
+                y.y = fmaf(c, s.y, y.y);
+                y.z = fmaf(c, s.z, y.z);
+                y.w = fmaf(c, s.w, y.w);
+            }
+            float yz = 0.f;
+            const float* Z = reinterpret_cast<const float*>(buf) + (int64_t)F * kDV;
+            float* GZ = state + h * stride + (int64_t)F * kDV;
+            for (int f = t; f < F; f += kWGThreads) {
+                const float z = Z[f] + A.pk[f];
+                GZ[f] = z;
+                yz = fmaf(A.pq[f], z, yz);
+            }
+            // the buffer has been read: hand it back once the whole warpgroup is past here
+            ptx::fence_proxy_async_smem();
+            y.x += __shfl_xor_sync(0xffffffffu, y.x, 16);
+            y.y += __shfl_xor_sync(0xffffffffu, y.y, 16);
+            y.z += __shfl_xor_sync(0xffffffffu, y.z, 16);
+            y.w += __shfl_xor_sync(0xffffffffu, y.w, 16);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) yz += __shfl_xor_sync(0xffffffffu, yz, o);
+            if (lane < kDV4) A.red[wl][lane] = y;
+            if (lane == 0) A.zr[wl] = yz;
+            wg_sync(wg);
+            if (t == 0) ptx::mbar_arrive(&empty[b]);
+            if (t < kDV) {
+                const int g4 = t >> 2, c4 = t & 3;
+                float acc = 0.f, den = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const float4 r4 = A.red[w][g4];
+                    acc += c4 == 0 ? r4.x : c4 == 1 ? r4.y : c4 == 2 ? r4.z : r4.w;
+                    den += A.zr[w];
+                }
+                out[h * kDV + t] = acc / den;
+            }
+            // A.pk, A.pq, A.red are rewritten only after the next head's first barrier
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && s_bad) atomicOr(err, kErrDecodeLoad);
+}
+
+}  // namespace
+
+template <typename Tin>
+cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
+                             int dv, int n, float tau, int64_t F, int64_t stride, cudaStream_t stream) {
+    if (dv != kDV || F > kMaxF || (d * (int)sizeof(Tin)) % 16 != 0) return cudaErrorNotSupported;
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t set_err[kMaxDevices];
+    static int num_sms[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&]() {
+        set_err[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(decode_ws_kernel<Tin>),
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDynWS);
+        if (set_err[dev] == cudaSuccess)
+            set_err[dev] = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    });
+    if (set_err[dev] != cudaSuccess) return set_err[dev];
+    if (BH < 2 * num_sms[dev]) return cudaErrorNotSupported;  // few heads: one CTA per head is as good
+    const uint32_t bytes = (uint32_t)((F * (kDV + 1) * 4 + 15) / 16 * 16);
+    const uint32_t tok = (uint32_t)(((d * sizeof(Tin) + 15) / 16 * 16) * 2 + kDV * sizeof(Tin));
+    const uint32_t buf_bytes = (bytes + 15u) / 16u * 16u + tok;
+    const uint32_t buf_al = (buf_bytes + 127u) & ~127u;
+    const size_t area = kWG * sizeof(WGArea);
+    int nbuf = (int)((kMaxDynWS - area) / buf_al);
+    if (nbuf > kMaxBuf) nbuf = kMaxBuf;
+    if (nbuf < 2) return cudaErrorNotSupported;
+    const size_t dyn = (size_t)nbuf * buf_al + area;
+    unsigned int* err = device_error_word();
+    if (!err) return cudaErrorNotSupported;
+    const int grid = num_sms[dev] < BH ? num_sms[dev] : BH;
+    TA_TIMED(stream, "decode_ws_kernel",
+             decode_ws_kernel<Tin><<<grid, kThreadsWS, dyn, stream>>>(q, k, v, state, out, BH, d, n, tau, (int)F,
+                                                                       stride, bytes, buf_al, nbuf, err));
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_decode_ws<float>(const float*, const float*, const float*, float*, float*, int, int, int,
+                                             int, float, int64_t, int64_t, cudaStream_t);
+template cudaError_t launch_decode_ws<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                                     const __nv_bfloat16*, float*, float*, int, int, int, int, float,
+                                                     int64_t, int64_t, cudaStream_t);
+
+}  // namespace ta

@@ -38,6 +38,13 @@ cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state
                           int BH, int d, int dv, int n, float tau, int64_t F, int64_t stride,
                           cudaStream_t stream);
 
+// Persistent warp-specialised decode for d_v 64 and at most 256 features;
+// cudaErrorNotSupported when the shape (or a small number of heads) is
+// better served by the one-CTA-per-head kernel.
+template <typename Tin>
+cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
+                             int dv, int n, float tau, int64_t F, int64_t stride, cudaStream_t stream);
+
 // Batched multi-token decode: T (1..16) new tokens per head against
 // state_in, outputs for all of them and (if state_out) the updated state;
 // cudaErrorNotSupported when the shape is outside the kernel's range.
