@@ -55,7 +55,7 @@ constexpr uint32_t kSboQK = 2 * 128;                 // Q, K: [128][16] K-major
 constexpr uint32_t kLboV1 = (kNV / 8) * 128;         // [V|1]: [K=128 keys][80] MN-major
 constexpr uint32_t kSboP = (kC / 8) * 128;           // P: [128][128] K-major
 constexpr uint32_t kSboPhiQ = (kFP / 8) * 128;       // Phi_Q: [128][160] K-major
-constexpr uint32_t kLboS = (kNV / 8) * 128;          // S: [K=160][80] MN-major
+constexpr uint32_t kLboS = (2 * kNV / 8) * 128;      // S: [K=160][hi 80 | lo 80] MN-major
 constexpr uint32_t kLboVT = 16 * 128;                // [V|1|0]^T: [M=128 rows][K=128 tokens] MN-major
 constexpr uint32_t kLboPhiK = (kFP / 8) * 128;       // Phi_K: [K=128 tokens][N=160] MN-major
 
@@ -201,11 +201,14 @@ tc_chunk_state_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v, fl
 
     if (tid == 0) {
         const uint32_t id = idesc_bf16(128, kFP, 1, 1);
+        // descriptors built once and advanced by constants (16-byte units)
+        const uint64_t va = smem_desc(sVT, kLboVT, 128);
+        const uint64_t bh_ = smem_desc(sBh, kLboPhiK, 128), bl_ = smem_desc(sBl, kLboPhiK, 128);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks) {
-            const uint64_t a = smem_desc(sVT + ks * 2 * kLboVT, kLboVT, 128);
-            mma_bf16(tbase, a, smem_desc(sBh + ks * 2 * kLboPhiK, kLboPhiK, 128), id, ks > 0 ? 1u : 0u);
-            mma_bf16(tbase, a, smem_desc(sBl + ks * 2 * kLboPhiK, kLboPhiK, 128), id, 1u);
+            const uint64_t a = va + (2 * kLboVT / 16) * ks;
+            mma_bf16(tbase, a, bh_ + (2 * kLboPhiK / 16) * ks, id, ks > 0 ? 1u : 0u);
+            mma_bf16(tbase, a, bl_ + (2 * kLboPhiK / 16) * ks, id, 1u);
         }
         mma_commit(&mb);
     }
@@ -288,8 +291,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     uint8_t* sPl = sm + kOffPl;
     uint8_t* sQh = sm + kOffQh;
     uint8_t* sQl = sm + kOffQl;
-    uint8_t* sSh = sm + kOffSh;
-    uint8_t* sSl = sm + kOffSl;
+    uint8_t* sS = sm + kOffSh;  // S hi in column groups 0..9, lo in 10..19 (the Sh and Sl space)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, bh = blockIdx.y;
@@ -309,7 +311,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
         ptx::fence_mbar_init();
     }
     if (warp == 8) {
-        tmem_alloc(&tslot, 256);
+        tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
     fence_before_sync();
@@ -317,13 +319,17 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     fence_after_sync();
     const uint32_t tbase = tslot;
     const uint32_t tA = tbase;          // scores, columns [0, 128)
-    const uint32_t tO = tbase + 128;    // [numerator | denominator], columns [128, 208)
+    // O in columns [128, 288): [0, 80) takes P[V|1|0] + Phi_Q,hi S_hi + Phi_Q,lo S_hi,
+    // [80, 160) Phi_Q,hi S_lo (the read-out's hi operand meets [S_hi | S_lo] in one N = 160 MMA)
+    const uint32_t tO = tbase + 128;
     TA_PHASE(1, 1, tid == 0);
 
     if (warp == 8) {
         // ------------------------------------------------ MMA issue (one thread)
         if (lane == 0) {
+            // descriptors are built once and advanced by constants (16-byte units)
             const uint32_t id = idesc_bf16(128, kNV, 0, 1);
+            const uint32_t id160 = idesc_bf16(128, 2 * kNV, 0, 1);
             bool good = ptx::mbar_wait(&bar_qk, 0, kWaitPolls);
             fence_after_sync();
             if (good)
@@ -334,11 +340,13 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
                 fence_after_sync();
                 TA_PHASE(1, 11, true);
                 if (good) {
+                    const uint64_t bv = smem_desc(sV1, kLboV1, 128);
+                    const uint64_t ph = smem_desc(sPh, 128, kSboP), pl = smem_desc(sPl, 128, kSboP);
 #pragma unroll
                     for (int ks = 0; ks < kC / 16; ++ks) {
-                        const uint64_t b = smem_desc(sV1 + ks * 2 * kLboV1, kLboV1, 128);
-                        mma_bf16(tO, smem_desc(sPh + ks * 256, 128, kSboP), b, id, ks > 0 ? 1u : 0u);
-                        mma_bf16(tO, smem_desc(sPl + ks * 256, 128, kSboP), b, id, 1u);
+                        const uint64_t b = bv + (2 * kLboV1 / 16) * ks;
+                        mma_bf16(tO, ph + 16 * ks, b, id, ks > 0 ? 1u : 0u);
+                        mma_bf16(tO, pl + 16 * ks, b, id, 1u);
                     }
                 }
             }
@@ -347,15 +355,13 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
                 fence_after_sync();
                 TA_PHASE(1, 12, true);
                 if (good) {
+                    const uint64_t ah = smem_desc(sQh, 128, kSboPhiQ), al = smem_desc(sQl, 128, kSboPhiQ);
+                    const uint64_t bs = smem_desc(sS, kLboS, 128);
 #pragma unroll
                     for (int ks = 0; ks < kFP / 16; ++ks) {
-                        const uint64_t ah = smem_desc(sQh + ks * 256, 128, kSboPhiQ);
-                        const uint64_t al = smem_desc(sQl + ks * 256, 128, kSboPhiQ);
-                        const uint64_t bh_ = smem_desc(sSh + ks * 2 * kLboS, kLboS, 128);
-                        const uint64_t bl_ = smem_desc(sSl + ks * 2 * kLboS, kLboS, 128);
-                        mma_bf16(tO, ah, bh_, id, 1u);
-                        mma_bf16(tO, ah, bl_, id, 1u);
-                        mma_bf16(tO, al, bh_, id, 1u);
+                        const uint64_t b = bs + (2 * kLboS / 16) * ks;
+                        mma_bf16(tO, ah + 16 * ks, b, id160, 1u);
+                        mma_bf16(tO, al + 16 * ks, b, id, 1u);
                     }
                 }
             }
@@ -483,18 +489,30 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
                 const float xs[8] = {sa[i].x, sa[i].y, sa[i].z, sa[i].w, sb[i].x, sb[i].y, sb[i].z, sb[i].w};
                 uint4 hi, lo;
                 split8(xs, hi, lo);
-                *reinterpret_cast<uint4*>(sSh + mnmaj(f, g, kLboS)) = hi;
-                *reinterpret_cast<uint4*>(sSl + mnmaj(f, g, kLboS)) = lo;
+                *reinterpret_cast<uint4*>(sS + mnmaj(f, g, kLboS)) = hi;
+                *reinterpret_cast<uint4*>(sS + mnmaj(f, 10 + g, kLboS)) = lo;
             }
             if (tid < kFP) {
                 const float xs[8] = {zf, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 uint4 hi, lo;
                 split8(xs, hi, lo);
-                *reinterpret_cast<uint4*>(sSh + mnmaj(tid, 8, kLboS)) = hi;
-                *reinterpret_cast<uint4*>(sSl + mnmaj(tid, 8, kLboS)) = lo;
-                *reinterpret_cast<uint4*>(sSh + mnmaj(tid, 9, kLboS)) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(sSl + mnmaj(tid, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(sS + mnmaj(tid, 8, kLboS)) = hi;
+                *reinterpret_cast<uint4*>(sS + mnmaj(tid, 18, kLboS)) = lo;
+                *reinterpret_cast<uint4*>(sS + mnmaj(tid, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(sS + mnmaj(tid, 19, kLboS)) = make_uint4(0, 0, 0, 0);
             }
+            // O columns 80..159 start at zero: the read-out MMAs into them accumulate
+            if (half == 0) {
+                uint32_t z[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) z[i] = 0;
+                const uint32_t lo_ = (uint32_t)((warp & 3) * 32) << 16;
+                tmem_st32(tO + lo_ + 80, z);
+                tmem_st32(tO + lo_ + 112, z);
+                tmem_st16(tO + lo_ + 144, *reinterpret_cast<uint32_t(*)[16]>(z));
+                tmem_st_wait();
+            }
+            fence_before_sync();
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bar_ops);
             TA_PHASE(1, 7, tid == 0);
@@ -510,8 +528,17 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
             tmem_ld32(tO + lane_off + half * 32, o);
             tmem_ld16(tO + lane_off + kDV, dn);
             tmem_ld_wait();
+            float d2 = 0.f;
+            if (inter) {
+                float o2[32];
+                tmem_ld32(tO + lane_off + kNV + half * 32, o2);
+                d2 = tmem_ld1(tO + lane_off + kNV + kDV);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] += o2[i];
+            }
             if (valid) {
-                const float r = __frcp_rn(dn[0]);
+                const float r = __frcp_rn(dn[0] + d2);
                 float4* dst = reinterpret_cast<float4*>(out + tok * kDV + half * 32);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
@@ -527,7 +554,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     __syncthreads();
     if (warp == 8) {
         fence_after_sync();
-        tmem_dealloc(tbase, 256);
+        tmem_dealloc(tbase, 512);
     }
     TA_PHASE(1, 14, tid == 0);
 }
