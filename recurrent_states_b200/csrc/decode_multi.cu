@@ -38,14 +38,17 @@ struct MultiLayout {
     uint32_t s, pk, pq, xq, xk, vv, p, red, zr, bytes;
 };
 
+// phi(k_j), phi(q_i) are stored feature-major with the block's tokens
+// contiguous ([F][Tp], Tp = T rounded up to 4, zero padded), so that the row
+// loop reads the coefficients of four tokens with one 16-byte load.
 __host__ __device__ inline MultiLayout multi_layout(int T, int d, int dv, int F, uint32_t state_bytes) {
     auto al = [](uint32_t x) { return (x + 127u) & ~127u; };
-    const uint32_t Fp = (uint32_t)((F + 3) & ~3);
+    const uint32_t Tp = (uint32_t)((T + 3) & ~3);
     MultiLayout L;
     L.s = 0;
     L.pk = al(state_bytes);
-    L.pq = L.pk + al((uint32_t)T * Fp * 4);
-    L.xq = L.pq + al((uint32_t)T * Fp * 4);
+    L.pq = L.pk + al((uint32_t)F * Tp * 4);
+    L.xq = L.pq + al((uint32_t)F * Tp * 4);
     L.xk = L.xq + al((uint32_t)(T * d) * 4);
     L.vv = L.xk + al((uint32_t)(T * d) * 4);
     L.p = L.vv + al((uint32_t)(T * dv) * 4);
@@ -66,7 +69,7 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
     __shared__ __align__(8) uint64_t bar;
     __shared__ float qc[kMaxN];
     const MultiLayout L = multi_layout(T, d, DV, F, bytes);
-    const int Fp = (F + 3) & ~3;
+    const int Tp = (T + 3) & ~3;
     const float* S = reinterpret_cast<const float*>(dsm + L.s);
     float* pk = reinterpret_cast<float*>(dsm + L.pk);
     float* pq = reinterpret_cast<float*>(dsm + L.pq);
@@ -93,12 +96,13 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
     if (tid < n) qc[tid] = query_coeff(tid, tau);
     __syncthreads();
     const PackedFeat* tab = feat_table(d, n);
-    for (int e = tid; e < T * F; e += kThreads) {
-        const int j = e / F, f = e % F;
+    for (int f = tid; f < F; f += kThreads) {  // one descriptor load per feature, all tokens
         const FeatDesc dk = tab ? desc_from_packed(tab[f], qc, false) : make_desc(d, n, f, tau, false);
         const FeatDesc dq = tab ? desc_from_packed(tab[f], qc, true) : make_desc(d, n, f, tau, true);
-        pk[j * Fp + f] = eval_desc(dk, xk + j * d);
-        pq[j * Fp + f] = eval_desc(dq, xq + j * d);
+        for (int j = 0; j < Tp; ++j) {
+            pk[f * Tp + j] = j < T ? eval_desc(dk, xk + j * d) : 0.f;
+            pq[f * Tp + j] = j < T ? eval_desc(dq, xq + j * d) : 0.f;
+        }
     }
     for (int e = tid; e < T * T; e += kThreads) {
         const int i = e / T, j = e % T;
@@ -125,28 +129,35 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
     float4 y[kTMax];
 #pragma unroll
     for (int i = 0; i < kTMax; ++i) y[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto fma4 = [](float c, const float4& a, float4& acc) {
+        acc.x = fmaf(c, a.x, acc.x);
+        acc.y = fmaf(c, a.y, acc.y);
+        acc.z = fmaf(c, a.z, acc.z);
+        acc.w = fmaf(c, a.w, acc.w);
+    };
     for (int r = rs; r < F; r += RS) {
         float4 s = S4[r * DV4 + cg];
+        const float4* cq = reinterpret_cast<const float4*>(pq + r * Tp);
 #pragma unroll
-        for (int i = 0; i < kTMax; ++i) {
-            if (i < T) {
-                const float b = pq[i * Fp + r];
-                y[i].x = fmaf(b, s.x, y[i].x);
-                y[i].y = fmaf(b, s.y, y[i].y);
-                y[i].z = fmaf(b, s.z, y[i].z);
-                y[i].w = fmaf(b, s.w, y[i].w);
+        for (int i4 = 0; i4 < kTMax / 4; ++i4) {
+            if (4 * i4 < T) {
+                const float4 c = cq[i4];
+                fma4(c.x, s, y[4 * i4]);
+                fma4(c.y, s, y[4 * i4 + 1]);
+                fma4(c.z, s, y[4 * i4 + 2]);
+                fma4(c.w, s, y[4 * i4 + 3]);
             }
         }
         if (G4) {
+            const float4* ck = reinterpret_cast<const float4*>(pk + r * Tp);
 #pragma unroll
-            for (int j = 0; j < kTMax; ++j) {
-                if (j < T) {
-                    const float a = pk[j * Fp + r];
-                    const float4 vj = V4[j * DV4 + cg];
-                    s.x = fmaf(a, vj.x, s.x);
-                    s.y = fmaf(a, vj.y, s.y);
-                    s.z = fmaf(a, vj.z, s.z);
-                    s.w = fmaf(a, vj.w, s.w);
+            for (int j4 = 0; j4 < kTMax / 4; ++j4) {
+                if (4 * j4 < T) {  // padded tokens have coefficient 0 (and finite v rows)
+                    const float4 a = ck[j4];
+                    fma4(a.x, V4[(4 * j4) * DV4 + cg], s);
+                    if (4 * j4 + 1 < T) fma4(a.y, V4[(4 * j4 + 1) * DV4 + cg], s);
+                    if (4 * j4 + 2 < T) fma4(a.z, V4[(4 * j4 + 2) * DV4 + cg], s);
+                    if (4 * j4 + 3 < T) fma4(a.w, V4[(4 * j4 + 3) * DV4 + cg], s);
                 }
             }
             G4[r * DV4 + cg] = s;
@@ -161,11 +172,11 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
         float z = Z[f];
 #pragma unroll
         for (int i = 0; i < kTMax; ++i)
-            if (i < T) yz[i] = fmaf(pq[i * Fp + f], z, yz[i]);
+            if (i < T) yz[i] = fmaf(pq[f * Tp + i], z, yz[i]);
         if (GZ) {
 #pragma unroll
             for (int j = 0; j < kTMax; ++j)
-                if (j < T) z += pk[j * Fp + f];
+                if (j < T) z += pk[f * Tp + j];
             GZ[f] = z;
         }
     }
