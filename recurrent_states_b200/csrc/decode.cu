@@ -187,167 +187,6 @@ decode_tma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     TA_PHASE(3, 6, tid == 0);
 }
 
-// Persistent variant for states small enough that two of them fit a CTA's
-// shared memory twice over (two CTAs per SM): each CTA walks heads
-// blockIdx.x, blockIdx.x + gridDim.x, ... and, while it updates one head's
-// state, the bulk copy of the next head's state and the plain loads of the
-// next head's token are already in flight, so HBM sees a continuous stream
-// instead of one wave of CTAs, a gap, and a partial second wave.
-constexpr int kPersistThreads = 256;
-// Largest shared-memory footprint (two states plus features) that takes the
-// persistent kernel; 0 (the default) keeps every shape on the one-CTA-per-head
-// kernel, which measured faster on the decode workload (64 x 16 heads of
-// 153 x 65 floats).  Two CTAs per SM need at most about 100 KB each.
-#ifndef TA_DECODE_PERSIST_MAX_DYN
-#define TA_DECODE_PERSIST_MAX_DYN 0
-#endif
-constexpr size_t kPersistMaxDyn = TA_DECODE_PERSIST_MAX_DYN;
-constexpr int kPersistWarps = kPersistThreads / 32;
-constexpr int kPersistDescPerThread = (kTmaMaxFeatures + kPersistThreads - 1) / kPersistThreads;
-
-template <typename Tin, int DV4>
-__global__ void __launch_bounds__(kPersistThreads, 2)
-decode_persist_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-                      float* __restrict__ state, float* __restrict__ out, int BH, int d, int n, float tau, int F,
-                      int64_t stride, uint32_t bytes, unsigned int* __restrict__ err) {
-    constexpr int DV = DV4 * 4;
-    constexpr int RS = kPersistThreads / DV4;  // row sets
-    extern __shared__ __align__(128) unsigned char dsm[];
-    __shared__ float xq[kMaxDk], xk[kMaxDk], vv[DV], qc[kMaxN];
-    __shared__ float4 red[kPersistWarps][DV4];
-    __shared__ float zr[kPersistWarps];
-    __shared__ __align__(8) uint64_t bar[2];
-
-    const uint32_t sbytes = (bytes + 127u) & ~127u;
-    float* pk = reinterpret_cast<float*>(dsm + 2 * sbytes);
-    float* pq = pk + ((F + 3) & ~3);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    auto issue_load = [&](int head, int buf) {
-        ptx::mbar_arrive_expect_tx(&bar[buf], bytes);
-        ptx::bulk_g2s(dsm + buf * sbytes, state + (int64_t)head * stride, bytes, &bar[buf]);
-    };
-    if (tid == 0) {
-        ptx::mbar_init(&bar[0], 1);
-        ptx::mbar_init(&bar[1], 1);
-        ptx::fence_mbar_init();
-        issue_load(blockIdx.x, 0);
-    }
-    const PackedFeat* tab = feat_table(d, n);
-    PackedFeat pf[kPersistDescPerThread];
-#pragma unroll
-    for (int j = 0; j < kPersistDescPerThread; ++j) {
-        const int f = tid + j * kPersistThreads;
-        if (tab && f < F) pf[j] = tab[f];
-    }
-    if (tid < n) qc[tid] = query_coeff(tid, tau);
-    float aq = 0.f, ak = 0.f, av = 0.f;
-    {
-        const int h = blockIdx.x;
-        if (tid < d) {
-            aq = ldf(q + (int64_t)h * d + tid);
-            ak = ldf(k + (int64_t)h * d + tid);
-        }
-        if (tid < DV) av = ldf(v + (int64_t)h * DV + tid);
-    }
-    const int cg = tid % DV4, rs = tid / DV4;
-
-    int i = 0;
-    for (int h = blockIdx.x; h < BH; h += gridDim.x, ++i) {
-        const int buf = i & 1;
-        const int hn = h + gridDim.x;
-        // the other buffer was last read in the previous iteration, before
-        // the barrier that ended it
-        if (tid == 0 && hn < BH) issue_load(hn, buf ^ 1);
-        if (tid < d) {
-            xq[tid] = aq;
-            xk[tid] = ak;
-        }
-        if (tid < DV) vv[tid] = av;
-        if (hn < BH) {  // next head's token, consumed next iteration
-            if (tid < d) {
-                aq = ldf(q + (int64_t)hn * d + tid);
-                ak = ldf(k + (int64_t)hn * d + tid);
-            }
-            if (tid < DV) av = ldf(v + (int64_t)hn * DV + tid);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < kPersistDescPerThread; ++j) {
-            const int f = tid + j * kPersistThreads;
-            if (f < F) {
-                const FeatDesc dk = tab ? desc_from_packed(pf[j], qc, false) : make_desc(d, n, f, tau, false);
-                const FeatDesc dq = tab ? desc_from_packed(pf[j], qc, true) : make_desc(d, n, f, tau, true);
-                pk[f] = eval_desc(dk, xk);
-                pq[f] = eval_desc(dq, xq);
-            }
-        }
-        const bool landed = ptx::mbar_wait(&bar[buf], (uint32_t)(i >> 1) & 1u, kWaitPolls);
-        if (!__syncthreads_and(landed)) {
-            if (tid == 0) atomicOr(err, kErrDecodeLoad);
-            // bounded waits for the copies that may still be in flight
-            ptx::mbar_wait(&bar[buf], (uint32_t)(i >> 1) & 1u, kWaitPolls);
-            if (hn < BH) ptx::mbar_wait(&bar[buf ^ 1], (uint32_t)((i + 1) >> 1) & 1u, kWaitPolls);
-            return;
-        }
-
-        const float* S = reinterpret_cast<const float*>(dsm + buf * sbytes);
-        float* gS = state + (int64_t)h * stride;
-        const float4 v4 = reinterpret_cast<const float4*>(vv)[cg];
-        const float4* S4 = reinterpret_cast<const float4*>(S);
-        float4* G4 = reinterpret_cast<float4*>(gS);
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int r = rs; r < F; r += RS) {
-            const float a = pk[r], b = pq[r];
-            float4 s = S4[r * DV4 + cg];
-            s.x = fmaf(a, v4.x, s.x);
-            s.y = fmaf(a, v4.y, s.y);
-            s.z = fmaf(a, v4.z, s.z);
-            s.w = fmaf(a, v4.w, s.w);
-            G4[r * DV4 + cg] = s;
-            y.x = fmaf(b, s.x, y.x);
-            y.y = fmaf(b, s.y, y.y);
-            y.z = fmaf(b, s.z, y.z);
-            y.w = fmaf(b, s.w, y.w);
-        }
-        float yz = 0.f;
-        const float* Z = S + F * DV;
-        float* GZ = gS + (int64_t)F * DV;
-        for (int f = tid; f < F; f += kPersistThreads) {
-            const float z = Z[f] + pk[f];
-            GZ[f] = z;
-            yz = fmaf(pq[f], z, yz);
-        }
-        // this buffer's reads come before the next bulk copy into it
-        ptx::fence_proxy_async_smem();
-#pragma unroll
-        for (int o = DV4; o < 32; o <<= 1) {
-            y.x += __shfl_xor_sync(0xffffffffu, y.x, o);
-            y.y += __shfl_xor_sync(0xffffffffu, y.y, o);
-            y.z += __shfl_xor_sync(0xffffffffu, y.z, o);
-            y.w += __shfl_xor_sync(0xffffffffu, y.w, o);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) yz += __shfl_xor_sync(0xffffffffu, yz, o);
-        if (lane < DV4) red[warp][lane] = y;
-        if (lane == 0) zr[warp] = yz;
-        __syncthreads();
-        if (tid < DV) {
-            const int g = tid >> 2, c = tid & 3;
-            float acc = 0.f, den = 0.f;
-#pragma unroll
-            for (int w = 0; w < kPersistWarps; ++w) {
-                const float4 t = red[w][g];
-                acc += c == 0 ? t.x : c == 1 ? t.y : c == 2 ? t.z : t.w;
-                den += zr[w];
-            }
-            out[(int64_t)h * DV + tid] = acc / den;
-        }
-        // red/zr are rewritten only after the next iteration's two barriers
-    }
-}
-
 constexpr int kFeatTile = 1024;  // features whose phi(q), phi(k) sit in smem at once
 constexpr int kRows = 10;        // S_v rows per thread held in registers per batch
 
@@ -465,30 +304,6 @@ cudaError_t launch_tma(const Tin* q, const Tin* k, const Tin* v, float* state, f
     return cudaGetLastError();
 }
 
-template <typename Tin, int DV4>
-cudaError_t launch_persist(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
-                           int n, float tau, int F, int64_t stride, uint32_t bytes, size_t dyn,
-                           unsigned int* err, cudaStream_t stream) {
-    auto fn = decode_persist_kernel<Tin, DV4>;
-    static std::once_flag once[kMaxDevices];
-    static cudaError_t set_err[kMaxDevices];
-    static int num_sms[kMaxDevices];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(once[dev], [&]() {
-        set_err[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPersistMaxDyn);
-        if (set_err[dev] == cudaSuccess)
-            set_err[dev] = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
-    });
-    if (set_err[dev] != cudaSuccess) return set_err[dev];
-    const int grid = BH < 2 * num_sms[dev] ? BH : 2 * num_sms[dev];
-    TA_TIMED(stream, "decode_persist_kernel",
-             fn<<<grid, kPersistThreads, dyn, stream>>>(q, k, v, state, out, BH, d, n, tau, F, stride, bytes, err));
-    return cudaGetLastError();
-}
-
 }  // namespace
 
 template <typename Tin>
@@ -504,16 +319,6 @@ cudaError_t launch_decode(const Tin* q, const Tin* k, const Tin* v, float* state
     if (err != nullptr) {  // many heads of a small state: the persistent warp-specialised kernel
         const cudaError_t e = launch_decode_ws(q, k, v, state, out, BH, d, dv, n, tau, F, stride, stream);
         if (e != cudaErrorNotSupported) return e;
-    }
-    const size_t dyn2 = 2 * (size_t)((bytes + 127u) & ~127u) + 2 * (size_t)((F + 3) & ~3) * 4;
-    if (tma_ok && kPersistMaxDyn > 0 && dyn2 <= kPersistMaxDyn) {
-        switch (dv) {
-            case 16: return launch_persist<Tin, 4>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn2, err, stream);
-            case 32: return launch_persist<Tin, 8>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn2, err, stream);
-            case 64: return launch_persist<Tin, 16>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn2, err, stream);
-            case 128: return launch_persist<Tin, 32>(q, k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, dyn2, err, stream);
-            default: break;
-        }
     }
     if (tma_ok) {
         switch (dv) {
