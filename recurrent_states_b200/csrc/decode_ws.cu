@@ -7,12 +7,23 @@
 // One CTA per SM walks the heads blockIdx.x, blockIdx.x + gridDim.x, ...
 // One producer thread keeps a ring of state buffers in shared memory full:
 // for each head a bulk copy of its state and of its new token (q, k, v)
-// completing on the buffer's mbarrier, issued as soon as the buffer is free,
-// so several heads' loads per SM are always in flight.  Four consumer
-// warpgroups take the heads in turn; a warpgroup evaluates phi(k), phi(q) for
-// its head, updates the rows (one 16-byte column group per thread per row,
-// stored straight to HBM), reduces the read-out and writes o, synchronising
-// only its own 128 threads (named barriers), then hands the buffer back.
+// completing on the buffer's mbarrier, issued as soon as the buffer is free
+// (the first copies before anything else in the kernel), so several heads'
+// loads per SM are always in flight.  Four consumer warpgroups take the heads
+// in turn; a warpgroup evaluates phi(k), phi(q) for its head, updates the rows
+// (one 16-byte column group per thread per row, stored straight to HBM),
+// reduces the read-out and writes o, synchronising only its own 128 threads
+// (named barriers), then hands the buffer back.
+//
+// The ring holds a multiple of four buffers, so head i's buffer (i mod the
+// ring size) is only ever consumed by warpgroup i mod 4, in order: no
+// warpgroup can wait on a buffer phase while an earlier phase of the same
+// buffer is still outstanding, which a parity wait could not tell apart.
+//
+// With at most 256 features the series has degree <= 2 for every supported
+// d_k (d_k 16: n <= 3; d_k 32, 64: n <= 2), so each thread derives its
+// features' indices and weights arithmetically once, with no table lookup
+// in front of the first copies.
 #include <mutex>
 
 #include "common.cuh"
@@ -29,7 +40,7 @@ constexpr int kWG = 4;                      // consumer warpgroups
 constexpr int kWGThreads = 128;
 constexpr int kThreadsWS = kWG * kWGThreads + 32;
 constexpr int kMaxF = 256;
-constexpr int kMaxBuf = 6;
+constexpr int kMaxBuf = 8;  // a multiple of kWG
 constexpr uint32_t kWaitPolls = 1u << 22;
 constexpr size_t kMaxDynWS = 218 * 1024;  // with the static arrays, within the 227 KB per CTA
 constexpr int kMaxDevices = 64;
@@ -40,6 +51,31 @@ struct WGArea {                 // per consumer warpgroup
     float zr[4];
     int fail;                   // written only before a warpgroup barrier, read after it
 };
+
+// Feature f of degree <= 2 over d_k = d in the library's order (degree-major,
+// non-decreasing index pairs in lexicographic order): degree m, indices i <= j
+// and the multinomial weight sqrt(m!/alpha!) (sqrt 2 for i != j, else 1).
+__device__ __forceinline__ void feature_deg2(int d, int f, int& m, int& i, int& j, float& w) {
+    m = 0;
+    i = 0;
+    j = 0;
+    w = 1.0f;
+    if (f == 0) return;
+    if (f <= d) {
+        m = 1;
+        i = f - 1;
+        return;
+    }
+    int r = f - 1 - d, a = 0;
+    while (r >= d - a) {
+        r -= d - a;
+        ++a;
+    }
+    m = 2;
+    i = a;
+    j = a + r;
+    if (i != j) w = 1.41421356237309505f;
+}
 
 __device__ __forceinline__ void wg_sync(int wg) {
     asm volatile("bar.sync %0, %1;" ::"r"(1 + wg), "r"(kWGThreads) : "memory");
@@ -52,8 +88,6 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                  int64_t stride, uint32_t bytes, uint32_t buf_bytes, int nbuf, unsigned int* __restrict__ err) {
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ __align__(8) uint64_t full[kMaxBuf], empty[kMaxBuf];
-    __shared__ FeatDesc dk_s[kMaxF], dq_s[kMaxF];
-    __shared__ float qc[kMaxN];
     __shared__ int s_bad;
     WGArea* wga = reinterpret_cast<WGArea*>(dsm + (size_t)nbuf * buf_bytes);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -62,40 +96,39 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     // token area of a buffer: q, k, v rows right after the state, 16-byte aligned
     const uint32_t offq = (bytes + 15u) & ~15u, offk = offq + ((tok_in + 15u) & ~15u),
                    offv = offk + ((tok_in + 15u) & ~15u);
+    const int producer = kWG * kWGThreads;
+    auto issue = [&](int i) {
+        const int b = i % nbuf;
+        const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+        unsigned char* buf = dsm + (size_t)b * buf_bytes;
+        ptx::mbar_arrive_expect_tx(&full[b], bytes + 2 * tok_in + tok_v);
+        ptx::bulk_g2s(buf, state + h * stride, bytes, &full[b]);
+        ptx::bulk_g2s(buf + offq, q + h * d, tok_in, &full[b]);
+        ptx::bulk_g2s(buf + offk, k + h * d, tok_in, &full[b]);
+        ptx::bulk_g2s(buf + offv, v + h * kDV, tok_v, &full[b]);
+    };
 
-    if (tid == 0) {
+    // the producer sets up the ring and starts the first copies at once
+    int issued = 0;
+    if (tid == producer) {
         for (int i = 0; i < nbuf; ++i) {
             ptx::mbar_init(&full[i], 1);
             ptx::mbar_init(&empty[i], 1);
         }
-        s_bad = 0;
         ptx::fence_mbar_init();
+        for (; issued < nbuf && issued < nheads; ++issued) issue(issued);
     }
-    if (tid < n) qc[tid] = query_coeff(tid, tau);
+    if (tid == 0) s_bad = 0;
     if (tid < kWG) wga[tid].fail = 0;
-    __syncthreads();
-    {
-        const PackedFeat* tab = feat_table(d, n);
-        for (int f = tid; f < F; f += kThreadsWS) {
-            dk_s[f] = tab ? desc_from_packed(tab[f], qc, false) : make_desc(d, n, f, tau, false);
-            dq_s[f] = tab ? desc_from_packed(tab[f], qc, true) : make_desc(d, n, f, tau, true);
-        }
-    }
     __syncthreads();
 
     if (warp == kWG * kWGThreads / 32) {
         if (lane == 0) {
-            int i = 0;
+            int i = issued;
             for (; i < nheads; ++i) {
                 const int b = i % nbuf;
-                if (i >= nbuf && !ptx::mbar_wait_or_abort(&empty[b], ((i / nbuf) - 1) & 1, kWaitPolls, &s_bad)) break;
-                const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
-                unsigned char* buf = dsm + (size_t)b * buf_bytes;
-                ptx::mbar_arrive_expect_tx(&full[b], bytes + 2 * tok_in + tok_v);
-                ptx::bulk_g2s(buf, state + h * stride, bytes, &full[b]);
-                ptx::bulk_g2s(buf + offq, q + h * d, tok_in, &full[b]);
-                ptx::bulk_g2s(buf + offk, k + h * d, tok_in, &full[b]);
-                ptx::bulk_g2s(buf + offv, v + h * kDV, tok_v, &full[b]);
+                if (!ptx::mbar_wait_or_abort(&empty[b], ((i / nbuf) - 1) & 1, kWaitPolls, &s_bad)) break;
+                issue(i);
             }
             // copies that no warpgroup consumed (only after a failure) land before the CTA leaves
             for (int j = (i > nbuf ? i - nbuf : 0); j < i; ++j)
@@ -105,8 +138,15 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         const int wg = warp >> 2, t = tid & (kWGThreads - 1), wl = (warp & 3);
         WGArea& A = wga[wg];
         const int cg = t % kDV4, rs = t / kDV4;  // 8 row sets
+        // this thread's features t and t + 128: phi_f(x) = w x_i x_j (factors
+        // past the degree are 1); the query weight carries tau^m / m!
+        int m0, i0, j0, m1, i1, j1;
+        float w0, w1;
+        feature_deg2(d, t < F ? t : 0, m0, i0, j0, w0);
+        feature_deg2(d, t + kWGThreads < F ? t + kWGThreads : 0, m1, i1, j1, w1);
+        const float wq0 = w0 * query_coeff(m0, tau), wq1 = w1 * query_coeff(m1, tau);
         for (int i = wg; i < nheads; i += kWG) {
-            const int b = i % nbuf;
+            const int b = i % nbuf;  // == wg modulo kWG: only this warpgroup consumes buffer b
             if (!ptx::mbar_wait_or_abort(&full[b], (i / nbuf) & 1, kWaitPolls, &s_bad)) A.fail = 1;
             wg_sync(wg);
             if (A.fail) break;  // the same value for all 128 threads: set only before this barrier
@@ -115,13 +155,17 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             const Tin* xq = reinterpret_cast<const Tin*>(buf + offq);
             const Tin* xk = reinterpret_cast<const Tin*>(buf + offk);
             const Tin* vv = reinterpret_cast<const Tin*>(buf + offv);
-            for (int f = t; f < F; f += kWGThreads) {
-                const FeatDesc fk = dk_s[f], fq = dq_s[f];
-                float pk = fk.w, pq = fq.w;
-                for (int s = 0; s < fk.m; ++s) pk *= to_float(xk[(fk.packed >> (8 * s)) & 0xff]);
-                for (int s = 0; s < fq.m; ++s) pq *= to_float(xq[(fq.packed >> (8 * s)) & 0xff]);
-                A.pk[f] = pk;
-                A.pq[f] = pq;
+            if (t < F) {
+                const float ki = m0 >= 1 ? to_float(xk[i0]) : 1.0f, kj = m0 >= 2 ? to_float(xk[j0]) : 1.0f;
+                const float qi = m0 >= 1 ? to_float(xq[i0]) : 1.0f, qj = m0 >= 2 ? to_float(xq[j0]) : 1.0f;
+                A.pk[t] = w0 * ki * kj;
+                A.pq[t] = wq0 * qi * qj;
+            }
+            if (t + kWGThreads < F) {
+                const float ki = m1 >= 1 ? to_float(xk[i1]) : 1.0f, kj = m1 >= 2 ? to_float(xk[j1]) : 1.0f;
+                const float qi = m1 >= 1 ? to_float(xq[i1]) : 1.0f, qj = m1 >= 2 ? to_float(xq[j1]) : 1.0f;
+                A.pk[t + kWGThreads] = w1 * ki * kj;
+                A.pq[t + kWGThreads] = wq1 * qi * qj;
             }
             const float4 v4 = make_float4(to_float(vv[4 * cg]), to_float(vv[4 * cg + 1]), to_float(vv[4 * cg + 2]),
                                           to_float(vv[4 * cg + 3]));
@@ -186,7 +230,8 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
 template <typename Tin>
 cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
                              int dv, int n, float tau, int64_t F, int64_t stride, cudaStream_t stream) {
-    if (dv != kDV || F > kMaxF || (d * (int)sizeof(Tin)) % 16 != 0) return cudaErrorNotSupported;
+    // features of degree <= 2 only (always the case for F <= 256 at the supported d_k)
+    if (dv != kDV || F > kMaxF || n > 3 || (d * (int)sizeof(Tin)) % 16 != 0) return cudaErrorNotSupported;
     static std::once_flag once[kMaxDevices];
     static cudaError_t set_err[kMaxDevices];
     static int num_sms[kMaxDevices];
@@ -206,9 +251,11 @@ cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* st
     const uint32_t buf_bytes = (bytes + 15u) / 16u * 16u + tok;
     const uint32_t buf_al = (buf_bytes + 127u) & ~127u;
     const size_t area = kWG * sizeof(WGArea);
+    // a multiple of the warpgroup count, so that every buffer has one consumer
     int nbuf = (int)((kMaxDynWS - area) / buf_al);
     if (nbuf > kMaxBuf) nbuf = kMaxBuf;
-    if (nbuf < 2) return cudaErrorNotSupported;
+    nbuf -= nbuf % kWG;
+    if (nbuf < kWG) return cudaErrorNotSupported;
     const size_t dyn = (size_t)nbuf * buf_al + area;
     unsigned int* err = device_error_word();
     if (!err) return cudaErrorNotSupported;

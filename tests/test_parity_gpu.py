@@ -245,6 +245,28 @@ def test_decode_from_zero_equals_prefill_reference(d, dv, n):
     assert state_block_errors(st, ref_st, d, dv, n) <= TOL["f32"]
 
 
+@pytest.mark.parametrize("d,n", [(16, 1), (16, 2), (16, 3), (32, 2), (64, 2)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_many_heads_from_zero(d, n, dtype):
+    """1,280 heads (several per SM, so the persistent decode kernel's buffer
+    ring wraps more than once), d_v 64, six steps from a zero state, against
+    the oracle's recurrent form over the same six tokens.  tau = 1 keeps every
+    kernel weight 1 + x (n = 2) non-negative for |x| <= 1: at tau = 2 a row of
+    one or two tokens can have a denominator near 1e-3, which alone turns fp32
+    rounding into errors above the fp32 bound."""
+    B, H, dv, N, tau = 80, 16, 64, 6, 1.0
+    q, k, v = synth.qkv(B, H, N, d, dv, seed=10 * d + n, dtype=dtype)
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    st = torch.zeros((B, H, TA.taylor_attn_state_stride(d, dv, n)), device=DEV)
+    fn = TA.taylor_attn_decode if dtype == "bf16" else TA.taylor_attn_decode_f32
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    outs = [fn(qd[:, :, i].contiguous(), kd[:, :, i].contiguous(), vd[:, :, i].contiguous(), st, n, tau)
+            for i in range(N)]
+    got = torch.stack(outs, dim=2)
+    assert row_scaled_max_err(f64(got), ref_out) <= TOL[dtype]
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL[dtype]
+
+
 def test_merge_and_split_prefill():
     """state(A) + state(B) from two prefills equals the oracle's state of A+B,
     and prefill then decode continues the sequence."""
