@@ -41,6 +41,10 @@ LARGE = dict(B=4, H=16, N=32768, d_k=64, d_v=64, n=3, tau=2.0)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes of one decode_ws_kernel launch on the decode workload, from an ncu
+# capture (read 40,991,488 + write 38,400); to be retaken whenever the kernel changes.
+DECODE_WS_DRAM_BYTES = 41_029_888
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -428,7 +432,11 @@ def run_ours(args, world, rank, local):
                              "achieved": round(dbytes / (dec_kernel_us * 1e-6) / 1e9, 2),
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(dbytes / (dec_kernel_us * 1e-6) / 1e9 / hbm_peak, 4),
-                             "algorithmic_bytes_per_launch": dbytes, "traffic": None},
+                             "algorithmic_bytes_per_launch": dbytes,
+                             "traffic": DECODE_WS_DRAM_BYTES if dk_name == "decode_ws_kernel" else None,
+                             "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of "
+                                             "this kernel on this workload (cold caches): the states are read "
+                                             "once, their updates stay in L2 within the step"},
             },
             "multi_token_decode": {
                 "workload": "B=64 H=16 d_k=16 d_v=64 n=3, T new tokens per head per call against the carried "
