@@ -283,6 +283,23 @@ def run_ours(args, world, rank, local):
     dec_warm_us = warm_ev[0].elapsed_time(warm_ev[1]) * 1e3 / dsteps
     dec_us_max = allmax(dec_us, world, dev)
 
+    # ---- the mean-centred softmax expansion (order 2) on the same carried
+    # states: same state traffic, a three-way read-out
+    for s in range(3):
+        flush_l2()
+        TA.taylor_attn_centred_decode(*toks[s], dstate, 2, dw["tau"], out=dout)
+    torch.cuda.synchronize()
+    TA.taylor_attn_timing_read()
+    TA.taylor_attn_timing_enable(True)
+    for s in range(dsteps):
+        flush_l2()
+        TA.taylor_attn_centred_decode(*toks[s], dstate, 2, dw["tau"], out=dout)
+    torch.cuda.synchronize()
+    TA.taylor_attn_timing_enable(False)
+    ckern = TA.taylor_attn_timing_read()
+    ck_name, (ck_launch, ck_ms) = max(ckern.items(), key=lambda kv: kv[1][1])
+    cen_kernel_us = ck_ms / ck_launch * 1e3
+
     # ---- batched multi-token decode: T new tokens per head per call, in place
     multi = {}
     for T in (4, 16):
@@ -437,6 +454,17 @@ def run_ours(args, world, rank, local):
                              "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of "
                                              "this kernel on this workload (cold caches): the states are read "
                                              "once, their updates stay in L2 within the step"},
+            },
+            "centred_decode": {
+                "workload": "mean-centred softmax expansion, order 2, one token per head per step on the decode "
+                            "workload's carried n=3 states (B=64 H=16 d_k=16 d_v=64), L2 flushed before each step",
+                "kernel": ck_name,
+                "kernel_us": round(cen_kernel_us, 3),
+                "roofline": {"bound": "hbm", "kernel": ck_name,
+                             "achieved": round(dbytes / (cen_kernel_us * 1e-6) / 1e9, 2),
+                             "peak": hbm_peak, "unit": "GB/s",
+                             "frac": round(dbytes / (cen_kernel_us * 1e-6) / 1e9 / hbm_peak, 4),
+                             "algorithmic_bytes_per_launch": dbytes, "traffic": None},
             },
             "multi_token_decode": {
                 "workload": "B=64 H=16 d_k=16 d_v=64 n=3, T new tokens per head per call against the carried "

@@ -154,6 +154,32 @@ TAYLOR_API int taylor_attn_decode_f32(const float* q, const float* k, const floa
                            float* out, int B, int H, int d_k, int d_v, int n, float tau,
                            cudaStream_t stream);
 
+/* One new token per (b, h) for causal attention with the mean-centred
+ * Taylor expansion of softmax instead of the truncated exponential kernel
+ * (Su Jianlin, "Taylor expansions of logsumexp and softmax", kexue.fm
+ * translation 11814, sections "Calculating the Gradient" and "Linear
+ * Attention"): the row of token i weights v_j, j <= i, by
+ * (1 + y_j + (y_j^2 - mean(y^2))/2) / (i + 1) with y_j = tau q.(k_j - kbar)
+ * and kbar the mean of those keys; order 1 drops the square term.  Weights
+ * are used as they are (they sum to one; no clamp of negative ones).
+ * The carried state is the n = 3 Taylor state of the same keys and values
+ * ([B][H][taylor_attn_state_stride(d_k, d_v, 3)], layout as
+ * taylor_attn_decode; its degree-0..2 blocks hold every prefix sum the
+ * expansion needs), updated in place with S + phi(k)[v | 1]^T exactly as
+ * taylor_attn_decode with n = 3 would; it can come from taylor_attn_prefill
+ * with n = 3 and stays valid for both read-outs.  q, k [B][H][d_k], v
+ * [B][H][d_v] bf16 (the _f32 variant: fp32); out [B][H][d_v] fp32.  order is
+ * 1 or 2 (else TAYLOR_ERR_UNSUPPORTED); d_k in 1..64, d_v a multiple of 4 up
+ * to 256; pointers 16-byte aligned.  No workspace. */
+TAYLOR_API int taylor_attn_centred_decode(const void* q, const void* k, const void* v, float* state_inout,
+                                          float* out, int B, int H, int d_k, int d_v, int order, float tau,
+                                          cudaStream_t stream);
+
+/* taylor_attn_centred_decode with fp32 q, k, v. */
+TAYLOR_API int taylor_attn_centred_decode_f32(const float* q, const float* k, const float* v,
+                                              float* state_inout, float* out, int B, int H, int d_k, int d_v,
+                                              int order, float tau, cudaStream_t stream);
+
 /* out = a + b over B*H states (abstract: states are additive across chunks,
  * so the state of a concatenation is the sum of the parts' states).  out may
  * alias a or b.  No workspace. */

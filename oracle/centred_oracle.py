@@ -36,10 +36,16 @@ Two forms, pinned against each other and against independent routes in
 ``centred_recurrent``   the linear-attention form: prefix sums of 1, k, v,
                         k v^T, k k^T and (k k^T) v^T, updated once per token,
                         and a read-out of quadratic forms in q (O(N d^2 d_v)).
+``centred_step_from_state``  one decode step whose prefix sums are carried
+                        in the n = 3 Taylor-kernel state S = sum phi(k)[v|1]^T
+                        (its degree-0, 1 and 2 blocks hold exactly those sums,
+                        the degree-2 block through phi_2(q).phi_2(k) = (q.k)^2).
 """
 from __future__ import annotations
 
 import numpy as np
+
+from oracle import taylor_oracle as T
 
 
 def softmax_expansion(x: np.ndarray, order: int) -> np.ndarray:
@@ -130,6 +136,40 @@ def centred_recurrent(q, k, v, order: int, tau: float = 1.0) -> np.ndarray:
             o = o + (sum_a2v - sum_a2[..., None] * V / n) / (2.0 * n)
         out[..., i, :] = o
     return out
+
+
+def centred_step_from_state(state, q, k, v, order: int, tau: float = 1.0):
+    """One new token against a carried n = 3 Taylor state.
+
+    state: [..., F, d_v + 1] (F = 1 + d + d(d+1)/2, the logical layout of the
+    Taylor oracle); q, k: [..., d]; v: [..., d_v].  The state is first updated
+    with phi(k)[v | 1]^T; then R_m = phi_m(q)^T S_m for m = 0, 1, 2 (weights
+    sqrt(m!/alpha!) only, no tau) give n = R_0[z], V = R_0[v], q.sum(k) =
+    R_1[z], q^T Kv = R_1[v], q^T KK q = R_2[z], q^T KKv q = R_2[v], and the
+    output is centred_recurrent's combination.  Returns (out, new state)."""
+    if order not in (1, 2):
+        raise ValueError("order must be 1 or 2")
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    S = np.array(state, dtype=np.float64)
+    d, dv = q.shape[-1], v.shape[-1]
+    phik = T.feature_map(k, 3)
+    phiq = T.feature_map(q, 3)
+    v1 = np.concatenate([v, np.ones(v.shape[:-1] + (1,))], axis=-1)
+    S = S + phik[..., :, None] * v1[..., None, :]
+    deg = T.feature_degrees(d, 3)
+    R = [np.einsum("...f,...fc->...c", phiq[..., deg == m], S[..., deg == m, :]) for m in range(3)]
+    n = R[0][..., dv]
+    V = R[0][..., :dv]
+    qkbar = R[1][..., dv] / n
+    qKv = R[1][..., :dv]
+    o = V / n[..., None] + tau * (qKv - qkbar[..., None] * V) / n[..., None]
+    if order >= 2:
+        sum_a2v = tau * tau * (R[2][..., :dv] - 2.0 * qkbar[..., None] * qKv + (qkbar ** 2)[..., None] * V)
+        sum_a2 = tau * tau * (R[2][..., dv] - n * qkbar ** 2)
+        o = o + (sum_a2v - (sum_a2 / n)[..., None] * V) / (2.0 * n[..., None])
+    return o, S
 
 
 def softmax_attention(q, k, v, tau: float = 1.0) -> np.ndarray:

@@ -120,6 +120,27 @@ int decode_impl(const Tin* q, const Tin* k, const Tin* v, float* state, float* o
                                          stride_of(d_k, d_v, n), stream));
 }
 
+template <typename Tin>
+int centred_decode_impl(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int B, int H,
+                        int d_k, int d_v, int order, float tau, cudaStream_t stream) {
+    if (B < 0 || H < 0) return TAYLOR_ERR_INVALID_ARG;
+    int rc = check_dims(d_k, d_v, 3);
+    if (rc != TAYLOR_OK) return rc;
+    if (order != 1 && order != 2) return TAYLOR_ERR_UNSUPPORTED;
+    if (!isfinite(tau)) return TAYLOR_ERR_INVALID_ARG;
+    const int64_t BH = (int64_t)B * H;
+    if (BH >= ((int64_t)1 << 31)) return TAYLOR_ERR_UNSUPPORTED;
+    if (BH == 0) return TAYLOR_OK;
+    if (!q || !k || !v || !state || !out) return TAYLOR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out))
+        return TAYLOR_ERR_MISALIGNED;
+    const int64_t F = ta::num_features(d_k, 3);
+    const cudaError_t e = ta::launch_centred_decode(q, k, v, state, out, (int)BH, d_k, d_v, order, tau, F,
+                                                    stride_of(d_k, d_v, 3), stream);
+    if (e == cudaErrorNotSupported) return TAYLOR_ERR_UNSUPPORTED;
+    return cuda_status(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -215,6 +236,19 @@ int taylor_attn_decode_f32(const float* q, const float* k, const float* v, float
                            float* out, int B, int H, int d_k, int d_v, int n, float tau,
                            cudaStream_t stream) {
     return decode_impl(q, k, v, state_inout, out, B, H, d_k, d_v, n, tau, stream);
+}
+
+int taylor_attn_centred_decode(const void* q, const void* k, const void* v, float* state_inout, float* out,
+                               int B, int H, int d_k, int d_v, int order, float tau, cudaStream_t stream) {
+    using bf = __nv_bfloat16;
+    return centred_decode_impl(static_cast<const bf*>(q), static_cast<const bf*>(k), static_cast<const bf*>(v),
+                               state_inout, out, B, H, d_k, d_v, order, tau, stream);
+}
+
+int taylor_attn_centred_decode_f32(const float* q, const float* k, const float* v, float* state_inout,
+                                   float* out, int B, int H, int d_k, int d_v, int order, float tau,
+                                   cudaStream_t stream) {
+    return centred_decode_impl(q, k, v, state_inout, out, B, H, d_k, d_v, order, tau, stream);
 }
 
 int taylor_attn_state_merge(const float* a, const float* b, float* out, int B, int H, int d_k,

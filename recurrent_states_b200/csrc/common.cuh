@@ -118,6 +118,32 @@ TA_HD FeatDesc make_desc(int d, int n, int64_t f, float tau, bool query) {
     return fd;
 }
 
+// Feature f of degree <= 2 over d_k = d, arithmetically (no table): degree m,
+// indices i <= j and the multinomial weight sqrt(m!/alpha!) (sqrt 2 for
+// i != j, else 1), in the order unrank() defines (degree-major, index pairs
+// in lexicographic order).  Factors past the degree are to be taken as 1.
+__device__ __forceinline__ void feature_deg2(int d, int f, int& m, int& i, int& j, float& w) {
+    m = 0;
+    i = 0;
+    j = 0;
+    w = 1.0f;
+    if (f == 0) return;
+    if (f <= d) {
+        m = 1;
+        i = f - 1;
+        return;
+    }
+    int r = f - 1 - d, a = 0;
+    while (r >= d - a) {
+        r -= d - a;
+        ++a;
+    }
+    m = 2;
+    i = a;
+    j = a + r;
+    if (i != j) w = 1.41421356237309505f;
+}
+
 // phi_f(x) for x in shared memory with element stride 1.
 __device__ __forceinline__ float eval_desc(const FeatDesc& fd, const float* x) {
     float p = fd.w;

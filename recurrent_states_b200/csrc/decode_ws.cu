@@ -52,31 +52,6 @@ struct WGArea {                 // per consumer warpgroup
     int fail;                   // written only before a warpgroup barrier, read after it
 };
 
-// Feature f of degree <= 2 over d_k = d in the library's order (degree-major,
-// non-decreasing index pairs in lexicographic order): degree m, indices i <= j
-// and the multinomial weight sqrt(m!/alpha!) (sqrt 2 for i != j, else 1).
-__device__ __forceinline__ void feature_deg2(int d, int f, int& m, int& i, int& j, float& w) {
-    m = 0;
-    i = 0;
-    j = 0;
-    w = 1.0f;
-    if (f == 0) return;
-    if (f <= d) {
-        m = 1;
-        i = f - 1;
-        return;
-    }
-    int r = f - 1 - d, a = 0;
-    while (r >= d - a) {
-        r -= d - a;
-        ++a;
-    }
-    m = 2;
-    i = a;
-    j = a + r;
-    if (i != j) w = 1.41421356237309505f;
-}
-
 __device__ __forceinline__ void wg_sync(int wg) {
     asm volatile("bar.sync %0, %1;" ::"r"(1 + wg), "r"(kWGThreads) : "memory");
 }

@@ -44,6 +44,8 @@ SIGNATURES = {
     "taylor_attn_prefill_from_state_f32": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_decode_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "taylor_attn_centred_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "taylor_attn_centred_decode_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_state_merge": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "taylor_attn_prefill_f32_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_prefill_noalloc_scratch_floats": (_I64, []),
@@ -246,8 +248,8 @@ def taylor_attn_prefill_noalloc_scratch_floats() -> int:
     return int(lib().taylor_attn_prefill_noalloc_scratch_floats())
 
 
-def _decode(name, q, k, v, state, n, tau, out, stream):
-    dtype = torch.bfloat16 if name == "taylor_attn_decode" else torch.float32
+def _decode(name, q, k, v, state, n, tau, out, stream, order=None):
+    dtype = torch.float32 if name.endswith("_f32") else torch.bfloat16
     if q.dim() != 3:
         raise ValueError("q, k must be [B, H, d_k] and v [B, H, d_v]")
     B, H, d_k = q.shape
@@ -259,8 +261,8 @@ def _decode(name, q, k, v, state, n, tau, out, stream):
     if out is None:
         out = torch.empty((B, H, d_v), dtype=torch.float32, device=q.device)
     _need(out, "out", torch.float32, q.device, (B, H, d_v))
-    rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), B, H, d_k, d_v, n,
-                              float(tau), _stream(stream))
+    rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), B, H, d_k, d_v,
+                              n if order is None else order, float(tau), _stream(stream))
     _check(rc, name)
     return out
 
@@ -273,6 +275,18 @@ def taylor_attn_decode(q, k, v, state, n: int, tau: float, out=None, stream=None
 
 def taylor_attn_decode_f32(q, k, v, state, n: int, tau: float, out=None, stream=None):
     return _decode("taylor_attn_decode_f32", q, k, v, state, n, tau, out, stream)
+
+
+def taylor_attn_centred_decode(q, k, v, state, order: int, tau: float, out=None, stream=None):
+    """One token per (b, h) with the mean-centred softmax expansion of order
+    1 or 2: bf16 q, k [B,H,d_k], v [B,H,d_v]; ``state`` is the n = 3 Taylor
+    state [B,H,stride(d_k, d_v, 3)], updated in place; returns out fp32
+    [B,H,d_v]."""
+    return _decode("taylor_attn_centred_decode", q, k, v, state, 3, tau, out, stream, order=order)
+
+
+def taylor_attn_centred_decode_f32(q, k, v, state, order: int, tau: float, out=None, stream=None):
+    return _decode("taylor_attn_centred_decode_f32", q, k, v, state, 3, tau, out, stream, order=order)
 
 
 def taylor_attn_state_merge(a, b, d_k: int, d_v: int, n: int, out=None, stream=None):

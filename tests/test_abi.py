@@ -92,6 +92,13 @@ def test_argument_errors_need_no_device():
     assert L.taylor_attn_feature_map(None, None, 0, 16, 3, 2.0, 1, None) == TA.TAYLOR_OK
     deg = np.empty(4, dtype=np.int32)
     assert L.taylor_attn_feature_index(16, 3, None, deg.ctypes.data) == TA.TAYLOR_ERR_INVALID_ARG
+    # the centred-expansion decode: order 1 or 2 only, same pointer and size rules
+    for order in (0, 3):
+        assert L.taylor_attn_centred_decode(p, p, p, p, p, 1, 1, 16, 64, order, 2.0, None) == TA.TAYLOR_ERR_UNSUPPORTED
+    assert L.taylor_attn_centred_decode(p, p, p, p, p, 1, 1, 16, 62, 2, 2.0, None) == TA.TAYLOR_ERR_UNSUPPORTED
+    assert L.taylor_attn_centred_decode(p, p, None, p, p, 1, 1, 16, 64, 2, 2.0, None) == TA.TAYLOR_ERR_INVALID_ARG
+    assert L.taylor_attn_centred_decode_f32(p, p, p, p + 4, p, 1, 1, 16, 64, 1, 2.0, None) == TA.TAYLOR_ERR_MISALIGNED
+    assert L.taylor_attn_centred_decode(None, None, None, None, None, 0, 3, 16, 64, 2, 2.0, None) == TA.TAYLOR_OK
 
 
 def test_layout_helpers_roundtrip():

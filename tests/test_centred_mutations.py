@@ -17,6 +17,7 @@ PINS = [
     lambda: [P.test_equal_keys_give_the_causal_prefix_mean(r) for r in (1, 2)],
     lambda: P.test_single_token_rows_return_their_value(),
     lambda: P.test_second_order_term_changes_the_output_and_first_order_does_not_see_it(),
+    lambda: [P.test_step_from_the_taylor_state_continues_the_sequence(r, 3, 2) for r in (1, 2)],
 ]
 
 

@@ -11,6 +11,7 @@ import pytest
 import torch
 
 from oracle import centred_oracle as O
+from oracle import taylor_oracle as T
 
 
 def _unit(rng, shape):
@@ -106,3 +107,20 @@ def test_second_order_term_changes_the_output_and_first_order_does_not_see_it():
     v3 = np.array([[1.0], [2.0], [5.0]])
     q3 = np.repeat(q, 3, axis=0)
     assert abs(O.centred_direct(q3, k3, v3, 1)[2, 0] - O.centred_direct(q3, k3, v3, 2)[2, 0]) > 1e-3
+
+
+@pytest.mark.parametrize("order", [1, 2])
+@pytest.mark.parametrize("d,dv", [(3, 2), (5, 4)])
+def test_step_from_the_taylor_state_continues_the_sequence(order, d, dv):
+    """Decode against the n = 3 Taylor state of a prefix equals the direct
+    form's last row over prefix + token, and the returned state is the
+    Taylor state of prefix + token."""
+    rng = np.random.default_rng(7 + d)
+    N = 17
+    q, k = _unit(rng, (2, N, d)), _unit(rng, (2, N, d))
+    v = rng.standard_normal((2, N, dv))
+    S = T.state_of(k[:, : N - 1], v[:, : N - 1], 3)
+    o, S1 = O.centred_step_from_state(S, q[:, -1], k[:, -1], v[:, -1], order, 1.7)
+    ref = O.centred_direct(q, k, v, order, 1.7)[:, -1]
+    assert np.abs(o - ref).max() <= 1e-12
+    assert np.abs(S1 - T.state_of(k, v, 3)).max() <= 1e-12
