@@ -48,6 +48,13 @@ centred_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
     float* red = pq + F;       // [3][nrs][dv] column partials per degree
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t h = blockIdx.x;
+    float* S = state + h * stride;
+    // the head's state starts towards L2 while the token and the features
+    // are prepared (16-byte aligned: the stride is a multiple of 32 floats)
+    if (tid == 0) {
+        const uint32_t bytes = (uint32_t)(((int64_t)F * (dv + 1) * 4 + 15) / 16 * 16);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(S), "r"(bytes) : "memory");
+    }
 
     for (int i = tid; i < d; i += kThreadsC) {
         xq[i] = to_float(q[h * d + i]);
@@ -64,7 +71,6 @@ centred_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
     }
     __syncthreads();
 
-    float* S = state + h * stride;
     const int cg = tid % dv4, rs = tid / dv4;
     if (rs < nrs) {
         const float4 v4 = make_float4(xv[4 * cg], xv[4 * cg + 1], xv[4 * cg + 2], xv[4 * cg + 3]);
