@@ -13,7 +13,7 @@
  *   - each term is an inner product of tensor powers, packed to the
  *     binom(d+m-1, m) non-decreasing monomials with weight sqrt(m!/alpha!);
  *   - so the causal history is n states, S += phi(k) [v|1]^T per token.
- * Readings (not fixed by the pages): tau^m/m! on the query side, inclusive
+ * Readings (not fixed by the paper's abstract): tau^m/m! on the query side, inclusive
  * causality, the ones column of [v|1] as normaliser, a plain quotient.
  *
  * Logical state layout here: S[head][F][dv+1] (last column = normaliser).

@@ -20,7 +20,7 @@ arXiv 2610.20637, abstract):
   rank-one outer product per token (abstract, first sentence), additive across
   chunks (abstract, second sentence).
 
-Readings where the pages are silent (each listed in the design notes):
+Readings where the sources are silent (each listed in the design notes):
 n terms means degrees 0..n-1; tau multiplies q.k inside the series; the
 per-degree factor tau^m/m! sits on the query side so that the state is
 tau-free; the multinomial weight sqrt(m!/alpha!) sits on both sides;
@@ -28,7 +28,7 @@ causality is inclusive (token i attends to j <= i); the normaliser is the
 extra ones column of [v | 1]; the output is the plain quotient, no epsilon.
 
 Every function here is pinned by tests in ``tests/test_oracle*.py`` against
-closed forms, library routines, brute force and the numbers the pages print.
+closed forms, library routines, brute force and the numbers the abstract prints.
 """
 from __future__ import annotations
 

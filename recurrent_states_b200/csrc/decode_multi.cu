@@ -1,5 +1,5 @@
 // Several new tokens per head against a carried state in one pass over the
-// state (batched multi-token decode): the decode step of the pages (arXiv
+// state (batched multi-token decode): the decode step of the paper (arXiv
 // 2610.20637, abstract: constant per-token cost, the history held in the
 // additive states) generalised to a block of T <= 16 tokens, with the
 // block's own causal part computed pairwise.  For token i of the block,

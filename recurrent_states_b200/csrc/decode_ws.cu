@@ -1,6 +1,6 @@
 // Persistent, warp-specialised decode step for d_v = 64 and states of at most
 // 256 features (the decode workload: d_k 16, n 3, 153 x 65 floats per head).
-// Same arithmetic as the one-CTA-per-head kernel in decode.cu (the pages'
+// Same arithmetic as the one-CTA-per-head kernel in decode.cu (the paper's
 // constant-cost decode, arXiv 2610.20637, abstract):
 //   S += phi(k) [v | 1]^T,  y = (c (.) phi(q))^T S,  o = y[0:64] / y[64].
 //

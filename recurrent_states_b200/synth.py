@@ -2,8 +2,8 @@
 
 This module holds input recipes only, none of the method's arithmetic: draws
 from ``numpy.random.default_rng(seed)`` in the order q, k, v, an optional L2
-normalisation of q and k in float64 (the pages make unit-norm q and k a
-prerequisite; the library itself does not normalise), and the cast to the
+normalisation of q and k in float64 (the paper's abstract, arXiv 2610.20637,
+makes unit-norm q and k a prerequisite; the library itself does not normalise), and the cast to the
 dtype the kernels consume (round-to-nearest-even, done by torch on the CPU).
 
 The tensors returned are CPU tensors holding exactly the values a kernel sees;
@@ -58,8 +58,9 @@ def decode_tokens(B: int, H: int, d_k: int, d_v: int, step: int, seed: int = 0, 
     return q[:, :, 0], k[:, :, 0], v[:, :, 0]
 
 
-# Named workloads, sizes as the pages' experiments and the benchmark plan use
-# them (d = 16 from the pages' CPU study; the rest fixed here).
+# Named workloads, sizes as the paper's experiments and the benchmark plan use
+# them (d = 16 from the paper's CPU study, arXiv 2610.20637 abstract; the rest
+# fixed here).
 WORKLOADS = {
     "tiny": dict(B=1, H=1, N=256, d_k=16, d_v=16, n=3, tau=2.0, dtype="f32"),
     "main_prefill": dict(B=1, H=8, N=4096, d_k=16, d_v=64, n=3, tau=2.0, dtype="bf16"),

@@ -1,5 +1,5 @@
 """Pins for the float64 oracle: each test ties one part of it to something
-other than itself -- a number the pages print, a closed form, a library
+other than itself -- a number the abstract prints, a closed form, a library
 routine, brute force on tiny inputs, or an invariant the method states.
 
 Source of the method: "Expanding Attention: A Taylor-Series Route to

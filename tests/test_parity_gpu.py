@@ -161,7 +161,7 @@ def test_order_sweep_full_size(n):
 
 @pytest.mark.parametrize("n", [1, 3, 5])
 def test_order_sweep_unnormalised_odd_orders(n):
-    """q, k ~ N(0, 4) without normalisation (the case the pages say diverges
+    """q, k ~ N(0, 4) without normalisation (the case the abstract says diverges
     from softmax).  For odd n the kernel is positive, so the quotient is well
     conditioned; sampled rows against the pairwise form."""
     w = synth.WORKLOADS["order_sweep"]
