@@ -36,8 +36,14 @@
  *   stream) and returns after enqueueing.  Status TAYLOR_OK means the work
  *   was enqueued; launch failures are reported as TAYLOR_ERR_CUDA.  Calls
  *   keep no state between them and are safe from several host threads.
- * - Division is IEEE fp32 (no epsilon): for even n the denominator can reach
- *   zero for un-normalised inputs and the output is then inf/nan.
+ * - No epsilon in the quotient: IEEE fp32 division on the CUDA-core paths
+ *   and in decode, a multiplication by the correctly rounded reciprocal
+ *   (within 1.5 ulp of the quotient) in the tensor-core prefill.  For even n
+ *   the denominator can reach zero for un-normalised inputs and the output is
+ *   then inf/nan.
+ *
+ * The n = 3 state also serves a second read-out, the mean-centred Taylor
+ * expansion of softmax (taylor_attn_centred_decode, below).
  */
 #ifndef TAYLOR_ATTN_H
 #define TAYLOR_ATTN_H
