@@ -1,7 +1,8 @@
 """Plants plausible mistakes in the oracle (on the CPU, in this process only)
 and checks that the pins in test_oracle.py catch every one of them: a dropped
-term, a wrong weight, a wrong sign, an exclusive causal mask, a read-out before
-the update, a transposed state, a shuffled feature order."""
+term, a wrong or missing weight, a wrong sign, an exclusive or missing causal
+mask, a read-out before the update, a wrong normaliser column, a shuffled
+feature order or degree order."""
 import math
 
 import numpy as np
@@ -114,7 +115,34 @@ def _state_of_wrong_ones(k, v, n):
     return np.einsum("...jf,...jc->...fc", phik, v1)
 
 
+def _weight_one(t):
+    return 1.0
+
+
+def _index_degrees_reversed(d, n):
+    out = _orig_index(d, n)
+    blocks, i = [], 0
+    for m in range(n):
+        w = math.comb(d + m - 1, m)
+        blocks.append(out[i:i + w])
+        i += w
+    return [t for b in reversed(blocks) for t in b]
+
+
+def _direct_unmasked(q, k, v, n, tau, return_den=False, block=1024):
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    w = T.taylor_kernel(tau * np.einsum("...id,...jd->...ij", q, k), n)
+    den = w.sum(-1)
+    out = np.einsum("...ij,...jc->...ic", w, v) / den[..., None]
+    return (out, den) if return_den else out
+
+
 MUTATIONS = {
+    "multinomial weight left out": ("multinomial_weight", _weight_one),
+    "degrees stored highest first": ("feature_index", _index_degrees_reversed),
+    "no causal mask": ("attention_direct", _direct_unmasked),
     "dropped Taylor term": ("taylor_kernel", _kernel_drop_term),
     "wrong sign of the argument": ("taylor_kernel", _kernel_wrong_sign),
     "weight not square-rooted": ("multinomial_weight", _weight_unsquared),
