@@ -45,6 +45,19 @@ def _obj(src: str) -> str:
     return os.path.join(OBJ_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
 
 
+def _deps(src: str, headers) -> list:
+    """The files an object depends on: the dependency list nvcc wrote when it
+    last compiled the source (-MD), else every header of the library."""
+    dep = _obj(src)[:-2] + ".d"
+    if os.path.exists(dep):
+        with open(dep) as f:
+            text = f.read().replace("\\\n", " ")
+        files = [t for t in text.split(":", 1)[-1].split() if os.path.exists(t)]
+        if files:
+            return files + [os.path.abspath(__file__)]
+    return [src, *headers]
+
+
 def _stale(target: str, deps) -> bool:
     if not os.path.exists(target):
         return True
@@ -61,10 +74,11 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         return LIB
     os.makedirs(OBJ_DIR, exist_ok=True)
     headers = _headers()
-    todo = [s for s in sources() if force or extra or _stale(_obj(s), [s, *headers])]
+    todo = [s for s in sources() if force or extra or _stale(_obj(s), _deps(s, headers))]
 
     def compile_one(src):
-        cmd = [NVCC, *FLAGS, *extra, "-c", "-o", _obj(src), src]
+        dep = _obj(src)[:-2] + ".d"
+        cmd = [NVCC, *FLAGS, *extra, "-MD", "-MF", dep, "-c", "-o", _obj(src), src]
         if verbose:
             print(" ".join(cmd), flush=True)
         return subprocess.run(cmd, capture_output=True, text=True)

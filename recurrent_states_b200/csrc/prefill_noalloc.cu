@@ -12,16 +12,21 @@
 // The array exists once per GPU that loads this library and stays there until
 // the process exits.  Host code cannot use the array's name as a device
 // address (it names a host-side stand-in), so the device address is looked up
-// with cudaGetSymbolAddress once per device, on the first call made while
-// that device is current; make that first call before any stream capture.
-// Every call on a device shares the one array and leaves its contents behind;
-// nothing in it has to start at zero, because every element the kernels read
-// is written earlier in the same call.  Calls whose work overlaps on the GPU
-// (two streams, or two host threads, on one device) race on the array and
-// must be serialised by the caller.
+// with cudaGetSymbolAddress on the first call made while a device is current.
+// CUDA loads a library's device code lazily, so that first lookup is also what
+// loads the code holding the array and reserves its 16 MiB on the device: make
+// the first call during set-up, before the caller reserves the rest of the
+// device's memory and before any stream capture.  A lookup that fails (for
+// example for want of those 16 MiB) is not remembered; the next call tries
+// again.  Every call on a device shares the one array and leaves its contents
+// behind; nothing in it has to start at zero, because every element the
+// kernels read is written earlier in the same call.  Calls whose work overlaps
+// on the GPU (two streams, or two host threads, on one device) race on the
+// array and must be serialised by the caller.
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/taylor_attn.h"
@@ -35,23 +40,30 @@ constexpr int64_t kScratchFloats = int64_t(4) << 20;
 static __device__ __align__(256) float g_prefill_scratch[kScratchFloats];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-float* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_lookup_mutex;
+std::atomic<float*> g_scratch_ptr[kMaxDevices];
 
-// Device address of the array on the current device (looked up once).
+// Device address of the array on the current device.  Only a successful
+// lookup is kept; after a failure the next call looks it up again.
 cudaError_t scratch_on_current_device(float** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_once[dev], [dev]() {
-        void* p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_prefill_scratch);
-        g_scratch_ptr[dev] = static_cast<float*>(p);
-    });
-    *out = g_scratch_ptr[dev];
-    return g_scratch_err[dev];
+    float* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        std::lock_guard<std::mutex> lock(g_lookup_mutex);
+        p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+        if (p == nullptr) {
+            void* addr = nullptr;
+            e = cudaGetSymbolAddress(&addr, g_prefill_scratch);
+            if (e != cudaSuccess) return e;
+            p = static_cast<float*>(addr);
+            g_scratch_ptr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return cudaSuccess;
 }
 
 bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -88,9 +100,10 @@ extern "C" int taylor_attn_prefill_f32_noalloc(const float* q, const float* k, c
     const bool need_states = plan.NG > 1 || state_out != nullptr;
     if (need_states && BH * plan.NG * stride > kScratchFloats) return TAYLOR_ERR_SCRATCH_LIMIT;
     float* scratch = nullptr;
-    if (scratch_on_current_device(&scratch) != cudaSuccess || scratch == nullptr) {
+    const cudaError_t le = scratch_on_current_device(&scratch);
+    if (le != cudaSuccess || scratch == nullptr) {
         cudaGetLastError();
-        return TAYLOR_ERR_CUDA;
+        return le == cudaErrorMemoryAllocation ? TAYLOR_ERR_OUT_OF_MEMORY : TAYLOR_ERR_CUDA;
     }
     const cudaError_t e = ta::launch_prefill_cc(q, k, v, out, nullptr, state_out, scratch, plan, (int)BH, N,
                                                 d_k, d_v, n, tau, F, stride, stream);

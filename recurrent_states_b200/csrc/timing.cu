@@ -45,16 +45,24 @@ cudaEvent_t take_event() {
 
 bool enabled() { return g_on; }
 
+// Every begin() pushes one record, so that end() always closes the record of
+// its own launch; a launch whose events could not be had keeps a record with
+// null events, which end() and taylor_attn_timing_read() skip.
 void begin(cudaStream_t s, const char* name) {
     if (!g_on) return;
     Rec r{name, take_event(), take_event()};
-    if (!r.start || !r.stop) return;
-    cudaEventRecord(r.start, s);
+    if (!r.start || !r.stop) {
+        if (r.start) g_pool.push_back(r.start);
+        if (r.stop) g_pool.push_back(r.stop);
+        r.start = r.stop = nullptr;
+    } else {
+        cudaEventRecord(r.start, s);
+    }
     g_recs.push_back(r);
 }
 
 void end(cudaStream_t s) {
-    if (!g_on || g_recs.empty()) return;
+    if (!g_on || g_recs.empty() || !g_recs.back().stop) return;
     cudaEventRecord(g_recs.back().stop, s);
 }
 
@@ -86,6 +94,10 @@ int taylor_attn_timing_read(int max_kernels, char* names, int* launches, float* 
     std::vector<double> ms;
     int rc = TAYLOR_OK;
     for (auto& r : g_recs) {
+        if (!r.start || !r.stop) {  // no events could be had for this launch
+            rc = TAYLOR_ERR_CUDA;
+            continue;
+        }
         float t = 0.f;
         if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) {
             cudaGetLastError();

@@ -1,9 +1,13 @@
 // Stream-ordered workspace for the prefill scan.  Each device gets one
-// library-owned memory pool whose release threshold keeps up to
-// kCachedBytes of freed workspace mapped, so back-to-back calls reuse it
-// instead of unmapping and mapping memory on every call (which stalls the
-// stream for hundreds of microseconds).  taylor_attn_release_workspace()
-// returns the cached memory to the driver.
+// library-owned memory pool whose release threshold keeps freed workspace
+// mapped, so back-to-back calls reuse it instead of unmapping and mapping
+// memory on every call (which stalls the stream for hundreds of microseconds,
+// and for milliseconds at a gigabyte).  The threshold is the larger of
+// kCachedBytes and the largest single workspace requested so far on that
+// device, so a call whose workspace alone exceeds kCachedBytes still finds it
+// mapped on the next call.  taylor_attn_release_workspace() returns the cached
+// memory to the driver.
+#include <atomic>
 #include <mutex>
 
 #include "../../include/taylor_attn.h"
@@ -17,6 +21,8 @@ constexpr uint64_t kCachedBytes = uint64_t(1) << 30;  // 1 GiB per device
 std::once_flag g_once[kMaxDevices];
 cudaMemPool_t g_pool[kMaxDevices];
 cudaError_t g_err[kMaxDevices];
+std::atomic<uint64_t> g_threshold[kMaxDevices];
+std::mutex g_threshold_mutex;
 
 cudaError_t pool_for(int dev, cudaMemPool_t* out) {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
@@ -31,6 +37,7 @@ cudaError_t pool_for(int dev, cudaMemPool_t* out) {
         if (g_err[dev] == cudaSuccess) {
             uint64_t thr = kCachedBytes;
             g_err[dev] = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &thr);
+            g_threshold[dev].store(thr);
         }
         g_pool[dev] = p;
     });
@@ -48,6 +55,14 @@ cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     cudaMemPool_t pool = nullptr;
     if ((e = pool_for(dev, &pool)) != cudaSuccess) return e;
+    if (bytes > g_threshold[dev].load(std::memory_order_relaxed)) {
+        std::lock_guard<std::mutex> lock(g_threshold_mutex);
+        uint64_t thr = bytes;
+        if (thr > g_threshold[dev].load()) {
+            if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr)) != cudaSuccess) return e;
+            g_threshold[dev].store(thr);
+        }
+    }
     return cudaMallocFromPoolAsync(ptr, bytes, pool, stream);
 }
 
