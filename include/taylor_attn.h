@@ -106,8 +106,9 @@ TAYLOR_API int taylor_attn_feature_map(const float* x, float* phi, int64_t T, in
  * Writes out[B][H][N][d_v] and, when state_out != NULL, the state after all
  * N tokens.  N == 0 writes a zero state.  Takes stream-ordered workspace on
  * `stream` (one fp32 state per 64-128 tokens per head) from a memory pool the
- * library creates per device; up to 1 GiB of freed workspace stays cached in
- * that pool for later calls (taylor_attn_release_workspace returns it).
+ * library creates per device; freed workspace stays cached in that pool for
+ * later calls, up to the larger of 1 GiB and the largest workspace one call
+ * has needed (taylor_attn_release_workspace returns it).
  * TAYLOR_ERR_OUT_OF_MEMORY if the workspace cannot be had; accumulation is
  * fp32. */
 TAYLOR_API int taylor_attn_prefill(const void* q, const void* k, const void* v, float* out,
@@ -186,6 +187,30 @@ TAYLOR_API int taylor_attn_centred_decode_f32(const float* q, const float* k, co
                                               float* state_inout, float* out, int B, int H, int d_k, int d_v,
                                               int order, float tau, cudaStream_t stream);
 
+/* Causal prefill with the mean-centred Taylor expansion of softmax (the same
+ * method and readings as taylor_attn_centred_decode: Su Jianlin, "Taylor
+ * expansions of logsumexp and softmax", kexue.fm translation 11814, sections
+ * "Calculating the Gradient" and "Linear Attention").  Row i weights v_j,
+ * j <= i, by (1 + y_j + (y_j^2 - mean(y^2))/2) / (i + 1), y_j = tau
+ * q_i.(k_j - kbar_i), kbar_i the mean of k_0..k_i; order 1 drops the square
+ * term.  q, k [B][H][N][d_k], v [B][H][N][d_v] bf16 (the _f32 variant:
+ * fp32); out [B][H][N][d_v] fp32.  state_out (may be NULL) receives the n = 3
+ * Taylor state of the N tokens ([B][H][taylor_attn_state_stride(d_k, d_v,
+ * 3)]), from which taylor_attn_centred_decode (or taylor_attn_decode with
+ * n = 3) continues.  The three per-degree read-outs sum_j (q_i.k_j)^m [v_j | 1]
+ * (m = 0, 1, 2) are accumulated in fp32 on CUDA cores, pairwise inside a token
+ * group and through the group's exclusive n = 3 state across groups, and
+ * combined per column.  order is 1 or 2 (else TAYLOR_ERR_UNSUPPORTED); sizes,
+ * alignment and workspace as taylor_attn_prefill. */
+TAYLOR_API int taylor_attn_centred_prefill(const void* q, const void* k, const void* v, float* out,
+                                           float* state_out, int B, int H, int N, int d_k, int d_v, int order,
+                                           float tau, cudaStream_t stream);
+
+/* taylor_attn_centred_prefill with fp32 q, k, v. */
+TAYLOR_API int taylor_attn_centred_prefill_f32(const float* q, const float* k, const float* v, float* out,
+                                               float* state_out, int B, int H, int N, int d_k, int d_v,
+                                               int order, float tau, cudaStream_t stream);
+
 /* out = a + b over B*H states (abstract: states are additive across chunks,
  * so the state of a concatenation is the sum of the parts' states).  out may
  * alias a or b.  No workspace. */
@@ -202,10 +227,15 @@ TAYLOR_API int taylor_attn_state_merge(const float* a, const float* b, float* ou
  * cudaMalloc/cudaFree or other allocating call.  Work needing more scratch
  * than that (B*H * groups * stride floats; the B1 H8 N4096 d_k16 d_v64 n3
  * shape needs about 2.5 million) returns TAYLOR_ERR_SCRATCH_LIMIT before any launch.
- * The first call on a device looks up the array's device address (make it
- * before any stream capture).  All calls on a device share the array: calls
- * that overlap on the GPU race and must be serialised by the caller.  Same
- * arguments, layouts and results as taylor_attn_prefill_f32. */
+ * The first call on a device looks up the array's device address; CUDA loads
+ * device code lazily, so that first call is also the one that brings the
+ * array's 16 MiB onto the device, and it can fail with
+ * TAYLOR_ERR_OUT_OF_MEMORY when the device is already full.  Make it during
+ * set-up, before reserving the rest of the device's memory and before any
+ * stream capture; a failed first call is retried by the next one.  All calls
+ * on a device share the array: calls that overlap on the GPU race and must be
+ * serialised by the caller.  Same arguments, layouts and results as
+ * taylor_attn_prefill_f32. */
 TAYLOR_API int taylor_attn_prefill_f32_noalloc(const float* q, const float* k, const float* v,
                                                float* out, float* state_out, int B, int H, int N,
                                                int d_k, int d_v, int n, float tau,
