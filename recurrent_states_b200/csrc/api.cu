@@ -103,6 +103,44 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, const float* state_in
 }
 
 template <typename Tin>
+int centred_prefill_impl(const Tin* q, const Tin* k, const Tin* v, float* out, float* state_out, int B, int H,
+                         int N, int d_k, int d_v, int order, float tau, cudaStream_t stream) {
+    if (B < 0 || H < 0 || N < 0) return TAYLOR_ERR_INVALID_ARG;
+    int rc = check_dims(d_k, d_v, 3);
+    if (rc != TAYLOR_OK) return rc;
+    if (order != 1 && order != 2) return TAYLOR_ERR_UNSUPPORTED;
+    if (!isfinite(tau)) return TAYLOR_ERR_INVALID_ARG;
+    const int64_t BH = (int64_t)B * H;
+    if (BH > 65535) return TAYLOR_ERR_UNSUPPORTED;
+    if (BH * (int64_t)N >= ((int64_t)1 << 31)) return TAYLOR_ERR_UNSUPPORTED;
+    if (BH == 0) return TAYLOR_OK;
+    const int64_t F = ta::num_features(d_k, 3);
+    const int64_t stride = stride_of(d_k, d_v, 3);
+    if (state_out && !aligned16(state_out)) return TAYLOR_ERR_MISALIGNED;
+    if (N == 0) {
+        if (!state_out) return TAYLOR_OK;
+        return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)BH * stride * sizeof(float), stream));
+    }
+    if (!q || !k || !v || !out) return TAYLOR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TAYLOR_ERR_MISALIGNED;
+    const ta::CcPlan plan = ta::plan_prefill_cc((int)BH, N, d_k, d_v, 3, F, stride);
+    float* ws = nullptr;
+    if (plan.NG > 1 || state_out != nullptr) {
+        if (ta::workspace_alloc(reinterpret_cast<void**>(&ws), plan.ws_bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return TAYLOR_ERR_OUT_OF_MEMORY;
+        }
+    }
+    cudaError_t e = ta::launch_centred_prefill_cc(q, k, v, out, nullptr, state_out, ws, plan, (int)BH, N, d_k, d_v,
+                                                  order, tau, F, stride, stream);
+    if (ws) {
+        const cudaError_t e2 = ta::workspace_free(ws, stream);
+        if (e == cudaSuccess) e = e2;
+    }
+    return cuda_status(e);
+}
+
+template <typename Tin>
 int decode_impl(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int B, int H,
                 int d_k, int d_v, int n, float tau, cudaStream_t stream) {
     if (B < 0 || H < 0) return TAYLOR_ERR_INVALID_ARG;
@@ -249,6 +287,19 @@ int taylor_attn_centred_decode_f32(const float* q, const float* k, const float* 
                                    float* out, int B, int H, int d_k, int d_v, int order, float tau,
                                    cudaStream_t stream) {
     return centred_decode_impl(q, k, v, state_inout, out, B, H, d_k, d_v, order, tau, stream);
+}
+
+int taylor_attn_centred_prefill(const void* q, const void* k, const void* v, float* out, float* state_out, int B,
+                                int H, int N, int d_k, int d_v, int order, float tau, cudaStream_t stream) {
+    using bf = __nv_bfloat16;
+    return centred_prefill_impl(static_cast<const bf*>(q), static_cast<const bf*>(k), static_cast<const bf*>(v),
+                                out, state_out, B, H, N, d_k, d_v, order, tau, stream);
+}
+
+int taylor_attn_centred_prefill_f32(const float* q, const float* k, const float* v, float* out, float* state_out,
+                                    int B, int H, int N, int d_k, int d_v, int order, float tau,
+                                    cudaStream_t stream) {
+    return centred_prefill_impl(q, k, v, out, state_out, B, H, N, d_k, d_v, order, tau, stream);
 }
 
 int taylor_attn_state_merge(const float* a, const float* b, float* out, int B, int H, int d_k,

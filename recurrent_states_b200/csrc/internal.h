@@ -99,6 +99,14 @@ cudaError_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Prefill of the mean-centred softmax expansion (order 1 or 2) on CUDA cores,
+// over the n = 3 group states of the same plan (plan_prefill_cc with n = 3).
+template <typename Tin>
+cudaError_t launch_centred_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
+                                      const float* state_in, float* state_out, float* workspace,
+                                      const CcPlan& plan, int BH, int N, int d, int dv, int order, float tau,
+                                      int64_t F, int64_t stride, cudaStream_t stream);
+
 template <typename Tin>
 cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
                               const float* state_in, float* state_out, float* workspace,

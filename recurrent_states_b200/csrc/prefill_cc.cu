@@ -328,6 +328,172 @@ chunk_out_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     }
 }
 
+// ---------------------------------------------------------------- C'
+// Output kernel of the mean-centred softmax expansion (Su Jianlin, "Taylor
+// expansions of logsumexp and softmax", kexue.fm translation 11814, sections
+// "Calculating the Gradient" and "Linear Attention"), over the same group
+// states as C (those of the n = 3 Taylor kernel: their degree-0, 1 and 2 rows
+// hold every prefix sum the expansion needs).  For query i the three
+// per-degree read-outs R_m = sum_{j <= i} (q_i.k_j)^m [v_j | 1] (no tau, no
+// 1/m!) are accumulated apart: pairwise inside the group, through
+// phi_m(q_i)^T S_<g,m across groups.  Then, per column,
+//   n = R_0[z], V = R_0[v], qkbar = R_1[z] / n,
+//   sum a v   = tau (R_1[v] - qkbar V),
+//   sum a^2 v = tau^2 (R_2[v] - 2 qkbar R_1[v] + qkbar^2 V),
+//   sum a^2   = tau^2 (R_2[z] - n qkbar^2),
+//   o = V/n + (sum a v)/n  [+ (sum a^2 v - (sum a^2) V/n) / (2n) at order 2].
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads)
+centred_chunk_out_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                         const float* __restrict__ W, float* __restrict__ out, int N, int d, int dv, int order,
+                         float tau, int G, int NG, int F, int64_t stride, int carried) {
+    extern __shared__ float4 sm4[];
+    float* sm = reinterpret_cast<float*>(sm4);
+    const OutSmem L = out_smem_layout(d);
+    float* qs = sm + L.qs;
+    float* ks = sm + L.ks;
+    float* vs = sm + L.vs;
+    float* P = sm + L.P;
+    float* phq = sm + L.phq;
+    float* Ss = sm + L.Ss;
+    float* zs = sm + L.zs;
+    FeatDesc* ds = reinterpret_cast<FeatDesc*>(sm + L.ds);
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int i = tid >> 2, qq = tid & 3;
+    const int bh = blockIdx.y;
+    const int64_t q0 = (int64_t)blockIdx.x * kC;
+    const int nq = (int)min64(kC, N - q0);
+    const int g = (int)(q0 / G);
+    const int64_t gs = (int64_t)g * G;
+    const int dq = L.dq;
+
+    const Tin* qb = q + (int64_t)bh * N * d;
+    const Tin* kb = k + (int64_t)bh * N * d;
+    const Tin* vb = v + (int64_t)bh * N * dv;
+    const PackedFeat* tab = feat_table(d, 3);
+    for (int e = tid; e < kC * d; e += kThreads) {
+        const int r = e / d, s = e % d;
+        qs[r * dq + s] = r < nq ? ldf(qb + (q0 + r) * d + s) : 0.f;
+    }
+
+    for (int cb = 0; cb < dv; cb += 64) {
+        const int cw = min(64, dv - cb);
+        float a0[16], a1[16], a2[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) a0[c] = a1[c] = a2[c] = 0.f;
+        float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+
+        // pairwise part over the keys of this group up to the diagonal: the
+        // raw score s = q.k_j, its square, and 1
+        for (int64_t k0 = gs; k0 <= q0; k0 += kC) {
+            const int nk = (int)min64(kC, N - k0);
+            __syncthreads();
+            for (int e = tid; e < nk * d; e += kThreads) {
+                const int r = e / d, s = e % d;
+                ks[r * dq + s] = ldf(kb + (k0 + r) * d + s);
+            }
+            for (int e = tid; e < nk * cw; e += kThreads) {
+                const int r = e / cw, c = e % cw;
+                vs[r * 64 + c] = ldf(vb + (k0 + r) * dv + cb + c);
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int jj = 0; jj < 16; ++jj) {
+                const int j = qq * 16 + jj;
+                float dot = 0.f;
+                if (i < nq && j < nk)
+                    for (int s = 0; s < d; ++s) dot = fmaf(qs[i * dq + s], ks[j * dq + s], dot);
+                P[i * (kC + 1) + j] = dot;
+            }
+            __syncthreads();
+            // keys j <= i of this tile (all of them below the diagonal tile)
+            const int jn = i < nq ? (int)min64(nk, q0 + i - k0 + 1) : 0;
+            for (int j = 0; j < jn; ++j) {
+                const float s1 = P[i * (kC + 1) + j];
+                const float s2 = s1 * s1;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const float x = vs[j * 64 + qq * 16 + c];
+                    a0[c] += x;
+                    a1[c] = fmaf(s1, x, a1[c]);
+                    a2[c] = fmaf(s2, x, a2[c]);
+                }
+                if (qq == 0) {
+                    z0 += 1.f;
+                    z1 += s1;
+                    z2 += s2;
+                }
+            }
+        }
+
+        // across groups, through the exclusive prefix state S_<g: each
+        // feature's read-out goes to the accumulator of its degree
+        if (g > 0 || carried) {
+            const float* Sg = W + ((int64_t)bh * NG + g) * stride;
+            for (int f0 = 0; f0 < F; f0 += kFTC) {
+                const int nf = min(kFTC, F - f0);
+                __syncthreads();
+                if (tid < nf) ds[tid] = get_desc(tab, d, 3, f0 + tid, 1.f, nullptr, false);
+                for (int e = tid; e < nf * cw; e += kThreads) {
+                    const int r = e / cw, c = e % cw;
+                    Ss[r * 64 + c] = Sg[(int64_t)(f0 + r) * dv + cb + c];
+                }
+                if (tid < nf) zs[tid] = Sg[(int64_t)F * dv + f0 + tid];
+                __syncthreads();
+                for (int e = tid; e < kC * kFTC; e += kThreads) {
+                    const int r = e / kFTC, f = e % kFTC;
+                    phq[r * (kFTC + 1) + f] = (r < nq && f < nf) ? eval_desc(ds[f], qs + r * dq) : 0.f;
+                }
+                __syncthreads();
+                for (int f = 0; f < nf; ++f) {
+                    const float p = phq[i * (kFTC + 1) + f];
+                    const int m = ds[f].m;  // the same for every thread
+                    const float* sr = Ss + f * 64 + qq * 16;
+                    if (m == 0) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) a0[c] = fmaf(p, sr[c], a0[c]);
+                    } else if (m == 1) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) a1[c] = fmaf(p, sr[c], a1[c]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) a2[c] = fmaf(p, sr[c], a2[c]);
+                    }
+                    if (qq == 0) {
+                        const float pz = p * zs[f];
+                        if (m == 0) z0 += pz;
+                        else if (m == 1) z1 += pz;
+                        else z2 += pz;
+                    }
+                }
+            }
+        }
+
+        z0 = __shfl_sync(0xffffffffu, z0, lane & ~3);
+        z1 = __shfl_sync(0xffffffffu, z1, lane & ~3);
+        z2 = __shfl_sync(0xffffffffu, z2, lane & ~3);
+        if (i < nq) {
+            const float n = z0, qkbar = z1 / n, t2 = tau * tau;
+            const float sum_a2 = t2 * (z2 - n * qkbar * qkbar);
+            float* o = out + ((int64_t)bh * N + q0 + i) * dv + cb + qq * 16;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                if (qq * 16 + c < cw) {
+                    const float V = a0[c];
+                    float r = V / n + tau * (a1[c] - qkbar * V) / n;
+                    if (order >= 2) {
+                        const float sum_a2v = t2 * (a2[c] - 2.0f * qkbar * a1[c] + qkbar * qkbar * V);
+                        r += (sum_a2v - sum_a2 * V / n) / (2.0f * n);
+                    }
+                    o[c] = r;
+                }
+            }
+        }
+    }
+}
+
 template <typename T>
 cudaError_t set_smem(T* fn, size_t bytes) {
     return cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
@@ -357,16 +523,12 @@ CcPlan plan_prefill_cc(int BH, int N, int d, int dv, int n, int64_t F, int64_t s
     return p;
 }
 
+// A and B: per-group states of (d, n) and their exclusive scan, in W.
 template <typename Tin>
-cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
-                              const float* state_in, float* state_out, float* W, const CcPlan& plan,
-                              int BH, int N, int d, int dv, int n, float tau, int64_t F, int64_t stride,
-                              cudaStream_t stream) {
-    if (BH == 0 || N == 0) return cudaSuccess;
+cudaError_t launch_group_states(const Tin* k, const Tin* v, const float* state_in, float* state_out, float* W,
+                                const CcPlan& plan, int BH, int N, int d, int dv, int n, int64_t F, int64_t stride,
+                                cudaStream_t stream) {
     cudaError_t e;
-    // a single group with no state in or out needs neither A nor B
-    const bool need_states = plan.NG > 1 || state_out != nullptr || state_in != nullptr;
-    if (need_states) {
     // A
     const int dv4 = dv / 4;
     const int rsets = kThreads / dv4;
@@ -393,7 +555,21 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
     const dim3 gB((unsigned)((stride / 4 + kScanCols - 1) / kScanCols), BH);
     TA_TIMED(stream, "cc_scan_kernel",
              scan_kernel<<<gB, kScanThreads, 0, stream>>>(W, state_in, state_out, plan.NG, stride, F * (dv + 1)));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
+                              const float* state_in, float* state_out, float* W, const CcPlan& plan,
+                              int BH, int N, int d, int dv, int n, float tau, int64_t F, int64_t stride,
+                              cudaStream_t stream) {
+    if (BH == 0 || N == 0) return cudaSuccess;
+    cudaError_t e;
+    // a single group with no state in or out needs neither A nor B
+    const bool need_states = plan.NG > 1 || state_out != nullptr || state_in != nullptr;
+    if (need_states) {
+        e = launch_group_states(k, v, state_in, state_out, W, plan, BH, N, d, dv, n, F, stride, stream);
+        if (e != cudaSuccess) return e;
     }
     // C
     const OutSmem L = out_smem_layout(d);
@@ -402,6 +578,28 @@ cudaError_t launch_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* o
     const dim3 gC((unsigned)((N + kC - 1) / kC), BH);
     TA_TIMED(stream, "cc_chunk_out_kernel",
              fc<<<gC, kThreads, L.total, stream>>>(q, k, v, W, out, N, d, dv, n, tau, plan.G, plan.NG,
+                                                   (int)F, stride, state_in != nullptr ? 1 : 0));
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_centred_prefill_cc(const Tin* q, const Tin* k, const Tin* v, float* out,
+                                      const float* state_in, float* state_out, float* W, const CcPlan& plan,
+                                      int BH, int N, int d, int dv, int order, float tau, int64_t F,
+                                      int64_t stride, cudaStream_t stream) {
+    if (BH == 0 || N == 0) return cudaSuccess;
+    cudaError_t e;
+    const bool need_states = plan.NG > 1 || state_out != nullptr || state_in != nullptr;
+    if (need_states) {
+        e = launch_group_states(k, v, state_in, state_out, W, plan, BH, N, d, dv, 3, F, stride, stream);
+        if (e != cudaSuccess) return e;
+    }
+    const OutSmem L = out_smem_layout(d);
+    auto fc = centred_chunk_out_kernel<Tin>;
+    if ((e = set_smem(fc, L.total)) != cudaSuccess) return e;
+    const dim3 gC((unsigned)((N + kC - 1) / kC), BH);
+    TA_TIMED(stream, "cc_centred_chunk_out_kernel",
+             fc<<<gC, kThreads, L.total, stream>>>(q, k, v, W, out, N, d, dv, order, tau, plan.G, plan.NG,
                                                    (int)F, stride, state_in != nullptr ? 1 : 0));
     return cudaGetLastError();
 }
@@ -423,5 +621,12 @@ template cudaError_t launch_prefill_cc<__nv_bfloat16>(const __nv_bfloat16*, cons
                                                       const __nv_bfloat16*, float*, const float*, float*,
                                                       float*, const CcPlan&, int, int, int, int, int, float,
                                                       int64_t, int64_t, cudaStream_t);
+template cudaError_t launch_centred_prefill_cc<float>(const float*, const float*, const float*, float*,
+                                                      const float*, float*, float*, const CcPlan&, int, int, int,
+                                                      int, int, float, int64_t, int64_t, cudaStream_t);
+template cudaError_t launch_centred_prefill_cc<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                                              const __nv_bfloat16*, float*, const float*, float*,
+                                                              float*, const CcPlan&, int, int, int, int, int,
+                                                              float, int64_t, int64_t, cudaStream_t);
 
 }  // namespace ta

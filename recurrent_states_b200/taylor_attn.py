@@ -46,6 +46,8 @@ SIGNATURES = {
     "taylor_attn_decode_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_centred_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_centred_decode_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "taylor_attn_centred_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "taylor_attn_centred_prefill_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_state_merge": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "taylor_attn_prefill_f32_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "taylor_attn_prefill_noalloc_scratch_floats": (_I64, []),
@@ -287,6 +289,42 @@ def taylor_attn_centred_decode(q, k, v, state, order: int, tau: float, out=None,
 
 def taylor_attn_centred_decode_f32(q, k, v, state, order: int, tau: float, out=None, stream=None):
     return _decode("taylor_attn_centred_decode_f32", q, k, v, state, 3, tau, out, stream, order=order)
+
+
+def _centred_prefill(name, q, k, v, order, tau, out, state_out, stream):
+    dtype = torch.bfloat16 if name == "taylor_attn_centred_prefill" else torch.float32
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, H, N, d_k = q.shape
+    d_v = v.shape[-1]
+    _need(q, "q", dtype)
+    _need(k, "k", dtype, q.device, (B, H, N, d_k))
+    _need(v, "v", dtype, q.device, (B, H, N, d_v))
+    if out is None:
+        out = torch.empty((B, H, N, d_v), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, q.device, (B, H, N, d_v))
+    stride = taylor_attn_state_stride(d_k, d_v, 3)
+    if state_out is True:
+        if stride < 0:
+            raise TaylorAttnError(TAYLOR_ERR_UNSUPPORTED, name)
+        state_out = torch.empty((B, H, stride), dtype=torch.float32, device=q.device)
+    if state_out is not None:
+        _need(state_out, "state_out", torch.float32, q.device, (B, H, stride))
+    rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state_out), B, H, N, d_k,
+                              d_v, int(order), float(tau), _stream(stream))
+    _check(rc, name)
+    return out, state_out
+
+
+def taylor_attn_centred_prefill(q, k, v, order: int, tau: float, out=None, state_out=None, stream=None):
+    """Mean-centred softmax expansion (order 1 or 2), causal prefill: bf16 q,
+    k [B,H,N,d_k], v [B,H,N,d_v] -> (out fp32, n = 3 Taylor state or None)."""
+    return _centred_prefill("taylor_attn_centred_prefill", q, k, v, order, tau, out, state_out, stream)
+
+
+def taylor_attn_centred_prefill_f32(q, k, v, order: int, tau: float, out=None, state_out=None, stream=None):
+    """taylor_attn_centred_prefill with fp32 q, k, v."""
+    return _centred_prefill("taylor_attn_centred_prefill_f32", q, k, v, order, tau, out, state_out, stream)
 
 
 def taylor_attn_state_merge(a, b, d_k: int, d_v: int, n: int, out=None, stream=None):
