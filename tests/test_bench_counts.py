@@ -21,7 +21,8 @@ def _F(d, n):
 
 
 def test_bench_workloads_are_the_named_workloads():
-    for key, name in (("MAIN", "main_prefill"), ("DECODE", "decode"), ("LARGE", "large_head")):
+    for key, name in (("MAIN", "main_prefill"), ("DECODE", "decode"), ("LARGE", "large_head"),
+                      ("SWEEP", "order_sweep")):
         w, ref = getattr(bench, key), synth.WORKLOADS[name]
         for f in w:
             assert w[f] == ref[f], (key, f)

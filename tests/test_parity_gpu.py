@@ -159,19 +159,63 @@ def test_order_sweep_full_size(n):
     assert state_block_errors(st[0, hs], ref_st, 16, 64, n) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("n", [1, 3, 5])
-def test_order_sweep_unnormalised_odd_orders(n):
+def _abs_kernel_mass(q, k, n, tau, heads, rows):
+    """sum_{j<=i} |K(tau q_i.k_j)| per sampled (head, row), float64: the scale
+    of the terms whose sum is the denominator.  Used only to decide which rows
+    have a cancelling (ill-conditioned) denominator, never as an expected
+    value."""
+    out = np.empty(len(rows))
+    for r, (h, i) in enumerate(zip(heads, rows)):
+        x = tau * (k[h, :i + 1] @ q[h, i])
+        w = np.zeros_like(x)
+        term = np.ones_like(x)
+        for m in range(n):
+            w += term
+            term = term * x / (m + 1)
+        out[r] = np.abs(w).sum()
+    return out
+
+
+# Rows whose denominator cancels: kappa = sum|K| / |sum K| multiplies the
+# relative rounding of the kernel's sums (hi/lo bf16 operands, fp32
+# accumulation: about 1e-5) into the quotient; from this kappa on that product
+# alone approaches the 2e-3 bound.
+KAPPA_MAX = 100.0
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5])
+def test_order_sweep_unnormalised(n):
     """q, k ~ N(0, 4) without normalisation (the case the abstract says diverges
-    from softmax).  For odd n the kernel is positive, so the quotient is well
-    conditioned; sampled rows against the pairwise form."""
+    from softmax), sampled rows against the pairwise form.  For odd n the
+    kernel is positive (kappa = 1) and every row is held to 2e-3.  For even n
+    (the podcast page: an even highest order lets the kernel go negative) the
+    denominator can cancel: rows with |den| < 1e-6 (i + 1) are dropped and
+    counted, rows with kappa = sum|K| / |sum K| > KAPPA_MAX are counted and
+    held to the conditioning-scaled bound 2e-3 kappa / KAPPA_MAX, and every
+    other row is held to 2e-3."""
     w = synth.WORKLOADS["order_sweep"]
-    q, k, v = synth.qkv(1, 8, w["N"], 16, 64, seed=1, dtype="bf16", normalise=False, qk_var=4.0)
-    out, _ = _prefill("bf16", q, k, v, n, w["tau"], state=False)
-    rows = sample_rows(w["N"], 48, seed=10 + n)
-    heads = np.repeat(np.arange(8), len(rows))
-    rr = np.tile(rows, 8)
-    ref, _ = C.direct_rows(f64(q)[0], f64(k)[0], f64(v)[0], n, w["tau"], heads, rr)
-    assert row_scaled_max_err(f64(out)[0][heads, rr], ref) <= TOL["bf16"]
+    H, N, tau = 8, w["N"], w["tau"]
+    q, k, v = synth.qkv(1, H, N, 16, 64, seed=1, dtype="bf16", normalise=False, qk_var=4.0)
+    out, _ = _prefill("bf16", q, k, v, n, tau, state=False)
+    rows = sample_rows(N, 48, seed=10 + n)
+    heads = np.repeat(np.arange(H), len(rows))
+    rr = np.tile(rows, H)
+    qd, kd, vd = f64(q)[0], f64(k)[0], f64(v)[0]
+    ref, den = C.direct_rows(qd, kd, vd, n, tau, heads, rr)
+    got = f64(out)[0][heads, rr]
+    tiny = np.abs(den) < 1e-6 * (rr + 1)
+    kappa = _abs_kernel_mass(qd, kd, n, tau, heads, rr) / np.abs(den)
+    ill = ~tiny & (kappa > KAPPA_MAX)
+    keep = ~tiny & ~ill
+    err = np.abs(got - ref).max(-1) / np.abs(ref).max(-1)
+    print(f"n={n}: {len(rr)} rows, {int(tiny.sum())} with |den| < 1e-6 (i+1), "
+          f"{int(ill.sum())} with kappa > {KAPPA_MAX:g} (max kappa {kappa[~tiny].max():.3g}), "
+          f"max err {err[keep].max():.3g} over the other rows")
+    if n % 2 == 1:
+        assert not tiny.any() and not ill.any()
+    assert keep.sum() >= 0.9 * len(rr)
+    assert err[keep].max() <= TOL["bf16"]
+    assert (err[ill] <= TOL["bf16"] * kappa[ill] / KAPPA_MAX).all()
 
 
 def test_large_head_full_size():
