@@ -361,6 +361,23 @@ def run_ours(args, world, rank, local):
     cen_kernel_us = ck_ms * 1e3
     errs.check("centred_decode")
 
+    # ---- the mean-centred expansion's prefill (order 2) on the main workload's inputs
+    cout = torch.empty_like(out)
+    cst = torch.empty_like(st)
+
+    def cstep(i=0):
+        TA.taylor_attn_centred_prefill(q, k, v, 2, tau, out=cout, state_out=cst)
+
+    for _ in range(3):
+        flush_l2()
+        cstep()
+    cp_ms, _ = timed(cstep, 10)
+    _, cpkern = timed(cstep, 5, kernels=True)
+    errs.check("centred_prefill")
+    cp_med = statistics.median(cp_ms)
+    cp_name, _, cp_dom_ms = dominant(cpkern)
+    del cout, cst
+
     # ---- batched multi-token decode: T new tokens per head per call, in place
     multi = {}
     for T in (4, 16):
@@ -564,6 +581,20 @@ def run_ours(args, world, rank, local):
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(dbytes / (cen_kernel_us * 1e-6) / 1e9 / hbm_peak, 4),
                              "algorithmic_bytes_per_launch": dbytes, "traffic": None},
+            },
+            "centred_prefill": {
+                "workload": "mean-centred softmax expansion, order 2, causal prefill of the main workload's inputs "
+                            "(B=1 H=8 N=4096 d_k=16 d_v=64, bf16 in, fp32 out + n=3 state), L2 flushed before each "
+                            "step, median of 10 steps",
+                "ms_per_step": round(cp_med, 5),
+                "Mtok_s": round(tokens / (cp_med * 1e-3) / 1e6, 3),
+                "kernels_ms": {k_: round(t / c, 5) for k_, (c, t) in cpkern.items()},
+                "roofline": {"bound": "hbm", "scope": "whole step", "achieved": round(byts / (cp_med * 1e-3) / 1e9, 2),
+                             "peak": hbm_peak, "unit": "GB/s",
+                             "frac": round(byts / (cp_med * 1e-3) / 1e9 / hbm_peak, 4),
+                             "algorithmic_bytes_per_step": byts,
+                             "note": "same inputs, outputs and state as the main prefill; the three per-degree "
+                                     "read-outs are fp32 CUDA-core work"},
             },
             "multi_token_decode": {
                 "workload": "B=64 H=16 d_k=16 d_v=64 n=3, T new tokens per head per call against the carried "

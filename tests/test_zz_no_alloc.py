@@ -4,14 +4,16 @@ It exists for callers that cannot let a library allocate device memory -- a
 plugin whose host framework owns all memory, or a serving loop that reserves
 memory up front and must not meet an allocation failure mid-step -- and keeps
 its scratch in a fixed array inside the library.  These tests check that it
-returns what the allocating entry point returns, on two calls in a row (the
-second call finds the first call's leftovers in the shared scratch), and that
-work too large for the fixed scratch is refused with a clear status.
+returns what the allocating entry point returns and what the float64 oracle
+returns, on two calls in a row (the second call finds the first call's
+leftovers in the shared scratch), and that work too large for the fixed
+scratch is refused with a clear status.
 
 This file is collected last on purpose."""
 import pytest
 import torch
 
+from oracle import c_oracle as C
 from recurrent_states_b200 import build as B
 from recurrent_states_b200 import synth
 from recurrent_states_b200 import taylor_attn as TA
@@ -53,3 +55,7 @@ def test_noalloc_matches_allocating_prefill_twice():
         assert row_scaled_max_err(f64(out), f64(ref_out)) <= TOL["f32"], call
         ref_logical = f64(TA.state_logical(ref_st.cpu(), d, dv, n))
         assert state_block_errors(st, ref_logical, d, dv, n) <= TOL["f32"], call
+        # and on its own against the float64 oracle
+        o_ref, s_ref = C.recurrent(f64(q), f64(k), f64(v), n, 2.0)
+        assert row_scaled_max_err(f64(out), o_ref) <= TOL["f32"], call
+        assert state_block_errors(st, s_ref, d, dv, n) <= TOL["f32"], call
