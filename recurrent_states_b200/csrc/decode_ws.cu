@@ -83,6 +83,11 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         ptx::bulk_g2s(buf + offv, v + h * kDV, tok_v, &full[b]);
     };
 
+    // launched with programmatic dependent launch: the next grid in the
+    // stream may be scheduled now, and this grid's first memory access (the
+    // producer's first copy; every other access follows one of its copies)
+    // waits until the previous grid has completed and its writes are visible
+    ptx::pdl_launch_dependents();
     // the producer sets up the ring and starts the first copies at once
     int issued = 0;
     if (tid == producer) {
@@ -91,6 +96,7 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             ptx::mbar_init(&empty[i], 1);
         }
         ptx::fence_mbar_init();
+        ptx::pdl_wait_primary();
         for (; issued < nbuf && issued < nheads; ++issued) issue(issued);
     }
     if (tid == 0) s_bad = 0;
@@ -235,10 +241,11 @@ cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* st
     unsigned int* err = device_error_word();
     if (!err) return cudaErrorNotSupported;
     const int grid = num_sms[dev] < BH ? num_sms[dev] : BH;
+    cudaError_t e = cudaSuccess;
     TA_TIMED(stream, "decode_ws_kernel",
-             decode_ws_kernel<Tin><<<grid, kThreadsWS, dyn, stream>>>(q, k, v, state, out, BH, d, n, tau, (int)F,
-                                                                       stride, bytes, buf_al, nbuf, err));
-    return cudaGetLastError();
+             e = launch_maybe_pdl(decode_ws_kernel<Tin>, dim3(grid), dim3(kThreadsWS), dyn, stream, true, q, k, v, state,
+                                  out, BH, d, n, tau, (int)F, stride, bytes, buf_al, nbuf, err));
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template cudaError_t launch_decode_ws<float>(const float*, const float*, const float*, float*, float*, int, int, int,
