@@ -220,6 +220,267 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
     }
 }
 
+// ---------------------------------------------------------------- persistent form
+// The same step for d_v = 64 and features of degree <= 2 (F <= 256), many
+// heads: one CTA per SM walks the heads blockIdx.x, blockIdx.x + gridDim.x,
+// ...  A producer thread keeps one buffer per consumer warpgroup full (a bulk
+// copy of the head's state and of its T tokens' q, k, v rows, completing on
+// the buffer's mbarrier); three consumer warpgroups take the heads in turn.
+// A warpgroup evaluates phi(k_j), phi(q_i) and the block's pairwise weights
+// into its own area, walks the state rows once (read-out of all T tokens from
+// the old row, the T rank-one updates, the new row stored straight to HBM),
+// hands the buffer back, then reduces the read-out and writes the outputs.
+// Head i of a CTA uses buffer i mod 3 and is consumed by warpgroup i mod 3, so
+// each buffer has one consumer that takes its phases in order.
+constexpr int kWGm = 3;
+constexpr int kWGmThreads = 128;
+constexpr int kThreadsWSm = kWGm * kWGmThreads + 32;
+constexpr int kDVw = 64, kDV4w = 16;
+constexpr size_t kMaxDynWSm = 226 * 1024;
+
+struct MultiWsLayout {
+    uint32_t offq, offk, offv, buf;  // one ring buffer: state, then the q, k, v rows
+    uint32_t pk, pq, vf, p, zr, area; // one warpgroup area
+};
+
+__host__ __device__ inline MultiWsLayout multi_ws_layout(int T, int d, int F, uint32_t state_bytes, uint32_t esize) {
+    auto al = [](uint32_t x) { return (x + 127u) & ~127u; };
+    MultiWsLayout L;
+    const uint32_t Tp = (uint32_t)((T + 3) & ~3);
+    L.offq = al(state_bytes);
+    L.offk = L.offq + al((uint32_t)(T * d) * esize);
+    L.offv = L.offk + al((uint32_t)(T * d) * esize);
+    L.buf = L.offv + al((uint32_t)(T * kDVw) * esize);
+    // pk, pq [F][Tp]; after the row walk the same space holds the column
+    // partials [4 warps][T][16 float4]
+    const uint32_t coeff = al((uint32_t)F * Tp * 4);
+    const uint32_t partials = al((uint32_t)(4 * T * kDVw) * 4);
+    L.pk = 0;
+    L.pq = coeff;
+    const uint32_t span = 2 * coeff > partials ? 2 * coeff : partials;
+    L.vf = span;                                   // v rows as fp32 [T][64]
+    L.p = L.vf + al((uint32_t)(T * kDVw) * 4);    // pairwise weights [16][16]
+    L.zr = L.p + al((uint32_t)(kTMax * kTMax) * 4);
+    L.area = L.zr + al((uint32_t)(4 * kTMax) * 4);
+    return L;
+}
+
+__device__ __forceinline__ void wgm_sync(int wg) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + wg), "r"(kWGmThreads) : "memory");
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreadsWSm, 1)
+decode_multi_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                       const float* state_in, float* state_out, float* __restrict__ out, int BH, int T, int d, int n,
+                       float tau, int F, int64_t stride, uint32_t bytes, unsigned int* __restrict__ err) {
+    extern __shared__ __align__(128) unsigned char dsm[];
+    __shared__ __align__(8) uint64_t full[kWGm], empty[kWGm];
+    __shared__ int s_bad, s_fail[kWGm];
+    const MultiWsLayout L = multi_ws_layout(T, d, F, bytes, (uint32_t)sizeof(Tin));
+    unsigned char* areas = dsm + (size_t)kWGm * L.buf;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nheads = BH > (int)blockIdx.x ? (BH - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const uint32_t tok_in = (uint32_t)(T * d) * (uint32_t)sizeof(Tin), tok_v = (uint32_t)(T * kDVw) * (uint32_t)sizeof(Tin);
+    const int producer = kWGm * kWGmThreads;
+    auto issue = [&](int i) {
+        const int b = i % kWGm;
+        const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+        unsigned char* buf = dsm + (size_t)b * L.buf;
+        ptx::mbar_arrive_expect_tx(&full[b], bytes + 2 * tok_in + tok_v);
+        ptx::bulk_g2s(buf, state_in + h * stride, bytes, &full[b]);
+        ptx::bulk_g2s(buf + L.offq, q + h * T * d, tok_in, &full[b]);
+        ptx::bulk_g2s(buf + L.offk, k + h * T * d, tok_in, &full[b]);
+        ptx::bulk_g2s(buf + L.offv, v + h * T * kDVw, tok_v, &full[b]);
+    };
+
+    // launched with programmatic dependent launch: every memory access of the
+    // grid follows the producer's wait on the previous grid
+    ptx::pdl_launch_dependents();
+    int issued = 0;
+    if (tid == producer) {
+        for (int i = 0; i < kWGm; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], 1);
+        }
+        ptx::fence_mbar_init();
+        ptx::pdl_wait_primary();
+        for (; issued < kWGm && issued < nheads; ++issued) issue(issued);
+    }
+    if (tid == 0) s_bad = 0;
+    if (tid < kWGm) s_fail[tid] = 0;
+    __syncthreads();
+
+    if (warp == producer / 32) {
+        if (lane == 0) {
+            int i = issued;
+            for (; i < nheads; ++i) {
+                const int b = i % kWGm;
+                if (!ptx::mbar_wait_or_abort(&empty[b], ((i / kWGm) - 1) & 1, kWaitPolls, &s_bad)) break;
+                issue(i);
+            }
+            for (int j = (i > kWGm ? i - kWGm : 0); j < i; ++j)
+                ptx::mbar_wait(&full[j % kWGm], (j / kWGm) & 1, kWaitPolls);
+        }
+    } else {
+        const int wg = warp >> 2, t = tid & (kWGmThreads - 1), wl = warp & 3;
+        unsigned char* area = areas + (size_t)wg * L.area;
+        float* pk = reinterpret_cast<float*>(area + L.pk);
+        float* pq = reinterpret_cast<float*>(area + L.pq);
+        float4* red = reinterpret_cast<float4*>(area + L.pk);  // after the row walk
+        float* vf = reinterpret_cast<float*>(area + L.vf);
+        float* P = reinterpret_cast<float*>(area + L.p);
+        float* zr = reinterpret_cast<float*>(area + L.zr);
+        const int Tp = (T + 3) & ~3;
+        const int cg = t % kDV4w, rs = t / kDV4w;  // 8 row sets
+        for (int i = wg; i < nheads; i += kWGm) {
+            const int b = i % kWGm;  // == wg: only this warpgroup consumes buffer b
+            if (!ptx::mbar_wait_or_abort(&full[b], (i / kWGm) & 1, kWaitPolls, &s_bad)) s_fail[wg] = 1;
+            wgm_sync(wg);
+            if (s_fail[wg]) break;  // the same value for all 128 threads: set only before this barrier
+            const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+            const unsigned char* buf = dsm + (size_t)b * L.buf;
+            const Tin* xq = reinterpret_cast<const Tin*>(buf + L.offq);
+            const Tin* xk = reinterpret_cast<const Tin*>(buf + L.offk);
+            const Tin* xv = reinterpret_cast<const Tin*>(buf + L.offv);
+            // phi(k_j) and (tau^m/m!) phi(q_i), feature-major with the tokens contiguous
+            for (int e = t; e < F * Tp; e += kWGmThreads) {
+                const int f = e / Tp, j = e % Tp;
+                int m, a, c2;
+                float w;
+                feature_deg2(d, f, m, a, c2, w);
+                float pkv = 0.f, pqv = 0.f;
+                if (j < T) {
+                    const float ka = m >= 1 ? to_float(xk[j * d + a]) : 1.f, kb = m >= 2 ? to_float(xk[j * d + c2]) : 1.f;
+                    const float qa = m >= 1 ? to_float(xq[j * d + a]) : 1.f, qb = m >= 2 ? to_float(xq[j * d + c2]) : 1.f;
+                    pkv = w * ka * kb;
+                    pqv = w * query_coeff(m, tau) * qa * qb;
+                }
+                pk[e] = pkv;
+                pq[e] = pqv;
+            }
+            for (int e = t; e < T * kDVw; e += kWGmThreads) vf[e] = to_float(xv[e]);
+            // the block's own causal part: K(tau q_i.k_j) for j <= i
+            for (int e = t; e < kTMax * kTMax; e += kWGmThreads) {
+                const int ii = e / kTMax, j = e % kTMax;
+                float w = 0.f;
+                if (ii < T && j <= ii) {
+                    float dot = 0.f;
+                    for (int c = 0; c < d; ++c) dot = fmaf(to_float(xq[ii * d + c]), to_float(xk[j * d + c]), dot);
+                    w = taylor_kernel(tau * dot, n);
+                }
+                P[e] = w;
+            }
+            wgm_sync(wg);
+
+            // one walk over the state rows: read-out of every token from the
+            // old row, then the T rank-one updates, the new row to HBM
+            const float4* S4 = reinterpret_cast<const float4*>(buf);
+            float4* G4 = state_out ? reinterpret_cast<float4*>(state_out + h * stride) : nullptr;
+            const float4* V4 = reinterpret_cast<const float4*>(vf);
+            float4 y[kTMax];
+#pragma unroll
+            for (int ii = 0; ii < kTMax; ++ii) y[ii] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int r = rs; r < F; r += kWGmThreads / kDV4w) {
+                float4 s = S4[r * kDV4w + cg];
+                const float4* cq = reinterpret_cast<const float4*>(pq + r * Tp);
+                const float4* ck = reinterpret_cast<const float4*>(pk + r * Tp);
+#pragma unroll
+                for (int i4 = 0; i4 < kTMax / 4; ++i4) {
+                    if (4 * i4 < T) {
+                        const float4 c = cq[i4];
+                        const float cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            y[4 * i4 + u].x = fmaf(cc[u], s.x, y[4 * i4 + u].x);
+                            y[4 * i4 + u].y = fmaf(cc[u], s.y, y[4 * i4 + u].y);
+                            y[4 * i4 + u].z = fmaf(cc[u], s.z, y[4 * i4 + u].z);
+                            y[4 * i4 + u].w = fmaf(cc[u], s.w, y[4 * i4 + u].w);
+                        }
+                    }
+                }
+                if (G4) {
+#pragma unroll
+                    for (int j4 = 0; j4 < kTMax / 4; ++j4) {
+                        if (4 * j4 < T) {  // padded tokens have coefficient 0 and zero v rows are not read
+                            const float4 a = ck[j4];
+                            const float aa[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                if (4 * j4 + u < T) {
+                                    const float4 vv4 = V4[(4 * j4 + u) * kDV4w + cg];
+                                    s.x = fmaf(aa[u], vv4.x, s.x);
+                                    s.y = fmaf(aa[u], vv4.y, s.y);
+                                    s.z = fmaf(aa[u], vv4.z, s.z);
+                                    s.w = fmaf(aa[u], vv4.w, s.w);
+                                }
+                            }
+                        }
+                    }
+                    G4[r * kDV4w + cg] = s;
+                }
+            }
+            float yz[kTMax];
+#pragma unroll
+            for (int ii = 0; ii < kTMax; ++ii) yz[ii] = 0.f;
+            const float* Z = reinterpret_cast<const float*>(buf) + (int64_t)F * kDVw;
+            float* GZ = state_out ? state_out + h * stride + (int64_t)F * kDVw : nullptr;
+            for (int f = t; f < F; f += kWGmThreads) {
+                float z = Z[f];
+#pragma unroll
+                for (int ii = 0; ii < kTMax; ++ii)
+                    if (ii < T) yz[ii] = fmaf(pq[f * Tp + ii], z, yz[ii]);
+                if (GZ) {
+#pragma unroll
+                    for (int j = 0; j < kTMax; ++j)
+                        if (j < T) z += pk[f * Tp + j];
+                    GZ[f] = z;
+                }
+            }
+            if (G4)  // the state's padding stays zero
+                for (int64_t e = (int64_t)F * (kDVw + 1) + t; e < stride; e += kWGmThreads) state_out[h * stride + e] = 0.f;
+            // the buffer and the coefficients have been read: hand the buffer
+            // back, and reuse the coefficient space for the column partials
+            ptx::fence_proxy_async_smem();
+            wgm_sync(wg);
+            if (t == 0) ptx::mbar_arrive(&empty[b]);
+#pragma unroll
+            for (int ii = 0; ii < kTMax; ++ii) {
+                if (ii < T) {
+                    y[ii].x += __shfl_xor_sync(0xffffffffu, y[ii].x, 16);
+                    y[ii].y += __shfl_xor_sync(0xffffffffu, y[ii].y, 16);
+                    y[ii].z += __shfl_xor_sync(0xffffffffu, y[ii].z, 16);
+                    y[ii].w += __shfl_xor_sync(0xffffffffu, y[ii].w, 16);
+                    if (lane < kDV4w) red[(wl * T + ii) * kDV4w + lane] = y[ii];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) yz[ii] += __shfl_xor_sync(0xffffffffu, yz[ii], o);
+                    if (lane == 0) zr[wl * kTMax + ii] = yz[ii];
+                }
+            }
+            wgm_sync(wg);
+            for (int e = t; e < T * kDVw; e += kWGmThreads) {
+                const int ii = e / kDVw, c = e % kDVw;
+                float acc = 0.f, den = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const float4 r4 = red[(w * T + ii) * kDV4w + (c >> 2)];
+                    acc += (c & 3) == 0 ? r4.x : (c & 3) == 1 ? r4.y : (c & 3) == 2 ? r4.z : r4.w;
+                    den += zr[w * kTMax + ii];
+                }
+                for (int j = 0; j <= ii; ++j) {
+                    const float w = P[ii * kTMax + j];
+                    acc = fmaf(w, vf[j * kDVw + c], acc);
+                    den += w;
+                }
+                out[(h * T + ii) * kDVw + c] = acc / den;
+            }
+            wgm_sync(wg);  // the area is rewritten only after every thread is done with it
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && s_bad) atomicOr(err, kErrDecodeLoad);
+}
+
 template <typename Tin, int DV4>
 cudaError_t launch_multi(const Tin* q, const Tin* k, const Tin* v, const float* state_in, float* state_out, float* out,
                          int BH, int T, int d, int n, float tau, int F, int64_t stride, uint32_t bytes, size_t dyn,
@@ -242,11 +503,51 @@ cudaError_t launch_multi(const Tin* q, const Tin* k, const Tin* v, const float* 
 
 }  // namespace
 
+// The persistent form, when it applies (else cudaErrorNotSupported).
+template <typename Tin>
+cudaError_t launch_multi_ws(const Tin* q, const Tin* k, const Tin* v, const float* state_in, float* state_out,
+                            float* out, int BH, int T, int d, int dv, int n, float tau, int64_t F, int64_t stride,
+                            cudaStream_t stream) {
+    // features of degree <= 2 only (always the case for F <= 256 at the supported d_k)
+    if (dv != kDVw || F > 256 || n > 3 || ((int64_t)T * d * sizeof(Tin)) % 16 != 0) return cudaErrorNotSupported;
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t set_err[kMaxDevices];
+    static int num_sms[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&]() {
+        set_err[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(decode_multi_ws_kernel<Tin>),
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDynWSm);
+        if (set_err[dev] == cudaSuccess)
+            set_err[dev] = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    });
+    if (set_err[dev] != cudaSuccess) return set_err[dev];
+    if (BH < 2 * num_sms[dev]) return cudaErrorNotSupported;  // few heads: one CTA per head is as good
+    const uint32_t bytes = (uint32_t)((F * (dv + 1) * 4 + 15) / 16 * 16);
+    const MultiWsLayout L = multi_ws_layout(T, d, (int)F, bytes, (uint32_t)sizeof(Tin));
+    const size_t dyn = (size_t)kWGm * (L.buf + L.area);
+    if (dyn > kMaxDynWSm) return cudaErrorNotSupported;
+    unsigned int* err = device_error_word();
+    if (!err) return cudaErrorNotSupported;
+    const int grid = num_sms[dev] < BH ? num_sms[dev] : BH;
+    cudaError_t e = cudaSuccess;
+    TA_TIMED(stream, "decode_multi_ws_kernel",
+             e = launch_maybe_pdl(decode_multi_ws_kernel<Tin>, dim3(grid), dim3(kThreadsWSm), dyn, stream, true, q, k,
+                                  v, state_in, state_out, out, BH, T, d, n, tau, (int)F, stride, bytes, err));
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <typename Tin>
 cudaError_t launch_decode_multi(const Tin* q, const Tin* k, const Tin* v, const float* state_in, float* state_out,
                                 float* out, int BH, int T, int d, int dv, int n, float tau, int64_t F, int64_t stride,
                                 cudaStream_t stream) {
     if (T < 1 || T > kTMax || F > 1024) return cudaErrorNotSupported;
+    {
+        const cudaError_t ew = launch_multi_ws(q, k, v, state_in, state_out, out, BH, T, d, dv, n, tau, F, stride,
+                                               stream);
+        if (ew != cudaErrorNotSupported) return ew;
+    }
     if (dv != 16 && dv != 32 && dv != 64 && dv != 128) return cudaErrorNotSupported;
     const int64_t used_bytes = F * (dv + 1) * 4;
     const uint32_t bytes = (uint32_t)((used_bytes + 15) / 16 * 16);

@@ -62,6 +62,13 @@ CASES = [
     (1, 1, 2600, 64, 64, 3),
     (1, 1, 700, 32, 64, 4),   # run-time feature descriptors on the tiled path
     (1, 1, 500, 64, 64, 2),
+    # the one-launch cluster prefill (d_k 16, d_v 64, n <= 3): segments of one
+    # chunk, of two chunks with a one-token last segment, full 16-CTA clusters
+    (2, 3, 2048, 16, 64, 3),
+    (1, 3, 2049, 16, 64, 3),
+    (2, 2, 3000, 16, 64, 2),
+    (1, 2, 4096, 16, 64, 1),
+    (1, 1, 3967, 16, 64, 3),
 ]
 
 
@@ -340,6 +347,7 @@ def test_merge_and_split_prefill():
 @pytest.mark.parametrize("d,dv,n,N,cut", [(16, 64, 3, 1000, 384), (16, 64, 3, 700, 77), (16, 64, 3, 300, 1),
                                           (16, 16, 3, 500, 256), (64, 64, 3, 600, 130), (16, 64, 5, 400, 200),
                                           (32, 64, 3, 2600, 300), (7, 12, 2, 200, 33),
+                                          (16, 64, 3, 4300, 200), (16, 64, 2, 2200, 130),
                                           # a few new tokens: the multi-token decode kernel
                                           (16, 64, 3, 300, 292), (16, 64, 3, 300, 299), (16, 16, 3, 200, 184),
                                           (32, 64, 3, 300, 290), (16, 128, 3, 100, 88),
@@ -386,6 +394,32 @@ def test_multi_token_decode_blocks_follow_the_recursion(dtype):
         o, _ = cont(sl(q, t0, t0 + T), sl(k, t0, t0 + T), sl(v, t0, t0 + T), st, n, tau, state_out=st)
         torch.cuda.synchronize()
         assert row_scaled_max_err(f64(o), ref_out[:, :, t0:t0 + T]) <= TOL[dtype]
+        t0 += T
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d,n", [(16, 3), (16, 2), (32, 2)])
+def test_multi_token_decode_many_heads(dtype, d, n):
+    """320 heads (enough for the persistent multi-token kernel, whose three
+    warpgroups take heads in turn): blocks of 16, 1, 7 and 4 new tokens fed in
+    place after a 200-token prefill, against the oracle's recursion (outputs
+    of every block, final state)."""
+    B, H, dv, tau = 32, 10, 64, 2.0 if n == 3 else 1.0
+    blocks = [16, 1, 7, 4]
+    prefix = 200
+    N = prefix + sum(blocks)
+    q, k, v = synth.qkv(B, H, N, d, dv, seed=91 + d + n, dtype=dtype)
+    prefill = TA.taylor_attn_prefill if dtype == "bf16" else TA.taylor_attn_prefill_f32
+    cont = TA.taylor_attn_prefill_from_state if dtype == "bf16" else TA.taylor_attn_prefill_from_state_f32
+    sl = lambda t, a, b: t[:, :, a:b].contiguous().to(DEV)  # noqa: E731
+    _, st = prefill(sl(q, 0, prefix), sl(k, 0, prefix), sl(v, 0, prefix), n, tau, state_out=True)
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    t0 = prefix
+    for T in blocks:
+        o, _ = cont(sl(q, t0, t0 + T), sl(k, t0, t0 + T), sl(v, t0, t0 + T), st, n, tau, state_out=st)
+        torch.cuda.synchronize()
+        assert row_scaled_max_err(f64(o), ref_out[:, :, t0:t0 + T]) <= TOL[dtype], T
         t0 += T
     assert state_block_errors(st, ref_st, d, dv, n) <= TOL[dtype]
 
