@@ -75,6 +75,9 @@ int prefill_impl(const Tin* q, const Tin* k, const Tin* v, const float* state_in
         if (e != cudaErrorNotSupported) return cuda_status(e);
     }
     if (allow_tc) {
+        const int fused = ta::tc::try_prefill_fused(q, k, v, out, state_in, state_out, (int)BH, N, d_k, d_v, n, tau, F,
+                                                    stride, stream);
+        if (fused != ta::tc::kNotApplicable) return fused;
         const int tc = ta::tc::try_prefill(q, k, v, out, state_in, state_out, (int)BH, N, d_k, d_v, n, tau, F,
                                            stride, stream);
         if (tc != ta::tc::kNotApplicable) return tc;

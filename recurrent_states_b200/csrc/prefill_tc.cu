@@ -30,6 +30,7 @@
 #include "internal.h"
 #include "prefill_tc.h"
 #include "phase.cuh"
+#include "phi16.cuh"
 #include "ptx.cuh"
 #include "tcgen05.cuh"
 
@@ -47,7 +48,6 @@ constexpr int kNV = 80;       // columns of [V | 1 | 0 ...]  (MMA N)
 constexpr int kFP = 160;      // features padded to a multiple of 16
 constexpr int kThreads = 256;
 constexpr uint32_t kWaitPolls = 1u << 24;
-constexpr float kSqrt2 = (float)cx_sqrt(2.0);
 
 // Shared-memory layouts (bytes).  K-major operands use LBO = 128; MN-major
 // operands use SBO = 128 (see tcgen05.cuh).
@@ -89,38 +89,6 @@ __device__ __forceinline__ void ld_row16(const bf16* p, float (&x)[16]) {
         x[2 * i] = __uint_as_float(w[i] << 16);
         x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     }
-}
-
-// Writes features [8*G0, 8*G1) of the 160 padded features of one token,
-// scaled per degree by (e0, e1, e2), as hi/lo bf16 groups of 8 through
-// `put(group, hi, lo)`.  All indices are compile-time constants after
-// unrolling, so features outside the range cost nothing.
-template <int G0, int G1, typename Put>
-__device__ __forceinline__ void phi16_groups(const float (&x)[16], float e0, float e1, float e2, Put put) {
-    float buf[8];
-    int f = 0;
-    auto emit = [&](auto make) {
-        if (f >= 8 * G0 && f < 8 * G1) {
-            buf[f & 7] = make();
-            if ((f & 7) == 7) {
-                uint4 hi, lo;
-                split8(buf, hi, lo);
-                put(f >> 3, hi, lo);
-            }
-        }
-        ++f;
-    };
-    emit([&] { return e0; });
-#pragma unroll
-    for (int i = 0; i < 16; ++i) emit([&] { return e1 * x[i]; });
-    const float e2o = e2 * kSqrt2;
-#pragma unroll
-    for (int a = 0; a < 16; ++a) {
-#pragma unroll
-        for (int b = a; b < 16; ++b) emit([&] { return (a == b ? e2 : e2o) * x[a] * x[b]; });
-    }
-#pragma unroll
-    for (int i = 153; i < kFP; ++i) emit([&] { return 0.f; });
 }
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
