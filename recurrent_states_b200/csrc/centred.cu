@@ -151,6 +151,10 @@ cudaError_t launch_centred_decode(const Tin* q, const Tin* k, const Tin* v, floa
                                   int d, int dv, int order, float tau, int64_t F, int64_t stride,
                                   cudaStream_t stream) {
     if (d < 1 || d > kMaxDk || dv < 4 || dv > kMaxDv || dv % 4 != 0) return cudaErrorNotSupported;
+    {  // many heads of a small state: the persistent warp-specialised kernel
+        const cudaError_t e = launch_centred_decode_ws(q, k, v, state, out, BH, d, dv, order, tau, F, stride, stream);
+        if (e != cudaErrorNotSupported) return e;
+    }
     const int nrs = kThreadsC / (dv / 4);
     const size_t smem = (size_t)(2 * F + 3 * (int64_t)nrs * dv) * sizeof(float);
     if (smem > 48 * 1024) return cudaErrorNotSupported;  // F <= 2145 (d_k 64) needs 29.4 KB

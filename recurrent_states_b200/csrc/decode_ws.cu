@@ -47,8 +47,8 @@ constexpr int kMaxDevices = 64;
 
 struct WGArea {                 // per consumer warpgroup
     float pk[kMaxF], pq[kMaxF];
-    float4 red[4][kDV4];
-    float zr[4];
+    float4 red[3][4][kDV4];     // column partials per degree (one degree for the Taylor read-out)
+    float zr[3][4];
     int fail;                   // written only before a warpgroup barrier, read after it
 };
 
@@ -56,11 +56,21 @@ __device__ __forceinline__ void wg_sync(int wg) {
     asm volatile("bar.sync %0, %1;" ::"r"(1 + wg), "r"(kWGThreads) : "memory");
 }
 
-template <typename Tin>
+// CENTRED: the read-out of the mean-centred softmax expansion (order 1 or 2)
+// over the n = 3 state instead of the Taylor read-out: the query features
+// carry no tau^m/m!, the row walk keeps one accumulator per degree, and the
+// epilogue combines the three per-degree read-outs R_m (Su Jianlin, "Taylor
+// expansions of logsumexp and softmax", kexue.fm translation 11814, sections
+// "Calculating the Gradient" and "Linear Attention"):
+//   n = R_0[z], V = R_0[v], qkbar = R_1[z] / n,
+//   o = V/n + tau (R_1[v] - qkbar V)/n
+//     [+ (tau^2 (R_2[v] - 2 qkbar R_1[v] + qkbar^2 V) - tau^2 (R_2[z] - n qkbar^2) V/n) / (2n)].
+template <typename Tin, bool CENTRED>
 __global__ void __launch_bounds__(kThreadsWS, 1)
 decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                  float* __restrict__ state, float* __restrict__ out, int BH, int d, int n, float tau, int F,
-                 int64_t stride, uint32_t bytes, uint32_t buf_bytes, int nbuf, unsigned int* __restrict__ err) {
+                 int64_t stride, uint32_t bytes, uint32_t buf_bytes, int nbuf, int order,
+                 unsigned int* __restrict__ err) {
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ __align__(8) uint64_t full[kMaxBuf], empty[kMaxBuf];
     __shared__ int s_bad;
@@ -125,7 +135,7 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         float w0, w1;
         feature_deg2(d, t < F ? t : 0, m0, i0, j0, w0);
         feature_deg2(d, t + kWGThreads < F ? t + kWGThreads : 0, m1, i1, j1, w1);
-        const float wq0 = w0 * query_coeff(m0, tau), wq1 = w1 * query_coeff(m1, tau);
+        const float wq0 = CENTRED ? w0 : w0 * query_coeff(m0, tau), wq1 = CENTRED ? w1 : w1 * query_coeff(m1, tau);
         for (int i = wg; i < nheads; i += kWG) {
             const int b = i % nbuf;  // == wg modulo kWG: only this warpgroup consumes buffer b
             if (!ptx::mbar_wait_or_abort(&full[b], (i / nbuf) & 1, kWaitPolls, &s_bad)) A.fail = 1;
@@ -153,51 +163,91 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             wg_sync(wg);
             const float4* S4 = reinterpret_cast<const float4*>(buf);
             float4* G4 = reinterpret_cast<float4*>(state + h * stride);
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+            constexpr int ND = CENTRED ? 3 : 1;  // accumulators: per degree, or one
+            float4 y[ND];
+#pragma unroll
+            for (int m = 0; m < ND; ++m) y[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+            // rows [lo, hi) of this thread's row set into accumulator m
+            auto walk = [&](int lo, int hi, float4& acc) {
+                const int r0 = lo + ((rs - lo) % (kWGThreads / kDV4) + kWGThreads / kDV4) % (kWGThreads / kDV4);
 #pragma unroll 4
-            for (int r = rs; r < F; r += kWGThreads / kDV4) {
-                const float a = A.pk[r], c = A.pq[r];
-                float4 s = S4[r * kDV4 + cg];
-                s.x = fmaf(a, v4.x, s.x);
-                s.y = fmaf(a, v4.y, s.y);
-                s.z = fmaf(a, v4.z, s.z);
-                s.w = fmaf(a, v4.w, s.w);
-                G4[r * kDV4 + cg] = s;
-                y.x = fmaf(c, s.x, y.x);
-                y.y = fmaf(c, s.y, y.y);
-                y.z = fmaf(c, s.z, y.z);
-                y.w = fmaf(c, s.w, y.w);
+                for (int r = r0; r < hi; r += kWGThreads / kDV4) {
+                    const float a = A.pk[r], c = A.pq[r];
+                    float4 s = S4[r * kDV4 + cg];
+                    s.x = fmaf(a, v4.x, s.x);
+                    s.y = fmaf(a, v4.y, s.y);
+                    s.z = fmaf(a, v4.z, s.z);
+                    s.w = fmaf(a, v4.w, s.w);
+                    G4[r * kDV4 + cg] = s;
+                    acc.x = fmaf(c, s.x, acc.x);
+                    acc.y = fmaf(c, s.y, acc.y);
+                    acc.z = fmaf(c, s.z, acc.z);
+                    acc.w = fmaf(c, s.w, acc.w);
+                }
+            };
+            if (CENTRED) {
+                walk(0, 1, y[0]);
+                walk(1, d + 1, y[ND > 1 ? 1 : 0]);
+                walk(d + 1, F, y[ND > 2 ? 2 : 0]);
+            } else {
+                walk(0, F, y[0]);
             }
-            float yz = 0.f;
+            float yz[ND];
+#pragma unroll
+            for (int m = 0; m < ND; ++m) yz[m] = 0.f;
             const float* Z = reinterpret_cast<const float*>(buf) + (int64_t)F * kDV;
             float* GZ = state + h * stride + (int64_t)F * kDV;
             for (int f = t; f < F; f += kWGThreads) {
                 const float z = Z[f] + A.pk[f];
                 GZ[f] = z;
-                yz = fmaf(A.pq[f], z, yz);
+                const int m = CENTRED ? (f == 0 ? 0 : (f <= d ? 1 : 2)) : 0;
+#pragma unroll
+                for (int mm = 0; mm < ND; ++mm)
+                    if (mm == m) yz[mm] = fmaf(A.pq[f], z, yz[mm]);
             }
             // the buffer has been read: hand it back once the whole warpgroup is past here
             ptx::fence_proxy_async_smem();
-            y.x += __shfl_xor_sync(0xffffffffu, y.x, 16);
-            y.y += __shfl_xor_sync(0xffffffffu, y.y, 16);
-            y.z += __shfl_xor_sync(0xffffffffu, y.z, 16);
-            y.w += __shfl_xor_sync(0xffffffffu, y.w, 16);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) yz += __shfl_xor_sync(0xffffffffu, yz, o);
-            if (lane < kDV4) A.red[wl][lane] = y;
-            if (lane == 0) A.zr[wl] = yz;
+            for (int m = 0; m < ND; ++m) {
+                y[m].x += __shfl_xor_sync(0xffffffffu, y[m].x, 16);
+                y[m].y += __shfl_xor_sync(0xffffffffu, y[m].y, 16);
+                y[m].z += __shfl_xor_sync(0xffffffffu, y[m].z, 16);
+                y[m].w += __shfl_xor_sync(0xffffffffu, y[m].w, 16);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) yz[m] += __shfl_xor_sync(0xffffffffu, yz[m], o);
+                if (lane < kDV4) A.red[m][wl][lane] = y[m];
+                if (lane == 0) A.zr[m][wl] = yz[m];
+            }
             wg_sync(wg);
             if (t == 0) ptx::mbar_arrive(&empty[b]);
             if (t < kDV) {
                 const int g4 = t >> 2, c4 = t & 3;
-                float acc = 0.f, den = 0.f;
+                float R[ND], Rz[ND];
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const float4 r4 = A.red[w][g4];
-                    acc += c4 == 0 ? r4.x : c4 == 1 ? r4.y : c4 == 2 ? r4.z : r4.w;
-                    den += A.zr[w];
+                for (int m = 0; m < ND; ++m) {
+                    R[m] = 0.f;
+                    Rz[m] = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float4 r4 = A.red[m][w][g4];
+                        R[m] += c4 == 0 ? r4.x : c4 == 1 ? r4.y : c4 == 2 ? r4.z : r4.w;
+                        Rz[m] += A.zr[m][w];
+                    }
                 }
-                out[h * kDV + t] = acc / den;
+                float o;
+                if (CENTRED) {
+                    const float cnt = Rz[0], V = R[0], qkbar = Rz[ND > 1 ? 1 : 0] / cnt;
+                    o = V / cnt + tau * (R[ND > 1 ? 1 : 0] - qkbar * V) / cnt;
+                    if (order >= 2) {
+                        const float t2 = tau * tau;
+                        const float sum_a2v = t2 * (R[ND > 2 ? 2 : 0] - 2.0f * qkbar * R[ND > 1 ? 1 : 0] + qkbar * qkbar * V);
+                        const float sum_a2 = t2 * (Rz[ND > 2 ? 2 : 0] - cnt * qkbar * qkbar);
+                        o += (sum_a2v - sum_a2 * V / cnt) / (2.0f * cnt);
+                    }
+                } else {
+                    o = R[0] / Rz[0];
+                }
+                out[h * kDV + t] = o;
             }
             // A.pk, A.pq, A.red are rewritten only after the next head's first barrier
         }
@@ -206,11 +256,9 @@ decode_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     if (tid == 0 && s_bad) atomicOr(err, kErrDecodeLoad);
 }
 
-}  // namespace
-
-template <typename Tin>
-cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
-                             int dv, int n, float tau, int64_t F, int64_t stride, cudaStream_t stream) {
+template <typename Tin, bool CENTRED>
+cudaError_t launch_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d, int dv,
+                      int n, float tau, int64_t F, int64_t stride, int order, cudaStream_t stream) {
     // features of degree <= 2 only (always the case for F <= 256 at the supported d_k)
     if (dv != kDV || F > kMaxF || n > 3 || (d * (int)sizeof(Tin)) % 16 != 0) return cudaErrorNotSupported;
     static std::once_flag once[kMaxDevices];
@@ -220,7 +268,7 @@ cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* st
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        set_err[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(decode_ws_kernel<Tin>),
+        set_err[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(decode_ws_kernel<Tin, CENTRED>),
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDynWS);
         if (set_err[dev] == cudaSuccess)
             set_err[dev] = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
@@ -242,12 +290,32 @@ cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* st
     if (!err) return cudaErrorNotSupported;
     const int grid = num_sms[dev] < BH ? num_sms[dev] : BH;
     cudaError_t e = cudaSuccess;
-    TA_TIMED(stream, "decode_ws_kernel",
-             e = launch_maybe_pdl(decode_ws_kernel<Tin>, dim3(grid), dim3(kThreadsWS), dyn, stream, true, q, k, v, state,
-                                  out, BH, d, n, tau, (int)F, stride, bytes, buf_al, nbuf, err));
+    TA_TIMED(stream, CENTRED ? "centred_decode_ws_kernel" : "decode_ws_kernel",
+             e = launch_maybe_pdl(decode_ws_kernel<Tin, CENTRED>, dim3(grid), dim3(kThreadsWS), dyn, stream, true, q,
+                                  k, v, state, out, BH, d, n, tau, (int)F, stride, bytes, buf_al, nbuf, order, err));
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+}  // namespace
+
+template <typename Tin>
+cudaError_t launch_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH, int d,
+                             int dv, int n, float tau, int64_t F, int64_t stride, cudaStream_t stream) {
+    return launch_ws<Tin, false>(q, k, v, state, out, BH, d, dv, n, tau, F, stride, 0, stream);
+}
+
+template <typename Tin>
+cudaError_t launch_centred_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH,
+                                     int d, int dv, int order, float tau, int64_t F, int64_t stride,
+                                     cudaStream_t stream) {
+    return launch_ws<Tin, true>(q, k, v, state, out, BH, d, dv, 3, tau, F, stride, order, stream);
+}
+
+template cudaError_t launch_centred_decode_ws<float>(const float*, const float*, const float*, float*, float*, int,
+                                                     int, int, int, float, int64_t, int64_t, cudaStream_t);
+template cudaError_t launch_centred_decode_ws<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                                             const __nv_bfloat16*, float*, float*, int, int, int, int,
+                                                             float, int64_t, int64_t, cudaStream_t);
 template cudaError_t launch_decode_ws<float>(const float*, const float*, const float*, float*, float*, int, int, int,
                                              int, float, int64_t, int64_t, cudaStream_t);
 template cudaError_t launch_decode_ws<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,

@@ -45,6 +45,13 @@ cudaError_t launch_centred_decode(const Tin* q, const Tin* k, const Tin* v, floa
                                   int d, int dv, int order, float tau, int64_t F, int64_t stride,
                                   cudaStream_t stream);
 
+// The same persistent kernel with the mean-centred expansion's read-out
+// (order 1 or 2) over the n = 3 state; cudaErrorNotSupported as above.
+template <typename Tin>
+cudaError_t launch_centred_decode_ws(const Tin* q, const Tin* k, const Tin* v, float* state, float* out, int BH,
+                                     int d, int dv, int order, float tau, int64_t F, int64_t stride,
+                                     cudaStream_t stream);
+
 // Persistent warp-specialised decode for d_v 64 and at most 256 features;
 // cudaErrorNotSupported when the shape (or a small number of heads) is
 // better served by the one-CTA-per-head kernel.

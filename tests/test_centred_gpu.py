@@ -87,3 +87,21 @@ def test_centred_decode_on_the_decode_workload_shape():
     assert row_scaled_max_err(f64(o)[bi, hi], ref_o) <= TOL_STEP
     got_S = f64(TA.state_logical(st.cpu(), d, dv, 3))[bi, hi]
     assert np.abs(got_S - ref_S).max() <= TOL_STEP * np.abs(ref_S).max()
+
+
+@pytest.mark.parametrize("order", [1, 2])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_centred_decode_many_heads_follows_the_definition(order, dtype):
+    """320 heads (enough for the persistent decode kernel, which carries the
+    centred read-out as three per-degree accumulators), 10 steps from a zero
+    state, each step's outputs against the per-row definition."""
+    B, H, N, d, dv, tau = 32, 10, 10, 16, 64, 2.0
+    q, k, v = synth.qkv(B, H, N, d, dv, seed=300 + order, dtype=dtype)
+    ref = O.centred_direct(f64(q), f64(k), f64(v), order, tau)
+    st = torch.zeros((B, H, TA.taylor_attn_state_stride(d, dv, 3)), device=DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    outs = [_fn(dtype)(qd[:, :, i].contiguous(), kd[:, :, i].contiguous(), vd[:, :, i].contiguous(), st, order, tau)
+            for i in range(N)]
+    got = torch.stack(outs, dim=2)
+    assert row_scaled_max_err(f64(got), ref) <= TOL_STEP
+    assert state_block_errors(st, T.state_of(f64(k), f64(v), 3), d, dv, 3) <= TOL_STEP
