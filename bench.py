@@ -244,6 +244,7 @@ def run_ours(args, world, rank, local):
         x = torch.randn(shape, device=dev, generator=g, dtype=torch.float32)
         return (x / x.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
 
+    blocks = {"decode", "centred_prefill", "sweep", "large"} if args.blocks == "all" else set(args.blocks.split(","))
     w = MAIN
     B, H, N, d, dv, n, tau = w["B"], w["H"], w["N"], w["d_k"], w["d_v"], w["n"], w["tau"]
     qh, kh, vh = synth.qkv(B, H, N, d, dv, seed=rank, dtype="bf16")
@@ -284,204 +285,6 @@ def run_ours(args, world, rank, local):
     byts, flops = kernel_algorithmic("prefill", w, 1)
     achieved = byts / (per_launch_ms * 1e-3) / 1e9
 
-    # ---- decode: states of 65,536-token random prefixes built by the library
-    dw = DECODE
-    dB, dH = dw["B"], dw["H"]
-    dstride = TA.taylor_attn_state_stride(dw["d_k"], dw["d_v"], dw["n"])
-    dstate = torch.zeros((dB, dH, dstride), dtype=torch.float32, device=dev)
-    g = torch.Generator(device=dev)
-    g.manual_seed(rank)
-    seg = 4096
-    tmp_state = torch.empty_like(dstate)
-    for s0 in range(0, dw["prefix"], seg):
-        pq_ = unit_dev(g, (dB, dH, seg, dw["d_k"]))
-        pk_ = unit_dev(g, (dB, dH, seg, dw["d_k"]))
-        pv_ = torch.randn((dB, dH, seg, dw["d_v"]), device=dev, generator=g).to(torch.bfloat16)
-        po = torch.empty((dB, dH, seg, dw["d_v"]), dtype=torch.float32, device=dev)
-        TA.taylor_attn_prefill(pq_, pk_, pv_, dw["n"], dw["tau"], out=po, state_out=tmp_state)
-        TA.taylor_attn_state_merge(dstate, tmp_state, dw["d_k"], dw["d_v"], dw["n"], out=dstate)
-        del pq_, pk_, pv_, po
-    del tmp_state
-    errs.check("decode_prefix")
-    dsteps = max(args.steps, 24)
-    toks = [synth.decode_tokens(dB, dH, dw["d_k"], dw["d_v"], s, seed=rank) for s in range(dsteps)]
-    toks = [(a.to(dev), b.to(dev), c.to(dev)) for a, b, c in toks]
-    dout = torch.empty((dB, dH, dw["d_v"]), dtype=torch.float32, device=dev)
-    # six independent batches of 1,024 carried states (245 MB > L2): step s
-    # updates batch s % 6, so its states were last touched six steps earlier
-    dstates = [dstate] + [dstate.clone() for _ in range(DECODE_BUFFERS - 1)]
-
-    def dec(i):
-        TA.taylor_attn_decode(*toks[i], dstates[i % DECODE_BUFFERS], dw["n"], dw["tau"], out=dout)
-
-    for s in range(max(args.warmup, 3) + DECODE_BUFFERS):
-        dec(s % dsteps)
-    torch.cuda.synchronize()
-    # steady state: back to back, one pair of events around the whole run
-    # (its device time over the steps), then per-launch events in a second run
-    e0, e1 = ev_pair()
-    e0.record(stream)
-    for s in range(dsteps):
-        dec(s)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    dec_us = e0.elapsed_time(e1) * 1e3 / dsteps
-    _, dkern = timed(dec, dsteps, flushed=False, kernels=True)
-    dk_name, _, dk_ms = dominant(dkern)
-    dec_kernel_us = dk_ms * 1e3
-    # one step after an L2 flush (cold reads, write-back after the kernel), context
-    dflush_ms, _ = timed(dec, dsteps, flushed=True)
-    # warm L2: the same batch of states step after step (it fits in L2), context
-    e0.record(stream)
-    for s in range(dsteps):
-        TA.taylor_attn_decode(*toks[s], dstate, dw["n"], dw["tau"], out=dout)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    dec_warm_us = e0.elapsed_time(e1) * 1e3 / dsteps
-    errs.check("decode")
-    dec_us_max = allmax(dec_us, world, dev)
-    dbytes, dflops = kernel_algorithmic("decode", dw, 1)
-
-    # ---- the mean-centred softmax expansion (order 2) on the same carried
-    # states: same state traffic, a three-way read-out; timed like decode
-    def cen(i):
-        TA.taylor_attn_centred_decode(*toks[i], dstates[i % DECODE_BUFFERS], 2, dw["tau"], out=dout)
-
-    for s in range(DECODE_BUFFERS + 3):
-        cen(s)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for s in range(dsteps):
-        cen(s)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    cen_us = e0.elapsed_time(e1) * 1e3 / dsteps
-    _, ckern = timed(cen, dsteps, flushed=False, kernels=True)
-    ck_name, _, ck_ms = dominant(ckern)
-    cen_kernel_us = ck_ms * 1e3
-    errs.check("centred_decode")
-
-    # ---- the mean-centred expansion's prefill (order 2) on the main workload's inputs
-    cout = torch.empty_like(out)
-    cst = torch.empty_like(st)
-
-    def cstep(i=0):
-        TA.taylor_attn_centred_prefill(q, k, v, 2, tau, out=cout, state_out=cst)
-
-    for _ in range(3):
-        flush_l2()
-        cstep()
-    cp_ms, _ = timed(cstep, 10)
-    _, cpkern = timed(cstep, 5, kernels=True)
-    errs.check("centred_prefill")
-    cp_med = statistics.median(cp_ms)
-    cp_name, _, cp_dom_ms = dominant(cpkern)
-    del cout, cst
-
-    # ---- batched multi-token decode: T new tokens per head per call, in place
-    multi = {}
-    for T in (4, 16):
-        mtoks = [(unit_dev(g, (dB, dH, T, dw["d_k"])), unit_dev(g, (dB, dH, T, dw["d_k"])),
-                  torch.randn((dB, dH, T, dw["d_v"]), device=dev, generator=g).to(torch.bfloat16))
-                 for _ in range(dsteps)]
-        mout = torch.empty((dB, dH, T, dw["d_v"]), dtype=torch.float32, device=dev)
-
-        def mdec(i):
-            sb = dstates[i % DECODE_BUFFERS]
-            TA.taylor_attn_prefill_from_state(*mtoks[i], sb, dw["n"], dw["tau"], out=mout, state_out=sb)
-
-        for s_ in range(DECODE_BUFFERS + 3):
-            mdec(s_)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for s_ in range(dsteps):
-            mdec(s_)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        m_us = e0.elapsed_time(e1) * 1e3 / dsteps
-        _, mk = timed(mdec, dsteps, flushed=False, kernels=True)
-        mk_name, _, mk_ms = dominant(mk)
-        mk_us = mk_ms * 1e3
-        Fd = TA.taylor_attn_num_features(dw["d_k"], dw["n"])
-        m_bytes = dB * dH * (2 * Fd * (dw["d_v"] + 1) * 4 + T * ((2 * dw["d_k"] + dw["d_v"]) * 2 + dw["d_v"] * 4))
-        multi[str(T)] = {"us_per_call": round(m_us, 3), "kernel": mk_name, "kernel_us": round(mk_us, 3),
-                         "Mtok_s": round(dB * dH * T / (m_us * 1e-6) / 1e6, 2),
-                         "hbm_frac": round(m_bytes / (mk_us * 1e-6) / 1e9 / hbm_peak, 4),
-                         "algorithmic_bytes_per_launch": m_bytes}
-        del mtoks, mout
-    errs.check("multi_token_decode")
-    del dstates
-
-    # ---- order sweep: n = 1..5 at B1 H8 N8192 d_k16 d_v64, q, k unit-normalised
-    # and (second arm) q, k ~ N(0, 4) as drawn
-    sw = SWEEP
-    sweep = {}
-    for arm, normalised in (("normalised", True), ("unnormalised_var4", False)):
-        sq, sk, sv = synth.qkv(sw["B"], sw["H"], sw["N"], sw["d_k"], sw["d_v"], seed=rank, dtype="bf16",
-                               normalise=normalised, qk_var=1.0 if normalised else 4.0)
-        sq, sk, sv = sq.to(dev), sk.to(dev), sv.to(dev)
-        sout = torch.empty((sw["B"], sw["H"], sw["N"], sw["d_v"]), dtype=torch.float32, device=dev)
-        res = {}
-        for sn in sw["orders"]:
-            sst = torch.empty((sw["B"], sw["H"], TA.taylor_attn_state_stride(sw["d_k"], sw["d_v"], sn)),
-                              dtype=torch.float32, device=dev)
-
-            def sstep(i, sn=sn, sst=sst):
-                TA.taylor_attn_prefill(sq, sk, sv, sn, sw["tau"], out=sout, state_out=sst)
-
-            for _ in range(3):
-                sstep(0)
-            s_ms, _ = timed(sstep, 10)
-            _, skern = timed(sstep, 5, kernels=True)
-            s_med = statistics.median(s_ms)
-            sbytes, sflops = kernel_algorithmic("prefill", dict(sw, n=sn), 1)
-            bound = ridge_bound(sbytes, sflops, pk)
-            entry = {"F": TA.taylor_attn_num_features(sw["d_k"], sn), "ms_per_step": round(s_med, 5),
-                     "Mtok_s": round(sw["B"] * sw["N"] / (s_med * 1e-3) / 1e6, 3),
-                     "algorithmic_bytes": sbytes, "algorithmic_flops": sflops,
-                     "kernels_ms": {k_: round(t / c, 5) for k_, (c, t) in skern.items()}}
-            if bound == "hbm":
-                a = sbytes / (s_med * 1e-3) / 1e9
-                entry["roofline"] = {"bound": "hbm", "scope": "whole step", "achieved": round(a, 2),
-                                     "peak": hbm_peak, "unit": "GB/s", "frac": round(a / hbm_peak, 4)}
-            else:
-                a = sflops / (s_med * 1e-3) / 1e12
-                entry["roofline"] = {"bound": "tensor", "scope": "whole step", "achieved": round(a, 3),
-                                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                                     "frac": round(a / pk["bf16_tflops"], 4)}
-            res[str(sn)] = entry
-            del sst
-        sweep[arm] = res
-        del sq, sk, sv, sout
-    errs.check("order_sweep")
-
-    # ---- large-head prefill (F = 2,145): the contraction-bound configuration
-    lw = LARGE
-    lB, lH, lN, ld, ldv, ln = lw["B"], lw["H"], lw["N"], lw["d_k"], lw["d_v"], lw["n"]
-    lF = TA.taylor_attn_num_features(ld, ln)
-    lq, lk = unit_dev(g, (lB, lH, lN, ld)), unit_dev(g, (lB, lH, lN, ld))
-    lv = torch.randn((lB, lH, lN, ldv), device=dev, generator=g).to(torch.bfloat16)
-    lout = torch.empty((lB, lH, lN, ldv), dtype=torch.float32, device=dev)
-    lst = torch.empty((lB, lH, TA.taylor_attn_state_stride(ld, ldv, ln)), dtype=torch.float32, device=dev)
-
-    def lstep(i=0):
-        TA.taylor_attn_prefill(lq, lk, lv, ln, lw["tau"], out=lout, state_out=lst)
-
-    for _ in range(3):
-        lstep()
-    torch.cuda.synchronize()
-    l_steps_ms, _ = timed(lstep, 10)
-    l_ms = statistics.median(l_steps_ms)
-    _, lkern = timed(lstep, 5, kernels=True)
-    errs.check("large_head_prefill")
-    l_tokens = lB * lH * lN
-    l_alg = l_tokens * 4 * lF * (ldv + 1)                      # state update + read-out, 2 F Dv each
-    lk_name, _, lk_ms = dominant(lkern)
-    # the dominant kernel's algorithmic work: the read-out contraction of every
-    # query past the first group, 2 F Dv per head-token
-    l_dom_alg = l_tokens * 2 * lF * (ldv + 1)
-    del lq, lk, lv, lout, lst
-
     # ---- end to end through the public call with pinned host buffers
     qp, kp, vp = qh.pin_memory(), kh.pin_memory(), vh.pin_memory()
     outp = torch.empty(out.shape, dtype=torch.float32).pin_memory()
@@ -505,12 +308,216 @@ def run_ours(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = out.numel() * 4 + st.numel() * 4
 
+    g = torch.Generator(device=dev)  # device-side inputs of the later blocks
+    g.manual_seed(rank)
+    if "decode" in blocks:
+        # ---- decode: states of 65,536-token random prefixes built by the library
+        dw = DECODE
+        dB, dH = dw["B"], dw["H"]
+        dstride = TA.taylor_attn_state_stride(dw["d_k"], dw["d_v"], dw["n"])
+        dstate = torch.zeros((dB, dH, dstride), dtype=torch.float32, device=dev)
+        seg = 4096
+        tmp_state = torch.empty_like(dstate)
+        for s0 in range(0, dw["prefix"], seg):
+            pq_ = unit_dev(g, (dB, dH, seg, dw["d_k"]))
+            pk_ = unit_dev(g, (dB, dH, seg, dw["d_k"]))
+            pv_ = torch.randn((dB, dH, seg, dw["d_v"]), device=dev, generator=g).to(torch.bfloat16)
+            po = torch.empty((dB, dH, seg, dw["d_v"]), dtype=torch.float32, device=dev)
+            TA.taylor_attn_prefill(pq_, pk_, pv_, dw["n"], dw["tau"], out=po, state_out=tmp_state)
+            TA.taylor_attn_state_merge(dstate, tmp_state, dw["d_k"], dw["d_v"], dw["n"], out=dstate)
+            del pq_, pk_, pv_, po
+        del tmp_state
+        errs.check("decode_prefix")
+        dsteps = max(args.steps, 24)
+        toks = [synth.decode_tokens(dB, dH, dw["d_k"], dw["d_v"], s, seed=rank) for s in range(dsteps)]
+        toks = [(a.to(dev), b.to(dev), c.to(dev)) for a, b, c in toks]
+        dout = torch.empty((dB, dH, dw["d_v"]), dtype=torch.float32, device=dev)
+        # six independent batches of 1,024 carried states (245 MB > L2): step s
+        # updates batch s % 6, so its states were last touched six steps earlier
+        dstates = [dstate] + [dstate.clone() for _ in range(DECODE_BUFFERS - 1)]
+
+        def dec(i):
+            TA.taylor_attn_decode(*toks[i], dstates[i % DECODE_BUFFERS], dw["n"], dw["tau"], out=dout)
+
+        for s in range(max(args.warmup, 3) + DECODE_BUFFERS):
+            dec(s % dsteps)
+        torch.cuda.synchronize()
+        # steady state: back to back, one pair of events around the whole run
+        # (its device time over the steps), then per-launch events in a second run
+        e0, e1 = ev_pair()
+        e0.record(stream)
+        for s in range(dsteps):
+            dec(s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dec_us = e0.elapsed_time(e1) * 1e3 / dsteps
+        _, dkern = timed(dec, dsteps, flushed=False, kernels=True)
+        dk_name, _, dk_ms = dominant(dkern)
+        dec_kernel_us = dk_ms * 1e3
+        # one step after an L2 flush (cold reads, write-back after the kernel), context
+        dflush_ms, _ = timed(dec, dsteps, flushed=True)
+        # warm L2: the same batch of states step after step (it fits in L2), context
+        e0.record(stream)
+        for s in range(dsteps):
+            TA.taylor_attn_decode(*toks[s], dstate, dw["n"], dw["tau"], out=dout)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dec_warm_us = e0.elapsed_time(e1) * 1e3 / dsteps
+        errs.check("decode")
+        dec_us_max = allmax(dec_us, world, dev)
+        dbytes, dflops = kernel_algorithmic("decode", dw, 1)
+
+        # ---- the mean-centred softmax expansion (order 2) on the same carried
+        # states: same state traffic, a three-way read-out; timed like decode
+        def cen(i):
+            TA.taylor_attn_centred_decode(*toks[i], dstates[i % DECODE_BUFFERS], 2, dw["tau"], out=dout)
+
+        for s in range(DECODE_BUFFERS + 3):
+            cen(s)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for s in range(dsteps):
+            cen(s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        cen_us = e0.elapsed_time(e1) * 1e3 / dsteps
+        _, ckern = timed(cen, dsteps, flushed=False, kernels=True)
+        ck_name, _, ck_ms = dominant(ckern)
+        cen_kernel_us = ck_ms * 1e3
+        errs.check("centred_decode")
+
+    if "centred_prefill" in blocks:
+        # ---- the mean-centred expansion's prefill (order 2) on the main workload's inputs
+        cout = torch.empty_like(out)
+        cst = torch.empty_like(st)
+
+        def cstep(i=0):
+            TA.taylor_attn_centred_prefill(q, k, v, 2, tau, out=cout, state_out=cst)
+
+        for _ in range(3):
+            flush_l2()
+            cstep()
+        cp_ms, _ = timed(cstep, 10)
+        _, cpkern = timed(cstep, 5, kernels=True)
+        errs.check("centred_prefill")
+        cp_med = statistics.median(cp_ms)
+        cp_name, _, cp_dom_ms = dominant(cpkern)
+        del cout, cst
+
+    if "decode" in blocks:
+        # ---- batched multi-token decode: T new tokens per head per call, in place
+        multi = {}
+        for T in (4, 16):
+            mtoks = [(unit_dev(g, (dB, dH, T, dw["d_k"])), unit_dev(g, (dB, dH, T, dw["d_k"])),
+                      torch.randn((dB, dH, T, dw["d_v"]), device=dev, generator=g).to(torch.bfloat16))
+                     for _ in range(dsteps)]
+            mout = torch.empty((dB, dH, T, dw["d_v"]), dtype=torch.float32, device=dev)
+
+            def mdec(i):
+                sb = dstates[i % DECODE_BUFFERS]
+                TA.taylor_attn_prefill_from_state(*mtoks[i], sb, dw["n"], dw["tau"], out=mout, state_out=sb)
+
+            for s_ in range(DECODE_BUFFERS + 3):
+                mdec(s_)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for s_ in range(dsteps):
+                mdec(s_)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            m_us = e0.elapsed_time(e1) * 1e3 / dsteps
+            _, mk = timed(mdec, dsteps, flushed=False, kernels=True)
+            mk_name, _, mk_ms = dominant(mk)
+            mk_us = mk_ms * 1e3
+            Fd = TA.taylor_attn_num_features(dw["d_k"], dw["n"])
+            m_bytes = dB * dH * (2 * Fd * (dw["d_v"] + 1) * 4 + T * ((2 * dw["d_k"] + dw["d_v"]) * 2 + dw["d_v"] * 4))
+            multi[str(T)] = {"us_per_call": round(m_us, 3), "kernel": mk_name, "kernel_us": round(mk_us, 3),
+                             "Mtok_s": round(dB * dH * T / (m_us * 1e-6) / 1e6, 2),
+                             "hbm_frac": round(m_bytes / (mk_us * 1e-6) / 1e9 / hbm_peak, 4),
+                             "algorithmic_bytes_per_launch": m_bytes}
+            del mtoks, mout
+        errs.check("multi_token_decode")
+        del dstates
+
+    if "sweep" in blocks:
+        # ---- order sweep: n = 1..5 at B1 H8 N8192 d_k16 d_v64, q, k unit-normalised
+        # and (second arm) q, k ~ N(0, 4) as drawn
+        sw = SWEEP
+        sweep = {}
+        for arm, normalised in (("normalised", True), ("unnormalised_var4", False)):
+            sq, sk, sv = synth.qkv(sw["B"], sw["H"], sw["N"], sw["d_k"], sw["d_v"], seed=rank, dtype="bf16",
+                                   normalise=normalised, qk_var=1.0 if normalised else 4.0)
+            sq, sk, sv = sq.to(dev), sk.to(dev), sv.to(dev)
+            sout = torch.empty((sw["B"], sw["H"], sw["N"], sw["d_v"]), dtype=torch.float32, device=dev)
+            res = {}
+            for sn in sw["orders"]:
+                sst = torch.empty((sw["B"], sw["H"], TA.taylor_attn_state_stride(sw["d_k"], sw["d_v"], sn)),
+                                  dtype=torch.float32, device=dev)
+
+                def sstep(i, sn=sn, sst=sst):
+                    TA.taylor_attn_prefill(sq, sk, sv, sn, sw["tau"], out=sout, state_out=sst)
+
+                for _ in range(3):
+                    sstep(0)
+                s_ms, _ = timed(sstep, 10)
+                _, skern = timed(sstep, 5, kernels=True)
+                s_med = statistics.median(s_ms)
+                sbytes, sflops = kernel_algorithmic("prefill", dict(sw, n=sn), 1)
+                bound = ridge_bound(sbytes, sflops, pk)
+                entry = {"F": TA.taylor_attn_num_features(sw["d_k"], sn), "ms_per_step": round(s_med, 5),
+                         "Mtok_s": round(sw["B"] * sw["N"] / (s_med * 1e-3) / 1e6, 3),
+                         "algorithmic_bytes": sbytes, "algorithmic_flops": sflops,
+                         "kernels_ms": {k_: round(t / c, 5) for k_, (c, t) in skern.items()}}
+                if bound == "hbm":
+                    a = sbytes / (s_med * 1e-3) / 1e9
+                    entry["roofline"] = {"bound": "hbm", "scope": "whole step", "achieved": round(a, 2),
+                                         "peak": hbm_peak, "unit": "GB/s", "frac": round(a / hbm_peak, 4)}
+                else:
+                    a = sflops / (s_med * 1e-3) / 1e12
+                    entry["roofline"] = {"bound": "tensor", "scope": "whole step", "achieved": round(a, 3),
+                                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                         "frac": round(a / pk["bf16_tflops"], 4)}
+                res[str(sn)] = entry
+                del sst
+            sweep[arm] = res
+            del sq, sk, sv, sout
+        errs.check("order_sweep")
+
+    if "large" in blocks:
+        # ---- large-head prefill (F = 2,145): the contraction-bound configuration
+        lw = LARGE
+        lB, lH, lN, ld, ldv, ln = lw["B"], lw["H"], lw["N"], lw["d_k"], lw["d_v"], lw["n"]
+        lF = TA.taylor_attn_num_features(ld, ln)
+        lq, lk = unit_dev(g, (lB, lH, lN, ld)), unit_dev(g, (lB, lH, lN, ld))
+        lv = torch.randn((lB, lH, lN, ldv), device=dev, generator=g).to(torch.bfloat16)
+        lout = torch.empty((lB, lH, lN, ldv), dtype=torch.float32, device=dev)
+        lst = torch.empty((lB, lH, TA.taylor_attn_state_stride(ld, ldv, ln)), dtype=torch.float32, device=dev)
+
+        def lstep(i=0):
+            TA.taylor_attn_prefill(lq, lk, lv, ln, lw["tau"], out=lout, state_out=lst)
+
+        for _ in range(3):
+            lstep()
+        torch.cuda.synchronize()
+        l_steps_ms, _ = timed(lstep, 10)
+        l_ms = statistics.median(l_steps_ms)
+        _, lkern = timed(lstep, 5, kernels=True)
+        errs.check("large_head_prefill")
+        l_tokens = lB * lH * lN
+        l_alg = l_tokens * 4 * lF * (ldv + 1)                      # state update + read-out, 2 F Dv each
+        lk_name, _, lk_ms = dominant(lkern)
+        # the dominant kernel's algorithmic work: the read-out contraction of every
+        # query past the first group, 2 F Dv per head-token
+        l_dom_alg = l_tokens * 2 * lF * (ldv + 1)
+        del lq, lk, lv, lout, lst
+
     clk = clocks.stop()
 
     cpu = cpu_dec = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_leg(target_s=args.cpu_seconds)
-        cpu_dec = cpu_oracle_decode_leg(target_s=min(args.cpu_seconds, 8.0))
+        if "decode" in blocks:
+            cpu_dec = cpu_oracle_decode_leg(target_s=min(args.cpu_seconds, 8.0))
 
     if rank == 0:
         line = {
@@ -548,7 +555,15 @@ def run_ours(args, world, rank, local):
             },
             "kernels": {k_: {"launches": c, "total_ms": round(t, 4)} for k_, (c, t) in kern.items()},
             "ms_per_step_with_kernel_events": round(statistics.mean(step_ms_k), 5),
-            "decode": {
+            "e2e": {"value": round(world * tokens / (e2e_ms * 1e-3) / 1e6, 3), "unit": "Mtok/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "wall_s_timed_region": round(t_wall, 4),
+        }
+        if "decode" in blocks:
+            line["decode"] = {
                 "workload": "decode: B=64 H=16 d_k=16 d_v=64 n=3, states of 65,536-token random prefixes, "
                             "one token per head per step; steps back to back over 6 independent batches of "
                             "states (6 x 40.8 MB > L2), so each step reads its states from HBM and the "
@@ -569,8 +584,9 @@ def run_ours(args, world, rank, local):
                                              "updated states are written back after the launch, so it holds the "
                                              "state reads only; in the back-to-back timing above each launch "
                                              "also carries earlier launches' write-backs"},
-            },
-            "centred_decode": {
+            }
+        if "decode" in blocks:
+            line["centred_decode"] = {
                 "workload": "mean-centred softmax expansion, order 2, one token per head per step on the decode "
                             "workload's carried n=3 states (B=64 H=16 d_k=16 d_v=64), timed like decode",
                 "kernel": ck_name,
@@ -581,8 +597,9 @@ def run_ours(args, world, rank, local):
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(dbytes / (cen_kernel_us * 1e-6) / 1e9 / hbm_peak, 4),
                              "algorithmic_bytes_per_launch": dbytes, "traffic": None},
-            },
-            "centred_prefill": {
+            }
+        if "centred_prefill" in blocks:
+            line["centred_prefill"] = {
                 "workload": "mean-centred softmax expansion, order 2, causal prefill of the main workload's inputs "
                             "(B=1 H=8 N=4096 d_k=16 d_v=64, bf16 in, fp32 out + n=3 state), L2 flushed before each "
                             "step, median of 10 steps",
@@ -595,20 +612,23 @@ def run_ours(args, world, rank, local):
                              "algorithmic_bytes_per_step": byts,
                              "note": "same inputs, outputs and state as the main prefill; the three per-degree "
                                      "read-outs are fp32 CUDA-core work"},
-            },
-            "multi_token_decode": {
+            }
+        if "decode" in blocks:
+            line["multi_token_decode"] = {
                 "workload": "B=64 H=16 d_k=16 d_v=64 n=3, T new tokens per head per call against the carried "
                             "states (taylor_attn_prefill_from_state in place), timed like decode",
                 "by_tokens_per_call": multi,
-            },
-            "order_sweep": {
+            }
+        if "sweep" in blocks:
+            line["order_sweep"] = {
                 "workload": "causal prefill B=1 H=8 N=8192 d_k=16 d_v=64 tau=2, n = 1..5 (F = 1, 17, 153, 969, "
                             "4845), bf16 q/k/v, fp32 out+state, L2 flushed before each step, median of 10 "
                             "steps; q, k unit-normalised, and q, k ~ N(0, 4) as drawn",
                 "bound_rule": "tensor when algorithmic flops / bytes exceeds the measured peaks' ridge point",
                 "by_arm_and_order": sweep,
-            },
-            "large_head_prefill": {
+            }
+        if "large" in blocks:
+            line["large_head_prefill"] = {
                 "workload": "causal prefill B=4 H=16 N=32768 d_k=64 d_v=64 n=3 (F=2145) tau=2, bf16 q/k/v, "
                             "fp32 out+state, L2 flushed before each step, median of 10 steps",
                 "ms_per_step": round(l_ms, 4),
@@ -624,16 +644,10 @@ def run_ours(args, world, rank, local):
                              "algorithmic_flops_per_launch": l_dom_alg, "traffic": None,
                              "note": "read-out contraction 2 F Dv per head-token; hi/lo bf16 operands execute "
                                      "3x these MMA flops, padded to 80 columns"},
-            },
-            "e2e": {"value": round(world * tokens / (e2e_ms * 1e-3) / 1e6, 3), "unit": "Mtok/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": round(e2e_ms, 4)},
-            "gpu_launches": launches,
-            "clocks": clk,
-            "wall_s_timed_region": round(t_wall, 4),
-        }
+            }
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if cpu_dec is not None and "decode" in blocks:
             line["decode"]["cpu_baseline"] = cpu_dec
         if errs.seen:
             line["device_errors"] = errs.seen
@@ -762,6 +776,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--blocks", default="all",
+                    help="all (default), or a comma list of decode, centred_prefill, sweep, large: the main "
+                         "prefill (with its end-to-end figure) always runs; a shorter list serves profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
