@@ -52,9 +52,16 @@ def _deps(src: str, headers) -> list:
     if os.path.exists(dep):
         with open(dep) as f:
             text = f.read().replace("\\\n", " ")
-        files = [t for t in text.split(":", 1)[-1].split() if os.path.exists(t)]
+        files = []
+        for t in text.split(":", 1)[-1].split():
+            # nvcc writes paths as it was given them: relative ones are taken
+            # against the package and the repository roots
+            for c in ([t] if os.path.isabs(t) else [os.path.join(HERE, t), os.path.join(ROOT, t), t]):
+                if os.path.exists(c):
+                    files.append(c)
+                    break
         if files:
-            return files + [os.path.abspath(__file__)]
+            return [src, *files, os.path.abspath(__file__)]
     return [src, *headers]
 
 

@@ -17,10 +17,12 @@
 // and storing the new row straight to HBM.  HBM traffic is one state read and
 // one state write per call, as for a single decode step.
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "feature_table.cuh"
 #include "internal.h"
+#include "phase.cuh"
 #include "ptx.cuh"
 
 namespace ta {
@@ -33,6 +35,7 @@ constexpr int kTMax = 16;
 constexpr uint32_t kWaitPolls = 1u << 22;
 constexpr size_t kMaxDyn = 226 * 1024;  // the 227 KB per-block limit, less static shared memory
 constexpr int kMaxDevices = 64;
+constexpr int kTcMinTokens = 8;  // the tensor-core multi-token kernel takes T > 8
 
 struct MultiLayout {
     uint32_t s, pk, pq, xq, xk, vv, p, red, zr, bytes;
@@ -223,26 +226,35 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
 // ---------------------------------------------------------------- persistent form
 // The same step for d_v = 64 and features of degree <= 2 (F <= 256), many
 // heads: one CTA per SM walks the heads blockIdx.x, blockIdx.x + gridDim.x,
-// ...  A producer thread keeps one buffer per consumer warpgroup full (a bulk
-// copy of the head's state and of its T tokens' q, k, v rows, completing on
-// the buffer's mbarrier); three consumer warpgroups take the heads in turn.
-// A warpgroup evaluates phi(k_j), phi(q_i) and the block's pairwise weights
-// into its own area, walks the state rows once (read-out of all T tokens from
-// the old row, the T rank-one updates, the new row stored straight to HBM),
-// hands the buffer back, then reduces the read-out and writes the outputs.
-// Head i of a CTA uses buffer i mod 3 and is consumed by warpgroup i mod 3, so
-// each buffer has one consumer that takes its phases in order.
-constexpr int kWGm = 3;
+// ...  Two warpgroups take the heads in turn, each with its own ring buffer
+// (the head's state and its T tokens' q, k, v rows, brought in by bulk
+// copies that complete on the buffer's mbarrier): warpgroup g takes heads g,
+// g + 2, ... of the CTA and, once it has read a head's buffer, itself issues
+// the copies of its next head into it, so a copy is in flight while it
+// finishes the head before.  A warpgroup evaluates phi(k_j), phi(q_j) and
+// the block's pairwise weights into its own area, walks the state rows once
+// (read-out of all T tokens from the old row, the T rank-one updates, the new
+// row stored straight to HBM), hands the buffer on, then reduces the
+// read-out and writes the outputs.  In the walk each thread keeps its column
+// group of the T v rows in registers, so a row costs one state load and the
+// row's read-out and update coefficients (broadcast within the row set) from
+// shared memory; two warpgroups and no other warp leave room for about 250
+// registers a thread.
+constexpr int kWGm = 2;
 constexpr int kWGmThreads = 128;
-constexpr int kThreadsWSm = kWGm * kWGmThreads + 32;
+constexpr int kThreadsWSm = kWGm * kWGmThreads;
 constexpr int kDVw = 64, kDV4w = 16;
 constexpr size_t kMaxDynWSm = 226 * 1024;
 
 struct MultiWsLayout {
-    uint32_t offq, offk, offv, buf;  // one ring buffer: state, then the q, k, v rows
-    uint32_t pk, pq, vf, p, zr, area; // one warpgroup area
+    uint32_t offq, offk, offv, buf;                  // one ring buffer: state, then the q, k, v rows
+    uint32_t pk, pq, vf, p, zr, xq, xk, area;        // one warpgroup area
+    uint32_t desc, bytes;                            // the feature table after the areas; the total
 };
 
+// Features per warpgroup walk; the q, k rows held as fp32 with one extra
+// slot of 1 (stride d + 1) so that degree 0 and 1 features read it as their
+// missing factors.
 __host__ __device__ inline MultiWsLayout multi_ws_layout(int T, int d, int F, uint32_t state_bytes, uint32_t esize) {
     auto al = [](uint32_t x) { return (x + 127u) & ~127u; };
     MultiWsLayout L;
@@ -252,16 +264,20 @@ __host__ __device__ inline MultiWsLayout multi_ws_layout(int T, int d, int F, ui
     L.offv = L.offk + al((uint32_t)(T * d) * esize);
     L.buf = L.offv + al((uint32_t)(T * kDVw) * esize);
     // pk, pq [F][Tp]; after the row walk the same space holds the column
-    // partials [4 warps][T][16 float4]
+    // partials [8 row sets][T][64]
     const uint32_t coeff = al((uint32_t)F * Tp * 4);
-    const uint32_t partials = al((uint32_t)(4 * T * kDVw) * 4);
+    const uint32_t partials = al((uint32_t)(8 * T * kDVw) * 4);
     L.pk = 0;
     L.pq = coeff;
     const uint32_t span = 2 * coeff > partials ? 2 * coeff : partials;
     L.vf = span;                                   // v rows as fp32 [T][64]
     L.p = L.vf + al((uint32_t)(T * kDVw) * 4);    // pairwise weights [16][16]
-    L.zr = L.p + al((uint32_t)(kTMax * kTMax) * 4);
-    L.area = L.zr + al((uint32_t)(4 * kTMax) * 4);
+    L.zr = L.p + al((uint32_t)(kTMax * kTMax) * 4);  // normaliser partials [8][16]
+    L.xq = L.zr + al((uint32_t)(8 * kTMax) * 4);
+    L.xk = L.xq + al((uint32_t)(T * (d + 1)) * 4);
+    L.area = L.xk + al((uint32_t)(T * (d + 1)) * 4);
+    L.desc = kWGm * (L.buf + L.area);              // [F] float4: {a | c << 8, w, w tau^m/m!, 0}
+    L.bytes = L.desc + al((uint32_t)F * 16);
     return L;
 }
 
@@ -275,15 +291,14 @@ decode_multi_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, con
                        const float* state_in, float* state_out, float* __restrict__ out, int BH, int T, int d, int n,
                        float tau, int F, int64_t stride, uint32_t bytes, unsigned int* __restrict__ err) {
     extern __shared__ __align__(128) unsigned char dsm[];
-    __shared__ __align__(8) uint64_t full[kWGm], empty[kWGm];
+    __shared__ __align__(8) uint64_t full[kWGm];
     __shared__ int s_bad, s_fail[kWGm];
     const MultiWsLayout L = multi_ws_layout(T, d, F, bytes, (uint32_t)sizeof(Tin));
     unsigned char* areas = dsm + (size_t)kWGm * L.buf;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int nheads = BH > (int)blockIdx.x ? (BH - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const uint32_t tok_in = (uint32_t)(T * d) * (uint32_t)sizeof(Tin), tok_v = (uint32_t)(T * kDVw) * (uint32_t)sizeof(Tin);
-    const int producer = kWGm * kWGmThreads;
-    auto issue = [&](int i) {
+    auto issue = [&](int i) {  // head i of this CTA into buffer i mod 2
         const int b = i % kWGm;
         const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
         unsigned char* buf = dsm + (size_t)b * L.buf;
@@ -295,92 +310,116 @@ decode_multi_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, con
     };
 
     // launched with programmatic dependent launch: every memory access of the
-    // grid follows the producer's wait on the previous grid
+    // grid follows thread 0's wait on the previous grid (directly, or through
+    // the barrier below)
     ptx::pdl_launch_dependents();
-    int issued = 0;
-    if (tid == producer) {
-        for (int i = 0; i < kWGm; ++i) {
-            ptx::mbar_init(&full[i], 1);
-            ptx::mbar_init(&empty[i], 1);
-        }
+    if (tid == 0) {
+        for (int i = 0; i < kWGm; ++i) ptx::mbar_init(&full[i], 1);
         ptx::fence_mbar_init();
         ptx::pdl_wait_primary();
-        for (; issued < kWGm && issued < nheads; ++issued) issue(issued);
+        for (int i = 0; i < kWGm && i < nheads; ++i) issue(i);
+        s_bad = 0;
     }
-    if (tid == 0) s_bad = 0;
     if (tid < kWGm) s_fail[tid] = 0;
+    // the feature table: degree, indices (d for a missing factor, which
+    // reads the slot of 1 after each q, k row) and both weights
+    float4* desc = reinterpret_cast<float4*>(dsm + L.desc);
+    for (int f = tid; f < F; f += kThreadsWSm) {
+        int m, a, c2;
+        float w;
+        feature_deg2(d, f, m, a, c2, w);
+        if (m < 2) c2 = d;
+        if (m < 1) a = d;
+        desc[f] = make_float4(__int_as_float(a | (c2 << 8)), w, w * query_coeff(m, tau), 0.f);
+    }
     __syncthreads();
 
-    if (warp == producer / 32) {
-        if (lane == 0) {
-            int i = issued;
-            for (; i < nheads; ++i) {
-                const int b = i % kWGm;
-                if (!ptx::mbar_wait_or_abort(&empty[b], ((i / kWGm) - 1) & 1, kWaitPolls, &s_bad)) break;
-                issue(i);
-            }
-            for (int j = (i > kWGm ? i - kWGm : 0); j < i; ++j)
-                ptx::mbar_wait(&full[j % kWGm], (j / kWGm) & 1, kWaitPolls);
-        }
-    } else {
-        const int wg = warp >> 2, t = tid & (kWGmThreads - 1), wl = warp & 3;
+    {
+        const int wg = warp >> 2, t = tid & (kWGmThreads - 1);
         unsigned char* area = areas + (size_t)wg * L.area;
         float* pk = reinterpret_cast<float*>(area + L.pk);
         float* pq = reinterpret_cast<float*>(area + L.pq);
-        float4* red = reinterpret_cast<float4*>(area + L.pk);  // after the row walk
+        float* red = reinterpret_cast<float*>(area + L.pk);  // after the row walk
         float* vf = reinterpret_cast<float*>(area + L.vf);
         float* P = reinterpret_cast<float*>(area + L.p);
         float* zr = reinterpret_cast<float*>(area + L.zr);
-        const int Tp = (T + 3) & ~3;
+        float* qf = reinterpret_cast<float*>(area + L.xq);
+        float* kf = reinterpret_cast<float*>(area + L.xk);
+        const int Tp = (T + 3) & ~3, Tp4 = Tp / 4;
+        const int zi = t & 15, zs = t >> 4;  // the z column: token zi, row set zs
         const int cg = t % kDV4w, rs = t / kDV4w;  // 8 row sets
+        TA_PHASE_VARS(p_t, p_wait = 0, p_prep = 0, p_walk = 0, p_z = 0, p_red = 0, p_out = 0);
         for (int i = wg; i < nheads; i += kWGm) {
             const int b = i % kWGm;  // == wg: only this warpgroup consumes buffer b
+            TA_PHASE_T0(p_t);
             if (!ptx::mbar_wait_or_abort(&full[b], (i / kWGm) & 1, kWaitPolls, &s_bad)) s_fail[wg] = 1;
             wgm_sync(wg);
-            if (s_fail[wg]) break;  // the same value for all 128 threads: set only before this barrier
+            TA_PHASE_ACC(p_wait, p_t);
+            TA_PHASE_T0(p_t);
+            if (s_fail[wg]) {  // the same value for all 128 threads: set only before this barrier
+                // the copies may still land: wait for them (bounded) before the block can exit
+                if (t == 0) ptx::mbar_wait(&full[b], (i / kWGm) & 1, kWaitPolls);
+                break;
+            }
             const int64_t h = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
             const unsigned char* buf = dsm + (size_t)b * L.buf;
             const Tin* xq = reinterpret_cast<const Tin*>(buf + L.offq);
             const Tin* xk = reinterpret_cast<const Tin*>(buf + L.offk);
             const Tin* xv = reinterpret_cast<const Tin*>(buf + L.offv);
-            // phi(k_j) and (tau^m/m!) phi(q_i), feature-major with the tokens contiguous
-            for (int e = t; e < F * Tp; e += kWGmThreads) {
-                const int f = e / Tp, j = e % Tp;
-                int m, a, c2;
-                float w;
-                feature_deg2(d, f, m, a, c2, w);
-                float pkv = 0.f, pqv = 0.f;
-                if (j < T) {
-                    const float ka = m >= 1 ? to_float(xk[j * d + a]) : 1.f, kb = m >= 2 ? to_float(xk[j * d + c2]) : 1.f;
-                    const float qa = m >= 1 ? to_float(xq[j * d + a]) : 1.f, qb = m >= 2 ? to_float(xq[j * d + c2]) : 1.f;
-                    pkv = w * ka * kb;
-                    pqv = w * query_coeff(m, tau) * qa * qb;
-                }
-                pk[e] = pkv;
-                pq[e] = pqv;
+            // q, k rows to fp32 with the slot of 1; v rows to fp32
+            for (int e = t; e < T * (d + 1); e += kWGmThreads) {
+                const int j = e / (d + 1), c = e - j * (d + 1);
+                qf[e] = c < d ? to_float(xq[j * d + c]) : 1.f;
+                kf[e] = c < d ? to_float(xk[j * d + c]) : 1.f;
             }
             for (int e = t; e < T * kDVw; e += kWGmThreads) vf[e] = to_float(xv[e]);
+            wgm_sync(wg);
+            // phi(k_j) and (tau^m/m!) phi(q_j), feature-major with the tokens
+            // contiguous; one thread per feature and four tokens
+            for (int u = t; u < F * Tp4; u += kWGmThreads) {
+                const int f = Tp4 == 4 ? u >> 2 : Tp4 == 2 ? u >> 1 : Tp4 == 1 ? u : u / 3;
+                const int j0 = 4 * (u - f * Tp4);
+                const float4 fd = desc[f];
+                const int a = __float_as_int(fd.x) & 255, c2 = __float_as_int(fd.x) >> 8;
+                float kk[4], qq[4];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = j0 + jj < T ? j0 + jj : 0;  // padded tokens get coefficient 0 below
+                    const float* kr = kf + j * (d + 1);
+                    const float* qr = qf + j * (d + 1);
+                    const float live = j0 + jj < T ? 1.f : 0.f;
+                    kk[jj] = live * fd.y * kr[a] * kr[c2];
+                    qq[jj] = live * fd.z * qr[a] * qr[c2];
+                }
+                reinterpret_cast<float4*>(pk)[u] = make_float4(kk[0], kk[1], kk[2], kk[3]);
+                reinterpret_cast<float4*>(pq)[u] = make_float4(qq[0], qq[1], qq[2], qq[3]);
+            }
             // the block's own causal part: K(tau q_i.k_j) for j <= i
             for (int e = t; e < kTMax * kTMax; e += kWGmThreads) {
                 const int ii = e / kTMax, j = e % kTMax;
                 float w = 0.f;
                 if (ii < T && j <= ii) {
                     float dot = 0.f;
-                    for (int c = 0; c < d; ++c) dot = fmaf(to_float(xq[ii * d + c]), to_float(xk[j * d + c]), dot);
+                    for (int c = 0; c < d; ++c) dot = fmaf(qf[ii * (d + 1) + c], kf[j * (d + 1) + c], dot);
                     w = taylor_kernel(tau * dot, n);
                 }
                 P[e] = w;
             }
             wgm_sync(wg);
+            TA_PHASE_ACC(p_prep, p_t);
+            TA_PHASE_T0(p_t);
 
             // one walk over the state rows: read-out of every token from the
             // old row, then the T rank-one updates, the new row to HBM
             const float4* S4 = reinterpret_cast<const float4*>(buf);
             float4* G4 = state_out ? reinterpret_cast<float4*>(state_out + h * stride) : nullptr;
             const float4* V4 = reinterpret_cast<const float4*>(vf);
-            float4 y[kTMax];
+            float4 y[kTMax], vr[kTMax];
 #pragma unroll
-            for (int ii = 0; ii < kTMax; ++ii) y[ii] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int ii = 0; ii < kTMax; ++ii) {
+                y[ii] = make_float4(0.f, 0.f, 0.f, 0.f);
+                vr[ii] = ii < T ? V4[ii * kDV4w + cg] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
             for (int r = rs; r < F; r += kWGmThreads / kDV4w) {
                 float4 s = S4[r * kDV4w + cg];
                 const float4* cq = reinterpret_cast<const float4*>(pq + r * Tp);
@@ -402,69 +441,64 @@ decode_multi_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, con
                 if (G4) {
 #pragma unroll
                     for (int j4 = 0; j4 < kTMax / 4; ++j4) {
-                        if (4 * j4 < T) {  // padded tokens have coefficient 0 and zero v rows are not read
+                        if (4 * j4 < T) {  // padded tokens have coefficient 0 and v rows of zeros
                             const float4 a = ck[j4];
                             const float aa[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
-                                if (4 * j4 + u < T) {
-                                    const float4 vv4 = V4[(4 * j4 + u) * kDV4w + cg];
-                                    s.x = fmaf(aa[u], vv4.x, s.x);
-                                    s.y = fmaf(aa[u], vv4.y, s.y);
-                                    s.z = fmaf(aa[u], vv4.z, s.z);
-                                    s.w = fmaf(aa[u], vv4.w, s.w);
-                                }
+                                s.x = fmaf(aa[u], vr[4 * j4 + u].x, s.x);
+                                s.y = fmaf(aa[u], vr[4 * j4 + u].y, s.y);
+                                s.z = fmaf(aa[u], vr[4 * j4 + u].z, s.z);
+                                s.w = fmaf(aa[u], vr[4 * j4 + u].w, s.w);
                             }
                         }
                     }
                     G4[r * kDV4w + cg] = s;
                 }
             }
-            float yz[kTMax];
-#pragma unroll
-            for (int ii = 0; ii < kTMax; ++ii) yz[ii] = 0.f;
+            TA_PHASE_ACC(p_walk, p_t);
+            TA_PHASE_T0(p_t);
+            // the z column: token zi's read-out over row set zs, and the
+            // update of each row's normaliser
             const float* Z = reinterpret_cast<const float*>(buf) + (int64_t)F * kDVw;
             float* GZ = state_out ? state_out + h * stride + (int64_t)F * kDVw : nullptr;
-            for (int f = t; f < F; f += kWGmThreads) {
-                float z = Z[f];
-#pragma unroll
-                for (int ii = 0; ii < kTMax; ++ii)
-                    if (ii < T) yz[ii] = fmaf(pq[f * Tp + ii], z, yz[ii]);
-                if (GZ) {
-#pragma unroll
-                    for (int j = 0; j < kTMax; ++j)
-                        if (j < T) z += pk[f * Tp + j];
+            float yz = 0.f;
+            if (zi < T)
+                for (int f = zs; f < F; f += kWGmThreads / 16) yz = fmaf(pq[f * Tp + zi], Z[f], yz);
+            if (GZ) {
+                for (int f = t; f < F; f += kWGmThreads) {
+                    float z = Z[f];
+                    const float4* c4 = reinterpret_cast<const float4*>(pk + f * Tp);
+                    for (int j4 = 0; j4 < Tp4; ++j4) {
+                        const float4 c = c4[j4];
+                        z += (c.x + c.y) + (c.z + c.w);
+                    }
                     GZ[f] = z;
                 }
-            }
-            if (G4)  // the state's padding stays zero
+                // the state's padding stays zero
                 for (int64_t e = (int64_t)F * (kDVw + 1) + t; e < stride; e += kWGmThreads) state_out[h * stride + e] = 0.f;
+            }
             // the buffer and the coefficients have been read: hand the buffer
             // back, and reuse the coefficient space for the column partials
             ptx::fence_proxy_async_smem();
             wgm_sync(wg);
-            if (t == 0) ptx::mbar_arrive(&empty[b]);
+            TA_PHASE_ACC(p_z, p_t);
+            TA_PHASE_T0(p_t);
+            if (t == 0 && i + kWGm < nheads) issue(i + kWGm);
+            float4* red4 = reinterpret_cast<float4*>(red);
 #pragma unroll
-            for (int ii = 0; ii < kTMax; ++ii) {
-                if (ii < T) {
-                    y[ii].x += __shfl_xor_sync(0xffffffffu, y[ii].x, 16);
-                    y[ii].y += __shfl_xor_sync(0xffffffffu, y[ii].y, 16);
-                    y[ii].z += __shfl_xor_sync(0xffffffffu, y[ii].z, 16);
-                    y[ii].w += __shfl_xor_sync(0xffffffffu, y[ii].w, 16);
-                    if (lane < kDV4w) red[(wl * T + ii) * kDV4w + lane] = y[ii];
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) yz[ii] += __shfl_xor_sync(0xffffffffu, yz[ii], o);
-                    if (lane == 0) zr[wl * kTMax + ii] = yz[ii];
-                }
-            }
+            for (int ii = 0; ii < kTMax; ++ii)
+                if (ii < T) red4[(rs * T + ii) * kDV4w + cg] = y[ii];
+            zr[zs * kTMax + zi] = yz;
             wgm_sync(wg);
+            TA_PHASE_ACC(p_red, p_t);
+            TA_PHASE_T0(p_t);
             for (int e = t; e < T * kDVw; e += kWGmThreads) {
                 const int ii = e / kDVw, c = e % kDVw;
                 float acc = 0.f, den = 0.f;
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const float4 r4 = red[(w * T + ii) * kDV4w + (c >> 2)];
-                    acc += (c & 3) == 0 ? r4.x : (c & 3) == 1 ? r4.y : (c & 3) == 2 ? r4.z : r4.w;
+                for (int w = 0; w < kWGmThreads / kDV4w; ++w) {
+                    acc += red[(w * T + ii) * kDVw + c];
                     den += zr[w * kTMax + ii];
                 }
                 for (int j = 0; j <= ii; ++j) {
@@ -475,9 +509,17 @@ decode_multi_ws_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, con
                 out[(h * T + ii) * kDVw + c] = acc / den;
             }
             wgm_sync(wg);  // the area is rewritten only after every thread is done with it
+            TA_PHASE_ACC(p_out, p_t);
         }
+        TA_PHASE_PUT(0, 1 + 6 * wg, t == 0, p_wait);
+        TA_PHASE_PUT(0, 2 + 6 * wg, t == 0, p_prep);
+        TA_PHASE_PUT(0, 3 + 6 * wg, t == 0, p_walk);
+        TA_PHASE_PUT(0, 4 + 6 * wg, t == 0, p_z);
+        TA_PHASE_PUT(0, 5 + 6 * wg, t == 0, p_red);
+        TA_PHASE_PUT(0, 6 + 6 * wg, t == 0, p_out);
     }
     __syncthreads();
+    TA_PHASE(0, 0, tid == 0);
     if (tid == 0 && s_bad) atomicOr(err, kErrDecodeLoad);
 }
 
@@ -509,7 +551,7 @@ cudaError_t launch_multi_ws(const Tin* q, const Tin* k, const Tin* v, const floa
                             float* out, int BH, int T, int d, int dv, int n, float tau, int64_t F, int64_t stride,
                             cudaStream_t stream) {
     // features of degree <= 2 only (always the case for F <= 256 at the supported d_k)
-    if (dv != kDVw || F > 256 || n > 3 || ((int64_t)T * d * sizeof(Tin)) % 16 != 0) return cudaErrorNotSupported;
+    if (dv != kDVw || F > 256 || n > 3 || d > 32 || ((int64_t)T * d * sizeof(Tin)) % 16 != 0) return cudaErrorNotSupported;
     static std::once_flag once[kMaxDevices];
     static cudaError_t set_err[kMaxDevices];
     static int num_sms[kMaxDevices];
@@ -526,7 +568,7 @@ cudaError_t launch_multi_ws(const Tin* q, const Tin* k, const Tin* v, const floa
     if (BH < 2 * num_sms[dev]) return cudaErrorNotSupported;  // few heads: one CTA per head is as good
     const uint32_t bytes = (uint32_t)((F * (dv + 1) * 4 + 15) / 16 * 16);
     const MultiWsLayout L = multi_ws_layout(T, d, (int)F, bytes, (uint32_t)sizeof(Tin));
-    const size_t dyn = (size_t)kWGm * (L.buf + L.area);
+    const size_t dyn = L.bytes;
     if (dyn > kMaxDynWSm) return cudaErrorNotSupported;
     unsigned int* err = device_error_word();
     if (!err) return cudaErrorNotSupported;
@@ -543,6 +585,16 @@ cudaError_t launch_decode_multi(const Tin* q, const Tin* k, const Tin* v, const 
                                 float* out, int BH, int T, int d, int dv, int n, float tau, int64_t F, int64_t stride,
                                 cudaStream_t stream) {
     if (T < 1 || T > kTMax || F > 1024) return cudaErrorNotSupported;
+    // Above 8 tokens per call the tensor-core kernel is the faster one on
+    // the decode workload (its cost is nearly flat in T; the CUDA-core row
+    // walk grows with T): 35.6 / 35.7 us at T = 8, 53.6 / 37.1 us at T = 16.
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+        if (T > kTcMinTokens) {
+            const cudaError_t et = launch_decode_multi_tc(q, k, v, state_in, state_out, out, BH, T, d, dv, n, tau,
+                                                          F, stride, stream);
+            if (et != cudaErrorNotSupported) return et;
+        }
+    }
     {
         const cudaError_t ew = launch_multi_ws(q, k, v, state_in, state_out, out, BH, T, d, dv, n, tau, F, stride,
                                                stream);

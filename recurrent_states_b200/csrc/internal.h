@@ -67,6 +67,12 @@ cudaError_t launch_decode_multi(const Tin* q, const Tin* k, const Tin* v, const 
                                 float* out, int BH, int T, int d, int dv, int n, float tau, int64_t F, int64_t stride,
                                 cudaStream_t stream);
 
+// The same on the tensor cores for bf16 inputs, d_v 64, at most 160 features
+// of degree <= 2 and many heads; cudaErrorNotSupported outside that range.
+cudaError_t launch_decode_multi_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                   const float* state_in, float* state_out, float* out, int BH, int T, int d, int dv,
+                                   int n, float tau, int64_t F, int64_t stride, cudaStream_t stream);
+
 cudaError_t launch_merge(const float* a, const float* b, float* out, int64_t count, int num_sms,
                          cudaStream_t stream);
 

@@ -16,4 +16,11 @@ namespace ta {
 cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                               uint32_t box0, uint32_t box1, uint32_t swizzle_bytes);
 
+// An fp32 tensor [d2][d1][d0] (d0 innermost, contiguous) with row strides
+// stride1 and stride2 bytes (multiples of 16), boxes of box0 x box1 x 1
+// elements, and the swizzle as above (box0 * 4 bytes at most that many).
+cudaError_t make_tmap_f32_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                             uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1,
+                             uint32_t swizzle_bytes);
+
 }  // namespace ta

@@ -401,10 +401,10 @@ def test_multi_token_decode_blocks_follow_the_recursion(dtype):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("d,n", [(16, 3), (16, 2), (32, 2)])
 def test_multi_token_decode_many_heads(dtype, d, n):
-    """320 heads (enough for the persistent multi-token kernel, whose three
-    warpgroups take heads in turn): blocks of 16, 1, 7 and 4 new tokens fed in
-    place after a 200-token prefill, against the oracle's recursion (outputs
-    of every block, final state)."""
+    """320 heads (enough for the persistent multi-token kernels: the
+    tensor-core one for bf16 inputs, the CUDA-core one for fp32): blocks of
+    16, 1, 7 and 4 new tokens fed in place after a 200-token prefill, against
+    the oracle's recursion (outputs of every block, final state)."""
     B, H, dv, tau = 32, 10, 64, 2.0 if n == 3 else 1.0
     blocks = [16, 1, 7, 4]
     prefix = 200
@@ -422,6 +422,38 @@ def test_multi_token_decode_many_heads(dtype, d, n):
         assert row_scaled_max_err(f64(o), ref_out[:, :, t0:t0 + T]) <= TOL[dtype], T
         t0 += T
     assert state_block_errors(st, ref_st, d, dv, n) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("d,n,T,inplace", [(8, 3, 16, True), (16, 1, 9, True), (16, 3, 10, False),
+                                           (16, 3, 13, False), (24, 2, 12, True), (16, 3, 6, False)])
+def test_multi_token_decode_tensor_core_shapes(d, n, T, inplace):
+    """The tensor-core multi-token kernel (more than 8 tokens per call) over
+    its range (F = 45, 1, 153, 153, 25; ragged T; in place and into a separate
+    state; outputs only when no state is asked for), and one case of the
+    CUDA-core kernel that takes fewer tokens: one block of T tokens after a
+    150-token prefill on 300 heads, against the oracle's recursion."""
+    B, H, dv, tau, prefix = 30, 10, 64, 2.0, 150
+    q, k, v = synth.qkv(B, H, prefix + T, d, dv, seed=7 * d + n + T, dtype="bf16")
+    sl = lambda t, a, b: t[:, :, a:b].contiguous().to(DEV)  # noqa: E731
+    _, st = TA.taylor_attn_prefill(sl(q, 0, prefix), sl(k, 0, prefix), sl(v, 0, prefix), n, tau, state_out=True)
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    before = st.clone()
+    target = st if inplace else torch.full_like(st, float("nan"))
+    o, _ = TA.taylor_attn_prefill_from_state(sl(q, prefix, prefix + T), sl(k, prefix, prefix + T),
+                                             sl(v, prefix, prefix + T), st, n, tau, state_out=target)
+    torch.cuda.synchronize()
+    assert row_scaled_max_err(f64(o), ref_out[:, :, prefix:]) <= TOL["bf16"]
+    assert state_block_errors(target, ref_st, d, dv, n) <= TOL["bf16"]
+    if not inplace:
+        assert torch.equal(st, before)
+        # the state's padding is written as zeros
+        stride = TA.taylor_attn_state_stride(d, dv, n)
+        F = TA.taylor_attn_num_features(d, n)
+        assert torch.count_nonzero(target[..., F * (dv + 1):stride]) == 0
+    o2, _ = TA.taylor_attn_prefill_from_state(sl(q, prefix, prefix + T), sl(k, prefix, prefix + T),
+                                              sl(v, prefix, prefix + T), before, n, tau, state_out=None)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, o)
 
 
 def test_prefill_from_state_with_no_new_tokens_copies_the_state():
