@@ -61,7 +61,7 @@ constexpr int kNV = 80;        // columns of [V | 1 | 0 ...]
 constexpr int kFP = 160;       // features, padded
 constexpr int kGroups = kFP / 8;
 constexpr int kCompute = 256;
-constexpr int kThreadsF = kCompute + 32;
+constexpr int kThreadsF = kCompute + 64;  // + the TMA / MMA warp (8) and the publishing warp (9)
 constexpr int kMaxChunks = 36;  // chunks per head this kernel takes (the scan's gather fits the Phi_K space)
 constexpr uint32_t kWaitPolls = 1u << 24;
 constexpr uint32_t kFlagPolls = 1u << 24;
@@ -175,7 +175,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
     extern __shared__ uint8_t sm_raw[];
     uint8_t* sm = align1k(sm_raw);
     __shared__ __align__(8) uint64_t ld, phik_full, phik_free, t_done, t_free, sc_full, p_full, p_free, gath,
-        e_loaded[2], phiq_full[2], ro_done[2];
+        e_loaded[2], phiq_full[2], ro_done[2], t_staged;
     __shared__ uint32_t tslot;
     __shared__ int s_bad, s_e_issued[2], s_gath_issued;
     volatile int* bad = &s_bad;
@@ -212,6 +212,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         ptx::mbar_init(&p_full, kCompute);
         ptx::mbar_init(&p_free, 1);
         ptx::mbar_init(&gath, 1);
+        ptx::mbar_init(&t_staged, 1);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&e_loaded[i], 1);
             ptx::mbar_init(&phiq_full[i], kCompute);
@@ -329,6 +330,23 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             TA_PHASE(1, 4, true);
             if (!go) *bad = 1;
         }
+    } else if (warp == 9) {
+        if (lane == 0) {
+            // ------------------------------------------------ publishing the chunk states
+            // the staged T_x^T rows leave in one bulk store per chunk; once
+            // they have completed, the head's count of published chunks grows
+            if (waitb(&t_staged, 0, bad)) {
+                for (int x = 0; x < nch; ++x)
+                    ptx::bulk_s2g(A.TG + ((int64_t)bh * NC + c0 + x) * kXFloats, sPhi + (uint32_t)x * kXFloats * 4u,
+                                  (uint32_t)kXFloats * 4u);
+                ptx::bulk_commit();
+                ptx::bulk_wait_all();
+                fence_proxy_async_global();
+                __threadfence();
+                TA_PHASE(1, 9, true);
+                if (!*bad) red_release_add(tcount, (unsigned)nch);
+            }
+        }
     } else {
         // ---------------------------------------------------- CUDA-core roles
         const int row = (warp & 3) * 32 + lane, half = warp >> 2;
@@ -380,8 +398,9 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         }
         TA_PHASE(0, 2, tid == 0);
 
-        // publish the chunk states T_x^T (lane = v column, 160 feature
-        // columns) as [feature][column] rows in L2
+        // stage the chunk states T_x^T (lane = v column, 160 feature columns)
+        // as [feature][column] rows in the Phi_K space, which the state MMAs
+        // have finished reading; the publishing warp takes them to L2
         ok = ok && waitb(&t_done, 0, bad);
         TA_PHASE(0, 3, tid == 0);
         if (ok) {
@@ -389,7 +408,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             if ((warp & 3) < 3) {
                 const int vc = row;  // lanes 0..64: v columns 0..63 and z
                 for (int x = 0; x < nch; ++x) {
-                    float* tg = A.TG + ((int64_t)bh * NC + c0 + x) * kXFloats;
+                    float* tg = reinterpret_cast<float*>(sPhi) + x * kXFloats;
 #pragma unroll
                     for (int p = 0; p < 5; ++p) {
                         float r[16];
@@ -417,9 +436,12 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                 *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
             }
         }
+        // the staged rows go to the publishing warp's bulk stores; the zeroed
+        // rows are read by this CTA's own bulk loads of E
+        ptx::fence_proxy_async_smem();
         __threadfence();
         compute_sync();
-        if (tid == 0 && ok && !*bad) red_release_add(tcount, (unsigned)nch);
+        if (tid == 0 && ok && !*bad) ptx::mbar_arrive(&t_staged);
         TA_PHASE(0, 4, tid == 0);
 
         // P = poly(tau q.k) of query `row` against keys [64 half, 64 half + 64),
