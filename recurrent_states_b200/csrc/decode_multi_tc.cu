@@ -127,21 +127,33 @@ struct MultiTcArgs {
     float tau;
 };
 
-// The update epilogue of feature row f (this thread's TMEM lane in the tile
-// at column tcol): reads the row's fp32 state into s, writes S'[f] = S[f] +
-// D_U[f][0..63] back in its place and z'_f = z_f + D_U[f][64] to HBM.
-__device__ __forceinline__ void update_row(unsigned char* buf, const float* Z, float* G, int F, int f, bool live,
-                                           uint32_t tcol, float (&s)[64]) {
-    if (live) {
+// Feature row f of the state from its two fp32 slab rows (zeros if not live).
+__device__ __forceinline__ void load_row(const unsigned char* buf, int f, bool live, float (&s)[64]) {
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
-            const float4 x = *reinterpret_cast<const float4*>(buf + (p >> 3) * kHalfS + sw128(f, p & 7));
-            s[4 * p] = x.x; s[4 * p + 1] = x.y; s[4 * p + 2] = x.z; s[4 * p + 3] = x.w;
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) s[e] = 0.f;
+    for (int p = 0; p < 16; ++p) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (live) x = *reinterpret_cast<const float4*>(buf + (p >> 3) * kHalfS + sw128(f, p & 7));
+        s[4 * p] = x.x; s[4 * p + 1] = x.y; s[4 * p + 2] = x.z; s[4 * p + 3] = x.w;
     }
+}
+
+// The bf16 hi and lo images of row f over its slab rows (slab 0 takes hi,
+// slab 1 lo); the thread has read the whole row before.
+__device__ __forceinline__ void image_row(unsigned char* buf, int f, const float (&s)[64]) {
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+        uint4 hi, lo;
+        split8(s + 8 * b, hi, lo);
+        *reinterpret_cast<uint4*>(buf + sw128(f, b)) = hi;
+        *reinterpret_cast<uint4*>(buf + kHalfS + sw128(f, b)) = lo;
+    }
+}
+
+// The update epilogue of feature row f (this thread's TMEM lane in the tile
+// at column tcol), once the read-out has finished with the images:
+// S'[f] = S[f] + D_U[f][0..63] into the slab rows, z'_f = z_f + D_U[f][64] to HBM.
+__device__ __forceinline__ void update_row(unsigned char* buf, const float* Z, float* G, int F, int f, bool live,
+                                           uint32_t tcol, const float (&s)[64]) {
     float dl[64];
     tmem_ld32(tcol, *reinterpret_cast<float(*)[32]>(dl));
     tmem_ld32(tcol + 32, *reinterpret_cast<float(*)[32]>(dl + 32));
@@ -154,17 +166,6 @@ __device__ __forceinline__ void update_row(unsigned char* buf, const float* Z, f
             make_float4(s[4 * p] + dl[4 * p], s[4 * p + 1] + dl[4 * p + 1], s[4 * p + 2] + dl[4 * p + 2],
                         s[4 * p + 3] + dl[4 * p + 3]);
     if (G) G[(int64_t)F * kDVt + f] = Z[f] + dz;
-}
-
-// The bf16 hi (part 0) or lo (part 1) image of the old row f over its slab
-// row (slab 0 for hi, slab 1 for lo).
-__device__ __forceinline__ void image_row(unsigned char* buf, int f, const float (&s)[64], int part) {
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-        uint4 hi, lo;
-        split8(s + 8 * b, hi, lo);
-        *reinterpret_cast<uint4*>(buf + part * kHalfS + sw128(f, b)) = part ? lo : hi;
-    }
 }
 
 __global__ void __launch_bounds__(kThreadsT, 1)
@@ -389,104 +390,96 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tms, const __grid_con
         TA_PHASE_ACC(p_prep, p_t);
         TA_PHASE_T0(p_t);
 
-        // (3) the update on the tensor cores: D_U[f][c'] = sum_j phi_f(k_j) [v_j | 1][c']
-        if (t == 0) {
-            fence_after_sync();
-            const uint64_t bv = smem_desc_sw(v2, 2048, 1024, kSwizzle128);
-            const uint32_t iu = idesc_bf16(128, 80, 0, 1);
-            for (int x = 0; x < ntiles; ++x) {
-                mma_bf16(tU + 80u * (uint32_t)x, smem_desc(pkh + 4096 * x, 128, 256), bv, iu, 0);
-                mma_bf16(tU + 80u * (uint32_t)x, smem_desc(pkl + 4096 * x, 128, 256), bv, iu, 1);
-            }
-            mma_commit(&mma_u[wg]);
-        }
-        // (4) meanwhile: the normalisers (their reciprocals)
-        float* G = A.state_out ? A.state_out + h * A.stride : nullptr;
-        {
-            const int i2 = t >> 3, g0 = t & 7;  // 8 threads a token
-            float s = g0 == 0 ? ps[i2] : 0.f;
-            for (int g = g0; g < 4 * nks; g += 8) s += zp[g * kTT + i2];
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
-            s += __shfl_xor_sync(0xffffffffu, s, 4);
-            if (g0 == 0) rden[i2] = 1.f / s;
-        }
-        if (G)  // the state's padding stays zero
-            for (int64_t e = (int64_t)F * (kDVt + 1) + t; e < A.stride; e += kWGtThreads) G[e] = 0.f;
-        // (5) the update epilogue, feature row by row (TMEM lane = row)
-        if (!ptx::mbar_wait(&mma_u[wg], (uint32_t)kh & 1u, kPolls)) s_bad = 1;
-        fence_after_sync();
+        // (3) every thread takes its feature row(s) of the state into registers
+        // and writes their bf16 images in place for the read-out
         float s0[64], s1[64];
         const int f0 = 32 * wl + lane, f1 = 128 + lane;
         const bool two = ntiles > 1 && wl == 0;  // tile 1 (features 128..255) lies in lanes 0..31 too
-        update_row(buf, Z, G, F, f0, f0 < F, tU + lane_off, s0);
-        if (two) update_row(buf, Z, G, F, f1, f1 < F, tU + 80u + lane_off, s1);
-        ptx::fence_proxy_async_smem();  // S' in the slabs, for the tensor stores
-        fence_before_sync();
-        wg_sync(wg);
-        if (t == 0 && G) {  // slab 0, then slab 1, in bulk groups of their own
-            ptx::tma_store_3d(&tmo, 0, 0, (int)h, buf);
-            ptx::bulk_commit();
-            ptx::tma_store_3d(&tmo, 32, 0, (int)h, buf + kHalfS);
-            ptx::bulk_commit();
-            ptx::bulk_wait_read<1>();
-        }
-        wg_sync(wg);  // slab 0 has been read: S_hi may replace it while slab 1 is stored
-        if (f0 < F) image_row(buf, f0, s0, 0);
-        if (two && f1 < F) image_row(buf, f1, s1, 0);
-        if (t == 0 && G) ptx::bulk_wait_read<0>();
-        wg_sync(wg);
-        if (f0 < F) image_row(buf, f0, s0, 1);
-        if (two && f1 < F) image_row(buf, f1, s1, 1);
+        load_row(buf, f0, f0 < F, s0);
+        if (two) load_row(buf, f1, f1 < F, s1);
+        if (f0 < F) image_row(buf, f0, s0);
+        if (two && f1 < F) image_row(buf, f1, s1);
         ptx::fence_proxy_async_smem();
         fence_before_sync();
         wg_sync(wg);
         TA_PHASE_ACC(p_upd, p_t);
         TA_PHASE_T0(p_t);
 
-        // (6) the read-out on the tensor cores; rows 64..127 of D_R are not used
+        // (4) both contractions on the tensor cores
         if (t == 0) {
             fence_after_sync();
+            // the update, D_U[f][c'] = sum_j phi_f(k_j) [v_j | 1][c']
+            const uint64_t bv = smem_desc_sw(v2, 2048, 1024, kSwizzle128);
+            const uint32_t iu = idesc_bf16(128, 80, 0, 1);
+            for (int x = 0; x < ntiles; ++x) {
+                mma_bf16(tU + 80u * (uint32_t)x, smem_desc(pkh + 4096 * x, 128, 256), bv, iu, 0);
+                mma_bf16(tU + 80u * (uint32_t)x, smem_desc(pkl + 4096 * x, 128, 256), bv, iu, 1);
+            }
+            // the read-out, A = [S_hi | S_lo] (the second 64-row atom, through
+            // LBO, is the lo image) against [Q_hi | Q_lo]; step s starts 2048 (A)
+            // and 1024 (B) bytes on, added to the address fields (>> 4)
             const uint32_t ir = idesc_bf16(128, 2 * kTT, 1, 0);
-            // A = [S_hi | S_lo]: the second 64-row atom (LBO) is the lo image.
-            // Step s starts 2048 (A) and 1024 (B) bytes on, added to the
-            // address field (>> 4) of the step-0 descriptors.
             const uint64_t as = smem_desc_sw(buf, kHalfS, 1024, kSwizzle128);
             const uint64_t bq = smem_desc(pq, 512, 128);
             for (int s = 0; s < nks; ++s)
                 mma_bf16(tR, as + (uint64_t)(128 * s), bq + (uint64_t)(64 * s), ir, s > 0 ? 1u : 0u);
             // A = [V | 0] (the zero atom as rows 64..127) against [P_hi | P_lo]
             mma_bf16(tR, smem_desc_sw(v2, 4096, 1024, kSwizzle128), smem_desc(pt, 512, 128), ir, 1);
-            mma_commit(&mma_r[wg]);
+            mma_commit(&mma_u[wg]);
         }
-        if (!ptx::mbar_wait(&mma_r[wg], (uint32_t)kh & 1u, kPolls)) s_bad = 1;
+        // meanwhile: the normalisers (their reciprocals), the state's padding
+        float* G = A.state_out ? A.state_out + h * A.stride : nullptr;
+        {
+            const int i2 = t >> 3, g0 = t & 7;  // 8 threads a token
+            float sm = g0 == 0 ? ps[i2] : 0.f;
+            for (int g = g0; g < 4 * nks; g += 8) sm += zp[g * kTT + i2];
+            sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+            sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+            sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+            if (g0 == 0) rden[i2] = 1.f / sm;
+        }
+        if (G)
+            for (int64_t e = (int64_t)F * (kDVt + 1) + t; e < A.stride; e += kWGtThreads) G[e] = 0.f;
+        if (!ptx::mbar_wait(&mma_u[wg], (uint32_t)kh & 1u, kPolls)) s_bad = 1;
         fence_after_sync();
         TA_PHASE_ACC(p_conv, p_t);
         TA_PHASE_T0(p_t);
-        {
-            // lane c' = 32 wl + lane: column c' % 64, hi rows (c' < 64) or lo rows;
-            // D columns 0..15 against the hi query features, 16..31 the lo
-            float y[32];
-            tmem_ld32(tR + lane_off, y);
-            tmem_ld_wait();
-            const int col = (32 * wl + lane) & 63;
-            if (wl >= 2) {
+
+        // (5) the update epilogue, feature row by row (TMEM lane = row): the
+        // images are no longer read, S' replaces them; the read-out's lo rows
+        update_row(buf, Z, G, F, f0, f0 < F, tU + lane_off, s0);
+        if (two) update_row(buf, Z, G, F, f1, f1 < F, tU + 80u + lane_off, s1);
+        float y[32];
+        tmem_ld32(tR + lane_off, y);
+        tmem_ld_wait();
+        const int col = (32 * wl + lane) & 63;
+        if (wl >= 2) {
 #pragma unroll
-                for (int i2 = 0; i2 < kTT; ++i2) rlo[i2 * kDVt + col] = y[i2] + y[kTT + i2];
-            }
-            wg_sync(wg);
-            if (wl < 2) {
+            for (int i2 = 0; i2 < kTT; ++i2) rlo[i2 * kDVt + col] = y[i2] + y[kTT + i2];
+        }
+        ptx::fence_proxy_async_smem();  // S' in the slabs, for the tensor stores
+        fence_before_sync();
+        wg_sync(wg);
+        if (t == 0 && G) {
+            ptx::tma_store_3d(&tmo, 0, 0, (int)h, buf);
+            ptx::tma_store_3d(&tmo, 32, 0, (int)h, buf + kHalfS);
+            ptx::bulk_commit();
+        }
+        // (6) the outputs: hi rows (warps 0, 1) plus the lo rows, times 1 / den
+        if (wl < 2) {
 #pragma unroll
-                for (int i2 = 0; i2 < kTT; ++i2)
-                    if (i2 < T) A.out[(h * T + i2) * kDVt + col] = (y[i2] + y[kTT + i2] + rlo[i2 * kDVt + col]) * rden[i2];
-            }
+            for (int i2 = 0; i2 < kTT; ++i2)
+                if (i2 < T) A.out[(h * T + i2) * kDVt + col] = (y[i2] + y[kTT + i2] + rlo[i2 * kDVt + col]) * rden[i2];
         }
         fence_before_sync();
         wg_sync(wg);
         TA_PHASE_ACC(p_ro, p_t);
-        // (7) the buffer is free (its last readers, the read-out MMAs, have
-        // completed): bring in head i + 3
-        if (t == 0 && i + kNBuf < nheads) issue(i + kNBuf);
+        // (7) once the tensor stores have read the slabs the buffer is free:
+        // bring in head i + 3
+        if (t == 0 && i + kNBuf < nheads) {
+            ptx::bulk_wait_read_all();
+            issue(i + kNBuf);
+        }
     }
     TA_PHASE_PUT(0, 1 + 5 * wg, tid == 128 * wg, p_wait);
     TA_PHASE_PUT(0, 2 + 5 * wg, tid == 128 * wg, p_prep);
