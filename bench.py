@@ -49,6 +49,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # decode is timed back to back over this many independent batches of states
 # (6 x 40.8 MB > the 126 MB L2)
 DECODE_BUFFERS = 6
+DECODE_GRAPH_STEPS = 100  # dependent decode steps per CUDA-graph replay
 
 
 # DRAM bytes of one decode_ws_kernel launch on the decode workload, from an ncu
@@ -363,6 +364,24 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
         dec_warm_us = e0.elapsed_time(e1) * 1e3 / dsteps
+        # 100 dependent steps over the six batches captured in one CUDA graph
+        # and replayed (no host work between launches), total / 100
+        dec_graph_us = None
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for s in range(DECODE_GRAPH_STEPS):
+                    dec(s % dsteps)
+            graph.replay()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            dec_graph_us = e0.elapsed_time(e1) * 1e3 / DECODE_GRAPH_STEPS
+            del graph
+        except RuntimeError as ex:  # capture refused: report the reason, keep the rest of the line
+            dec_graph_us = f"unavailable: {str(ex).splitlines()[0][:120]}"
         errs.check("decode")
         dec_us_max = allmax(dec_us, world, dev)
         dbytes, dflops = kernel_algorithmic("decode", dw, 1)
@@ -572,6 +591,8 @@ def run_ours(args, world, rank, local):
                 "kernel_us": round(dec_kernel_us, 3),
                 "us_per_step_l2_flushed": round(statistics.mean(dflush_ms) * 1e3, 3),
                 "us_per_step_warm_l2": round(dec_warm_us, 3),
+                "us_per_step_cuda_graph": round(dec_graph_us, 3) if isinstance(dec_graph_us, float) else dec_graph_us,
+                "cuda_graph_steps": DECODE_GRAPH_STEPS,
                 "roofline": {"bound": "hbm", "kernel": dk_name,
                              "achieved": round(dbytes / (dec_kernel_us * 1e-6) / 1e9, 2),
                              "peak": hbm_peak, "unit": "GB/s",

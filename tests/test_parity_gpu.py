@@ -456,6 +456,33 @@ def test_multi_token_decode_tensor_core_shapes(d, n, T, inplace):
     assert torch.equal(o2, o)
 
 
+def test_decode_steps_replay_in_a_cuda_graph():
+    """Four dependent decode steps on 320 heads (the persistent kernel, launched
+    with programmatic dependent launch) captured in one CUDA graph: a replay
+    gives exactly what the same steps give launched one by one."""
+    B, H, d, dv, n, tau, steps = 32, 10, 16, 64, 3, 2.0, 4
+    stride = TA.taylor_attn_state_stride(d, dv, n)
+    g = torch.Generator().manual_seed(5)
+    st0 = (torch.randn((B, H, stride), generator=g) * 0.01).to(DEV)
+    toks = [tuple(x[:, :, 0].contiguous().to(DEV) for x in synth.qkv(B, H, 1, d, dv, seed=40 + s)) for s in range(steps)]
+    eager_st = st0.clone()
+    eager = [TA.taylor_attn_decode(*toks[s], eager_st, n, tau) for s in range(steps)]
+    graph_st = st0.clone()
+    outs = [torch.empty((B, H, dv), device=DEV) for _ in range(steps)]
+    TA.taylor_attn_decode(*toks[0], st0.clone(), n, tau)  # the first call sets the kernel up outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for s in range(steps):
+            TA.taylor_attn_decode(*toks[s], graph_st, n, tau, out=outs[s])
+    graph_st.copy_(st0)
+    graph.replay()
+    torch.cuda.synchronize()
+    for s in range(steps):
+        assert torch.equal(outs[s], eager[s]), s
+    assert torch.equal(graph_st, eager_st)
+
+
 def test_prefill_from_state_with_no_new_tokens_copies_the_state():
     st = torch.randn((1, 2, TA.taylor_attn_state_stride(16, 64, 3)), device=DEV)
     e = torch.empty((1, 2, 0, 16), dtype=torch.bfloat16, device=DEV)
