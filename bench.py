@@ -52,11 +52,21 @@ DECODE_BUFFERS = 6
 DECODE_GRAPH_STEPS = 100  # dependent decode steps per CUDA-graph replay
 
 
-# DRAM bytes of one decode_ws_kernel launch on the decode workload, from an ncu
-# capture (read 40,991,488 + write 38,400); ncu empties the caches before the
-# launch and the updated states are written back only after the kernel ends,
-# so this is the read half.  To be retaken whenever the kernel changes.
-DECODE_WS_DRAM_BYTES = 41_029_888
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a
+# kernel on its bench workload, from ncu captures of the kernels as committed
+# (python -m recurrent_states_b200.profile_cases <case>).  ncu empties the
+# caches before the launch, and what a kernel writes stays in L2 until after it
+# ends, so these are mostly reads.  To be retaken whenever a kernel changes.
+DRAM_BYTES = {
+    "tc_fused_prefill_kernel": 6_399_488 + 7_168,       # main prefill
+    "decode_ws_kernel": 40_992_000 + 15_104,            # decode step
+    "centred_decode_ws_kernel": 41_000_704 + 22_528,    # centred decode step
+    "decode_multi_ws_kernel": 41_591_296 + 98_048,      # 4 tokens per call
+    "decode_multi_tc_kernel": 43_977_472 + 243_712,     # 16 tokens per call
+    # one eighth of the large head (8 of 64 heads) scaled by 8: traffic grows with the heads
+    "tcf_out_kernel": 8 * (184_387_328 + 50_061_568),
+}
+DECODE_WS_DRAM_BYTES = DRAM_BYTES["decode_ws_kernel"]
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -453,7 +463,7 @@ def run_ours(args, world, rank, local):
             multi[str(T)] = {"us_per_call": round(m_us, 3), "kernel": mk_name, "kernel_us": round(mk_us, 3),
                              "Mtok_s": round(dB * dH * T / (m_us * 1e-6) / 1e6, 2),
                              "hbm_frac": round(m_bytes / (mk_us * 1e-6) / 1e9 / hbm_peak, 4),
-                             "algorithmic_bytes_per_launch": m_bytes}
+                             "algorithmic_bytes_per_launch": m_bytes, "traffic": DRAM_BYTES.get(mk_name)}
             del mtoks, mout
         errs.check("multi_token_decode")
         del dstates
@@ -564,7 +574,7 @@ def run_ours(args, world, rank, local):
                 "bound": "hbm", "kernel": dom_name,
                 "achieved": round(achieved, 2), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "peak_source": pk["_source"] + " (hbm_gbs, burst copy)",
-                "traffic": None,
+                "traffic": DRAM_BYTES.get(dom_name),
                 "algorithmic_bytes_per_launch": byts,
                 "kernel_us_per_launch": round(per_launch_ms * 1e3, 3),
                 "timing": "CUDA events around each launch of the kernel, second pass of K steps",
@@ -617,7 +627,7 @@ def run_ours(args, world, rank, local):
                              "achieved": round(dbytes / (cen_kernel_us * 1e-6) / 1e9, 2),
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(dbytes / (cen_kernel_us * 1e-6) / 1e9 / hbm_peak, 4),
-                             "algorithmic_bytes_per_launch": dbytes, "traffic": None},
+                             "algorithmic_bytes_per_launch": dbytes, "traffic": DRAM_BYTES.get(ck_name)},
             }
         if "centred_prefill" in blocks:
             line["centred_prefill"] = {
@@ -662,7 +672,8 @@ def run_ours(args, world, rank, local):
                              "achieved": round(l_dom_alg / (lk_ms * 1e-3) / 1e12, 3),
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": round(l_dom_alg / (lk_ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
-                             "algorithmic_flops_per_launch": l_dom_alg, "traffic": None,
+                             "algorithmic_flops_per_launch": l_dom_alg, "traffic": DRAM_BYTES.get(lk_name),
+                             "traffic_note": "one eighth of the workload captured, scaled by heads",
                              "note": "read-out contraction 2 F Dv per head-token; hi/lo bf16 operands execute "
                                      "3x these MMA flops, padded to 80 columns"},
             }
