@@ -4,22 +4,26 @@
 //
 // Method (arXiv 2610.20637, abstract): the causal history is the state
 // S = sum_j phi(k_j) [v_j | 1]^T, additive across chunks, so prefill is a
-// scan over chunk states.  CTA s of head h takes chunks NCH s .. NCH s + NCH - 1
-// (NCH = 1 or 2; x below is one of them):
+// scan over chunk states.  CTA s of head h takes chunks a = NCH s and, when
+// NCH = 2, b = a + 1:
 //   1. loads its q, k, v rows with TMA (swizzled operand layouts);
-//   2. forms each chunk state T_x^T = [V_x | 1 | 0]^T Phi_K,x on the tensor
-//      cores (TMEM) and publishes it to global memory (L2) with a flag;
-//   3. meanwhile forms the pairwise parts O_x = (poly(tau Q_x K_x^T) (.) mask) [V_x | 1];
-//   4. the scan: the CTA that owns 8-feature group g of head h waits for
-//      every chunk state of the head, gathers that group of all of them into
-//      shared memory with bulk copies, forms the exclusive prefixes
-//      E_c = state_in + sum_{c' < c} T_c' for every chunk c, and writes them,
-//      split into hi/lo bf16, straight in the byte layout of the read-out
-//      MMA's operand (and the total into state_out), then sets the group's
-//      flag;
-//   5. once every group flag of its head is set, the CTA pulls the operands
-//      E_x of its chunks with bulk copies, evaluates c (.) Phi_Q,x into TMEM
-//      and adds (c (.) Phi_Q,x) E_x to O_x; o = O[:, :64] / O[:, 64].
+//   2. forms its state T_s^T = sum_x [V_x | 1 | 0]^T Phi_K,x on the tensor
+//      cores (TMEM, both chunks into one accumulator) and publishes it to
+//      global memory (L2): staged in shared memory, one bulk store by the
+//      publishing warp, then the head's count of published states is raised;
+//   3. meanwhile forms the pairwise parts O_a = (poly(tau Q_a K_a^T) (.) mask) [V_a | 1],
+//      O_b likewise with chunk b's own keys, plus all of chunk a's keys
+//      (no mask): chunk b's view of chunk a is pairwise, not through a state;
+//   4. the scan: the CTA that owns feature rows [R s, R s + R) of head h
+//      (R = ceil(F / CTAs of the head)) waits for every state of the head,
+//      gathers those rows of all of them into shared memory with bulk
+//      copies, forms the exclusive prefixes E_s = state_in + sum_{s' < s} T_s'
+//      for every CTA s of the head, and writes them, split into hi/lo bf16,
+//      straight in the byte layout of the read-out MMA's operand (and the
+//      total into state_out), then raises the head's count of scanned rows;
+//   5. once that count reaches F, the CTA pulls its operand E_s with a bulk
+//      copy, evaluates c (.) Phi_Q,x into TMEM and adds (c (.) Phi_Q,x) E_s to
+//      O_x of both its chunks; o = O[:, :64] / O[:, 64].
 // The launch is cooperative, so all CTAs that wait on one another's flags are
 // resident together; every flag wait and every mbarrier wait is bounded, and
 // a wait that runs out sets a device error bit and skips the work that
@@ -89,10 +93,12 @@ constexpr uint32_t kLboE = kGroupBytes;             // K-group stride of E (MN-m
 static_assert(kEBytes <= 2 * kPhiBytes, "E of chunk b fits the Phi_K space");
 static_assert(kSmemF <= 232448, "shared memory");
 
-// TMEM (512 columns): chunk states T_a^T [0, 160), T_b^T [160, 320); later
-// the scores / P [0, 128); later Phi_Q,a [0, 160) (hi 80 | lo 80) and Phi_Q,b
-// [160, 320); O_a [320, 400), O_b [400, 480)
+// TMEM (512 columns): the CTA's state T^T [0, 160); later the scores / P of
+// the pairwise rounds, in two buffers [0, 128) and [160, 288) used in turn;
+// later Phi_Q,a [0, 160) (hi 80 | lo 80) and Phi_Q,b [160, 320); O_a [320, 400),
+// O_b [400, 480)
 constexpr uint32_t kTT = 0, kTO = 320;
+constexpr uint32_t kPBuf = 160;  // the second scores / P buffer (columns 160..287)
 
 __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, volatile int* bad) {
     return ptx::mbar_wait_or_abort(bar, parity, kWaitPolls, bad);
@@ -160,8 +166,8 @@ struct FusedArgs {
     float* out;
     const float* state_in;
     float* state_out;
-    float* TG;        // [BH][NC][160][68] published chunk states
-    uint8_t* EG;      // [BH][NC][kEBytes] read-out operands
+    float* TG;        // [BH][NS][160][68] published states, one per CTA (its chunks together)
+    uint8_t* EG;      // [BH][NS][kEBytes] read-out operands of the state before each CTA
     unsigned* flags;  // [BH] published chunk states, then [BH] finished feature groups (counters)
     int N, n, F, NC, NCH, ngroups, BH;
     float tau;
@@ -174,7 +180,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                         const __grid_constant__ CUtensorMap tmv, const FusedArgs A) {
     extern __shared__ uint8_t sm_raw[];
     uint8_t* sm = align1k(sm_raw);
-    __shared__ __align__(8) uint64_t ld, phik_full, phik_free, t_done, t_free, sc_full, p_full, p_free, gath,
+    __shared__ __align__(8) uint64_t ld, phik_full, phik_free, t_done, t_free, sc_full[2], p_full[2], p_free[2], gath,
         e_loaded[2], phiq_full[2], ro_done[2], t_staged;
     __shared__ uint32_t tslot;
     __shared__ int s_bad, s_e_issued[2], s_gath_issued;
@@ -186,6 +192,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
     const int n = A.n, F = A.F, NC = A.NC, NCH = A.NCH, ngroups = A.ngroups;
     const int c0 = seg * NCH;                                   // first chunk of this CTA
     const int nch = min(NCH, NC - c0);                          // its chunks (1 or 2)
+    const int nrounds = nch == 2 ? 3 : 1;                       // pairwise blocks: aa (, bb, ba)
     const int64_t t0 = (int64_t)c0 * kC;
     const int rem = A.N - (int)t0;
     const int nval0 = min(kC, rem), nval1 = max(0, min(kC, rem - kC));  // valid rows of chunks a, b
@@ -208,9 +215,11 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         ptx::mbar_init(&phik_free, 1);
         ptx::mbar_init(&t_done, 1);
         ptx::mbar_init(&t_free, kCompute);
-        ptx::mbar_init(&sc_full, 1);
-        ptx::mbar_init(&p_full, kCompute);
-        ptx::mbar_init(&p_free, 1);
+        for (int i = 0; i < 2; ++i) {  // one set per scores / P buffer
+            ptx::mbar_init(&sc_full[i], 1);
+            ptx::mbar_init(&p_full[i], kCompute);
+            ptx::mbar_init(&p_free[i], 1);
+        }
         ptx::mbar_init(&gath, 1);
         ptx::mbar_init(&t_staged, 1);
         for (int i = 0; i < 2; ++i) {
@@ -253,32 +262,38 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                 const uint8_t* atom = sV + (2 * x + (ks >> 2)) * kVAtom;
                 return smem_desc_sw(atom, (uint32_t)(sOnes - atom), 1024, kSwizzle128) + 128 * (ks & 3);
             };
+            // the CTA's state: both chunks into one accumulator
             auto state = [&](int x) {
                 const uint64_t ph = smem_desc(sPhi, kLboPhi, 128), pl = smem_desc(sPhi + kPhiBytes, kLboPhi, 128);
-                const uint32_t d = tb + kTT + 160 * x;
+                const uint32_t d = tb + kTT;
 #pragma unroll
                 for (int ks = 0; ks < kC / 16; ++ks) {
                     const uint64_t vd = vdesc(x, ks);
-                    mma_bf16(d, vd, ph + (2 * kLboPhi / 16) * ks, id_st, ks > 0 ? 1u : 0u);
+                    mma_bf16(d, vd, ph + (2 * kLboPhi / 16) * ks, id_st, (x > 0 || ks > 0) ? 1u : 0u);
                     mma_bf16(d, vd, pl + (2 * kLboPhi / 16) * ks, id_st, 1u);
                 }
             };
-            auto scores = [&](int x) {
-                const uint64_t qd = smem_desc_sw(sQ + x * kQBytes, 16, 256, kSwizzle32);
-                const uint64_t kd = smem_desc_sw(sK + x * kQBytes, 16, 256, kSwizzle32);
-                mma_bf16(tb + kTT, qd, kd, idesc_bf16(kC, kC, 0, 0), 0u);
-                mma_commit(&sc_full);
+            // round r: queries of chunk qx(r) against keys of chunk kx(r), in
+            // scores / P buffer r % 2 (TMEM columns 0..127 or 160..287)
+            auto qxr = [](int r) { return r == 0 ? 0 : 1; };
+            auto kxr = [](int r) { return r == 1 ? 1 : 0; };
+            auto scores = [&](int r) {
+                const uint64_t qd = smem_desc_sw(sQ + qxr(r) * kQBytes, 16, 256, kSwizzle32);
+                const uint64_t kd = smem_desc_sw(sK + kxr(r) * kQBytes, 16, 256, kSwizzle32);
+                mma_bf16(tb + kTT + kPBuf * (r & 1), qd, kd, idesc_bf16(kC, kC, 0, 0), 0u);
+                mma_commit(&sc_full[r & 1]);
             };
             // P of keys 16 ks .. 16 ks + 15: hi words at 32 (ks / 2) + 8 (ks % 2), lo 16 further
-            auto pv = [&](int x) {
+            auto pv = [&](int r) {
+                const int ox = qxr(r), vx = kxr(r);
 #pragma unroll
                 for (int ks = 0; ks < kC / 16; ++ks) {
-                    const uint32_t a = tb + kTT + 32 * (ks >> 1) + 8 * (ks & 1);
-                    const uint64_t vd = vdesc(x, ks);
-                    mma_bf16_ts(tb + kTO + 80 * x, a, vd, id80, ks > 0 ? 1u : 0u);
-                    mma_bf16_ts(tb + kTO + 80 * x, a + 16, vd, id80, 1u);
+                    const uint32_t a = tb + kTT + kPBuf * (r & 1) + 32 * (ks >> 1) + 8 * (ks & 1);
+                    const uint64_t vd = vdesc(vx, ks);
+                    mma_bf16_ts(tb + kTO + 80 * ox, a, vd, id80, (r == 2 || ks > 0) ? 1u : 0u);
+                    mma_bf16_ts(tb + kTO + 80 * ox, a + 16, vd, id80, 1u);
                 }
-                mma_commit(&p_free);
+                mma_commit(&p_free[r & 1]);
             };
             bool go = waitb(&ld, 0, bad);
             TA_PHASE(1, 1, true);
@@ -292,28 +307,36 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                 }
             }
             TA_PHASE(1, 2, true);
-            // the pairwise parts, into the columns the states have left
+            // the pairwise parts, into the columns the state has left: round 0
+            // chunk a against itself, round 1 chunk b against itself, round 2
+            // chunk b against all of chunk a (which its read-out then leaves out)
             go = go && waitb(&t_free, 0, bad);
-            for (int x = 0; x < nch && go; ++x) {
-                if (x > 0) go = waitb(&p_free, 0, bad);  // P of chunk a consumed
+            if (go) {
+                fence_after_sync();
+                for (int r = 0; r < nrounds && r < 2; ++r) scores(r);
+            }
+            for (int r = 0; r < nrounds && go; ++r) {
+                go = waitb(&p_full[r & 1], (r >> 1) & 1, bad);
                 if (go) {
                     fence_after_sync();
-                    scores(x);
+                    pv(r);
                 }
-                go = go && waitb(&p_full, x & 1, bad);
-                if (go) {
-                    fence_after_sync();
-                    pv(x);
+                if (go && r + 2 < nrounds) {  // its buffer again, once pv(r) has read P
+                    go = waitb(&p_free[r & 1], (r >> 1) & 1, bad);
+                    if (go) {
+                        fence_after_sync();
+                        scores(r + 2);
+                    }
                 }
             }
             TA_PHASE(1, 3, true);
-            // the read-outs through the carried states
+            // the read-outs through the state before the CTA (one operand for both chunks)
             for (int x = 0; x < nch; ++x) {
-                if (x > 0 || inter0) {
-                    go = go && waitb(&phiq_full[x], 0, bad) && waitb(&e_loaded[x], 0, bad);
+                if (inter0) {
+                    go = go && waitb(&phiq_full[x], 0, bad) && waitb(&e_loaded[0], 0, bad);
                     if (go) {
                         fence_after_sync();
-                        uint8_t* e = x == 0 ? sE : sPhi;
+                        uint8_t* e = sE;
                         const uint64_t eh = smem_desc(e, kLboE, 128), el = smem_desc(e + 10 * 128, kLboE, 128);
                         const uint32_t dst = tb + kTO + 80 * x;
 #pragma unroll
@@ -332,19 +355,35 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         }
     } else if (warp == 9) {
         if (lane == 0) {
-            // ------------------------------------------------ publishing the chunk states
-            // the staged T_x^T rows leave in one bulk store per chunk; once
-            // they have completed, the head's count of published chunks grows
+            // ------------------------------------------------ publishing the state
+            // the staged T^T rows leave in one bulk store; once it has
+            // completed, the head's count of published states grows
             if (waitb(&t_staged, 0, bad)) {
-                for (int x = 0; x < nch; ++x)
-                    ptx::bulk_s2g(A.TG + ((int64_t)bh * NC + c0 + x) * kXFloats, sPhi + (uint32_t)x * kXFloats * 4u,
-                                  (uint32_t)kXFloats * 4u);
+                ptx::bulk_s2g(A.TG + ((int64_t)bh * NS + seg) * kXFloats, sPhi, (uint32_t)kXFloats * 4u);
                 ptx::bulk_commit();
                 ptx::bulk_wait_all();
                 fence_proxy_async_global();
                 __threadfence();
                 TA_PHASE(1, 9, true);
-                if (!*bad) red_release_add(tcount, (unsigned)nch);
+                if (!*bad) red_release_add(tcount, 1u);
+                // the scan's gather: rows [R seg, R seg + nrows) of every state of
+                // the head (the bulk store above has read the staging space)
+                const int R = (F + NS - 1) / NS, f_lo = R * seg, nrows = max(0, min(R, F - f_lo));
+                if (nrows > 0) {
+                    if (!*bad && wait_count(tcount, (unsigned)NS, bad)) {
+                        TA_PHASE(1, 5, true);
+                        fence_proxy_async_global();
+                        s_gath_issued = 1;
+                        const uint32_t bytes = (uint32_t)nrows * kRowBytes;
+                        ptx::mbar_arrive_expect_tx(&gath, (uint32_t)NS * bytes);
+                        const float* src = A.TG + (int64_t)bh * NS * kXFloats + (int64_t)f_lo * kXStride;
+                        for (int c = 0; c < NS; ++c)
+                            ptx::bulk_g2s(sPhi + c * bytes, src + (int64_t)c * kXFloats, bytes, &gath);
+                    } else {
+                        atomicOr(A.err, kErrPrefillPipe);
+                        *bad = 1;
+                    }
+                }
             }
         }
     } else {
@@ -407,7 +446,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             fence_after_sync();
             if ((warp & 3) < 3) {
                 const int vc = row;  // lanes 0..64: v columns 0..63 and z
-                for (int x = 0; x < nch; ++x) {
+                for (int x = 0; x < 1; ++x) {  // the CTA's state (both chunks)
                     float* tg = reinterpret_cast<float*>(sPhi) + x * kXFloats;
 #pragma unroll
                     for (int p = 0; p < 5; ++p) {
@@ -426,12 +465,11 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             // E of chunk a: its groups past the last feature group stay zero
             for (uint32_t o = (uint32_t)ngroups * kGroupBytes + 16u * tid; o < kEBytes; o += 16u * kCompute)
                 *reinterpret_cast<uint4*>(sE + o) = make_uint4(0, 0, 0, 0);
-            // and so do the rows F .. 8 ngroups - 1 of the published operands,
-            // which no owner writes (this CTA's chunks, all 20 column pieces)
-            for (int u = tid; u < nch * (8 * ngroups - F) * 20; u += kCompute) {
-                const int x = u / ((8 * ngroups - F) * 20), r = u % ((8 * ngroups - F) * 20);
-                const int f = F + r / 20, piece = r % 20;
-                uint8_t* d = A.EG + ((int64_t)bh * NC + c0 + x) * kEBytes + (f >> 3) * kGroupBytes + piece * 128 +
+            // and so do the rows F .. 8 ngroups - 1 of the published operand,
+            // which no owner writes (this CTA's entry, all 20 column pieces)
+            for (int u = tid; u < (8 * ngroups - F) * 20; u += kCompute) {
+                const int f = F + u / 20, piece = u % 20;
+                uint8_t* d = A.EG + ((int64_t)bh * NS + seg) * kEBytes + (f >> 3) * kGroupBytes + piece * 128 +
                              (f & 7) * 16;
                 *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
             }
@@ -448,35 +486,40 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         // each 32-key piece written in place over its own scores columns as
         // the TMEM A operand (16 hi words, then 16 lo words)
         const float c1 = n >= 2 ? A.tau : 0.f, c2 = n >= 3 ? 0.5f * A.tau * A.tau : 0.f;
-        for (int x = 0; x < nch && ok; ++x) {
-            ok = waitb(&sc_full, x & 1, bad);
-            if (!ok) break;
-            fence_after_sync();
+        auto p_rounds = [&](int r0, int r1) {
+            for (int r = r0; r < r1 && ok; ++r) {
+                ok = waitb(&sc_full[r & 1], (r >> 1) & 1, bad);
+                if (!ok) break;
+                fence_after_sync();
+                const bool causal = r < 2;  // round 2: chunk b against all of chunk a
 #pragma unroll
-            for (int pc = 0; pc < 2; ++pc) {
-                const uint32_t tp = tb + kTT + lane_off + 64 * half + 32 * pc;
-                float sc[32];
-                tmem_ld32(tp, sc);
-                tmem_ld_wait();
-                uint32_t hi[16], lo[16];
+                for (int pc = 0; pc < 2; ++pc) {
+                    const uint32_t tp = tb + kTT + kPBuf * (r & 1) + lane_off + 64 * half + 32 * pc;
+                    float sc[32];
+                    tmem_ld32(tp, sc);
+                    tmem_ld_wait();
+                    uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    float p2[2];
+                    for (int j = 0; j < 32; j += 2) {
+                        float p2[2];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float p = fmaf(fmaf(c2, sc[j + e], c1), sc[j + e], 1.f);
-                        if (64 * half + 32 * pc + j + e > row) p = 0.f;
-                        p2[e] = p;
+                        for (int e = 0; e < 2; ++e) {
+                            float p = fmaf(fmaf(c2, sc[j + e], c1), sc[j + e], 1.f);
+                            if (causal && 64 * half + 32 * pc + j + e > row) p = 0.f;
+                            p2[e] = p;
+                        }
+                        split2(p2[0], p2[1], hi[j >> 1], lo[j >> 1]);
                     }
-                    split2(p2[0], p2[1], hi[j >> 1], lo[j >> 1]);
+                    tmem_st16(tp, hi);
+                    tmem_st16(tp + 16, lo);
                 }
-                tmem_st16(tp, hi);
-                tmem_st16(tp + 16, lo);
+                tmem_st_wait();
+                fence_before_sync();
+                ptx::mbar_arrive(&p_full[r & 1]);
             }
-            tmem_st_wait();
-            fence_before_sync();
-            ptx::mbar_arrive(&p_full);
-        }
+        };
+        // every round now, while the states are published and gathered
+        p_rounds(0, nrounds);
         TA_PHASE(0, 5, tid == 0);
 
         // the scan: this CTA owns features [R seg, R seg + R) of its head (R =
@@ -485,28 +528,13 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         // thread per feature and column walks the chunks), then converts every
         // chunk's prefix into its rows of that chunk's hi/lo operand
         const float* sin = A.state_in ? A.state_in + (int64_t)bh * A.stride : nullptr;
-        float* gbuf = reinterpret_cast<float*>(sPhi);  // [NC][R][68]
+        float* gbuf = reinterpret_cast<float*>(sPhi);  // [NS][R][68]
         const int R = (F + NS - 1) / NS;
         const int f_lo = R * seg, nrows = max(0, min(R, F - f_lo));
         if (nrows > 0) {
-            compute_sync();  // the Phi_K space is free once the chunk states are formed
-            if (tid == 0) {
-                if (ok && wait_count(tcount, (unsigned)NC, bad)) {
-                    TA_PHASE(1, 5, true);
-                    fence_proxy_async_global();
-                    s_gath_issued = 1;
-                    const uint32_t bytes = (uint32_t)nrows * kRowBytes;
-                    ptx::mbar_arrive_expect_tx(&gath, (uint32_t)NC * bytes);
-                    const float* src = A.TG + (int64_t)bh * NC * kXFloats + (int64_t)f_lo * kXStride;
-                    for (int c = 0; c < NC; ++c)
-                        ptx::bulk_g2s(sPhi + c * bytes, src + (int64_t)c * kXFloats, bytes, &gath);
-                } else {
-                    atomicOr(A.err, kErrPrefillPipe);
-                    *bad = 1;
-                }
-            }
-            compute_sync();
-            const bool have = !*bad && waitb(&gath, 0, bad);
+            // the publishing warp gathers this CTA's rows of every state of
+            // the head into the Phi_K space once all of them are published
+            const bool have = ok && !*bad && waitb(&gath, 0, bad);
             TA_PHASE(1, 6, tid == 0);
             const int cstride = nrows * kXStride;  // floats per chunk in the gather
             if (have) {
@@ -517,7 +545,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                     float run = 0.f;
                     if (sin) run = col < kDV ? sin[(int64_t)f * kDV + col] : sin[(int64_t)F * kDV + f];
                     float* gcol = gbuf + fr * kXStride + col;
-                    for (int c = 0; c < NC; ++c) {
+                    for (int c = 0; c < NS; ++c) {
                         const float x = gcol[c * cstride];
                         gcol[c * cstride] = run;
                         run += x;
@@ -534,8 +562,8 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             if (have) {
                 // chunk c, column piece c8 (8 columns), feature row fr: 16 bytes hi, 16 lo
                 const int per_chunk = nrows * 10;
-                uint8_t* ebase = A.EG + (int64_t)bh * NC * kEBytes;
-                for (int u = tid; u < NC * per_chunk; u += kCompute) {
+                uint8_t* ebase = A.EG + (int64_t)bh * NS * kEBytes;
+                for (int u = tid; u < NS * per_chunk; u += kCompute) {
                     const int c = u / per_chunk, r = u % per_chunk, c8 = r / nrows, fr = r % nrows, f = f_lo + fr;
                     const float* xr = gbuf + c * cstride + fr * kXStride + 8 * c8;
                     float x8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -564,24 +592,19 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                 A.state_out[(int64_t)bh * A.stride + e] = 0.f;
         TA_PHASE(0, 6, tid == 0);
 
-        // the read-out operands E_x, once every group of the head is written;
-        // E of chunk b goes to the Phi_K space (this CTA's own gathers are read by then)
-        const bool inter_any = inter0 || nch > 1;
+        // the read-out operand E of the state before this CTA (both chunks
+        // read out through it; chunk b meets chunk a in the pairwise part),
+        // once every feature row of the head is scanned
+        const bool inter_any = inter0;
         if (inter_any) {
-            compute_sync();  // this CTA's gathers have been read: the Phi_K space takes E of chunk b
-            if (nch > 1)
-                for (uint32_t o = (uint32_t)ngroups * kGroupBytes + 16u * tid; o < kEBytes; o += 16u * kCompute)
-                    *reinterpret_cast<uint4*>(sPhi + o) = make_uint4(0, 0, 0, 0);
+            compute_sync();
             if (tid == 0) {
                 if (!*bad && wait_count(gcount, (unsigned)F, bad)) {
                     fence_proxy_async_global();
-                    for (int x = 0; x < nch; ++x) {
-                        if (x == 0 && !inter0) continue;
-                        s_e_issued[x] = 1;
-                        ptx::mbar_arrive_expect_tx(&e_loaded[x], (uint32_t)ngroups * kGroupBytes);
-                        ptx::bulk_g2s(x == 0 ? sE : sPhi, A.EG + ((int64_t)bh * NC + c0 + x) * kEBytes,
-                                      (uint32_t)ngroups * kGroupBytes, &e_loaded[x]);
-                    }
+                    s_e_issued[0] = 1;
+                    ptx::mbar_arrive_expect_tx(&e_loaded[0], (uint32_t)ngroups * kGroupBytes);
+                    ptx::bulk_g2s(sE, A.EG + ((int64_t)bh * NS + seg) * kEBytes, (uint32_t)ngroups * kGroupBytes,
+                                  &e_loaded[0]);
                 } else {
                     atomicOr(A.err, kErrPrefillPipe);
                 }
@@ -589,9 +612,10 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             TA_PHASE(0, 7, tid == 0);
             // c (.) Phi_Q,x into TMEM once the last P has been consumed: half 0
             // features 0..95 (words 0..47), half 1 features 96..159 (words 48..79)
-            ok = ok && waitb(&p_free, (nch - 1) & 1, bad);
+            // every P consumed: buffer 0 was used (nrounds + 1) / 2 times, buffer 1 nrounds / 2
+            ok = ok && waitb(&p_free[0], (((nrounds + 1) >> 1) - 1) & 1, bad);
+            if (nrounds > 1) ok = ok && waitb(&p_free[1], ((nrounds >> 1) - 1) & 1, bad);
             for (int x = 0; x < nch && ok; ++x) {
-                if (x == 0 && !inter0) continue;
                 fence_after_sync();
                 float q16[16];
                 ld_row_sw32(sQ + x * kQBytes, row, q16);
@@ -716,7 +740,7 @@ int try_prefill_fused(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv
     if ((int64_t)BH * NS > su.capacity) return kNotApplicable;
     // each CTA's share of the scan: R feature rows of every chunk state of its head
     const int R = (int)((F + NS - 1) / NS);
-    if ((int64_t)NC * R * kRowBytes > kGatherMax) return kNotApplicable;
+    if ((int64_t)NS * R * kRowBytes > kGatherMax) return kNotApplicable;
     unsigned int* err = device_error_word();
     if (!err) return TAYLOR_ERR_CUDA;
 
@@ -728,8 +752,8 @@ int try_prefill_fused(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv
 
     // workspace: published chunk states, read-out operands, flags
     const int ngroups = (int)((F + 7) / 8);
-    const size_t tg_bytes = (size_t)BH * NC * kXFloats * sizeof(float);
-    const size_t eg_bytes = (size_t)BH * NC * kEBytes;
+    const size_t tg_bytes = (size_t)BH * NS * kXFloats * sizeof(float);  // one state per CTA
+    const size_t eg_bytes = (size_t)BH * NS * kEBytes;                    // one read-out operand per CTA
     const size_t fl_bytes = (size_t)2 * BH * sizeof(unsigned);
     uint8_t* ws = nullptr;
     if (workspace_alloc(reinterpret_cast<void**>(&ws), tg_bytes + eg_bytes + fl_bytes, stream) != cudaSuccess) {
