@@ -384,6 +384,20 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                         *bad = 1;
                     }
                 }
+                // the read-out operand of the state before this CTA, once every
+                // feature row of the head is scanned
+                if (inter0) {
+                    if (!*bad && wait_count(gcount, (unsigned)F, bad)) {
+                        fence_proxy_async_global();
+                        s_e_issued[0] = 1;
+                        ptx::mbar_arrive_expect_tx(&e_loaded[0], (uint32_t)ngroups * kGroupBytes);
+                        ptx::bulk_g2s(sE, A.EG + ((int64_t)bh * NS + seg) * kEBytes, (uint32_t)ngroups * kGroupBytes,
+                                      &e_loaded[0]);
+                    } else {
+                        atomicOr(A.err, kErrPrefillPipe);
+                        *bad = 1;
+                    }
+                }
             }
         }
     } else {
@@ -595,20 +609,9 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         // the read-out operand E of the state before this CTA (both chunks
         // read out through it; chunk b meets chunk a in the pairwise part),
         // once every feature row of the head is scanned
+        // (the publishing warp loads it)
         const bool inter_any = inter0;
         if (inter_any) {
-            compute_sync();
-            if (tid == 0) {
-                if (!*bad && wait_count(gcount, (unsigned)F, bad)) {
-                    fence_proxy_async_global();
-                    s_e_issued[0] = 1;
-                    ptx::mbar_arrive_expect_tx(&e_loaded[0], (uint32_t)ngroups * kGroupBytes);
-                    ptx::bulk_g2s(sE, A.EG + ((int64_t)bh * NS + seg) * kEBytes, (uint32_t)ngroups * kGroupBytes,
-                                  &e_loaded[0]);
-                } else {
-                    atomicOr(A.err, kErrPrefillPipe);
-                }
-            }
             TA_PHASE(0, 7, tid == 0);
             // c (.) Phi_Q,x into TMEM once the last P has been consumed: half 0
             // features 0..95 (words 0..47), half 1 features 96..159 (words 48..79)
