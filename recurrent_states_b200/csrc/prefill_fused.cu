@@ -614,7 +614,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         if (inter_any) {
             TA_PHASE(0, 7, tid == 0);
             // c (.) Phi_Q,x into TMEM once the last P has been consumed: half 0
-            // features 0..95 (words 0..47), half 1 features 96..159 (words 48..79)
+            // features 0..79 (words 0..39), half 1 features 80..159 (words 40..79)
             // every P consumed: buffer 0 was used (nrounds + 1) / 2 times, buffer 1 nrounds / 2
             ok = ok && waitb(&p_free[0], (((nrounds + 1) >> 1) - 1) & 1, bad);
             if (nrounds > 1) ok = ok && waitb(&p_free[1], ((nrounds >> 1) - 1) & 1, bad);
@@ -624,23 +624,29 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                 ld_row_sw32(sQ + x * kQBytes, row, q16);
                 const float e0 = row < (x == 0 ? nval0 : nval1) ? 1.f : 0.f;
                 const uint32_t th = tb + kTT + 160 * x + lane_off, tl = th + 80;
+                // 16 features a step: words F0 / 2 .. F0 / 2 + 7 of the hi and lo halves
                 auto emit = [&](auto fb) {
                     constexpr int F0 = decltype(fb)::value;
-                    float o[32];
-                    phi16_range<F0, F0 + 32>(q16, e0, c1, c2, o);
-                    uint32_t hw[16], lw[16];
+                    float o[16];
+                    phi16_range<F0, F0 + 16>(q16, e0, c1, c2, o);
+                    uint32_t hw[8], lw[8];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) split2(o[2 * i], o[2 * i + 1], hw[i], lw[i]);
-                    tmem_st16(th + F0 / 2, hw);
-                    tmem_st16(tl + F0 / 2, lw);
+                    for (int i = 0; i < 8; ++i) split2(o[2 * i], o[2 * i + 1], hw[i], lw[i]);
+                    tmem_st8(th + F0 / 2, hw);
+                    tmem_st8(tl + F0 / 2, lw);
                 };
-                if (half == 0) {
+                if (half == 0) {  // features 0..79
                     emit(std::integral_constant<int, 0>());
+                    emit(std::integral_constant<int, 16>());
                     emit(std::integral_constant<int, 32>());
+                    emit(std::integral_constant<int, 48>());
                     emit(std::integral_constant<int, 64>());
-                } else {
+                } else {  // features 80..159
+                    emit(std::integral_constant<int, 80>());
                     emit(std::integral_constant<int, 96>());
+                    emit(std::integral_constant<int, 112>());
                     emit(std::integral_constant<int, 128>());
+                    emit(std::integral_constant<int, 144>());
                 }
                 tmem_st_wait();
                 ptx::fence_proxy_async_smem();  // the zeroed tails of E
