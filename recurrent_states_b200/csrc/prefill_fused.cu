@@ -334,6 +334,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             for (int x = 0; x < nch; ++x) {
                 if (inter0) {
                     go = go && waitb(&phiq_full[x], 0, bad) && waitb(&e_loaded[0], 0, bad);
+                    TA_PHASE(1, 10 + 2 * x, true);
                     if (go) {
                         fence_after_sync();
                         uint8_t* e = sE;
@@ -349,6 +350,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                     }
                 }
                 mma_commit(&ro_done[x]);  // covers every MMA issued so far, also after a failure
+                TA_PHASE(1, 11 + 2 * x, true);
             }
             TA_PHASE(1, 4, true);
             if (!go) *bad = 1;
@@ -652,6 +654,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                 ptx::fence_proxy_async_smem();  // the zeroed tails of E
                 fence_before_sync();
                 ptx::mbar_arrive(&phiq_full[x]);
+                TA_PHASE(0, 11 + x, tid == 0);
             }
             TA_PHASE(0, 8, tid == 0);
         }
@@ -660,6 +663,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         for (int x = 0; x < nch; ++x) {
             const bool done = waitb(&ro_done[x], 0, bad);
             fence_after_sync();
+            TA_PHASE(0, 13 + x, tid == 0);
             if (!done || *bad) break;
             float o[32];
             const uint32_t to = tb + kTO + 80 * x + lane_off;

@@ -62,13 +62,18 @@ CASES = [
     (1, 1, 2600, 64, 64, 3),
     (1, 1, 700, 32, 64, 4),   # run-time feature descriptors on the tiled path
     (1, 1, 500, 64, 64, 2),
-    # the one-launch cluster prefill (d_k 16, d_v 64, n <= 3): segments of one
-    # chunk, of two chunks with a one-token last segment, full 16-CTA clusters
+    # the one-launch prefill (d_k 16, d_v 64, n <= 3), one chunk per CTA
+    # (heads x chunks fit the SMs): a one-token last chunk, ragged tails
     (2, 3, 2048, 16, 64, 3),
     (1, 3, 2049, 16, 64, 3),
     (2, 2, 3000, 16, 64, 2),
     (1, 2, 4096, 16, 64, 1),
     (1, 1, 3967, 16, 64, 3),
+    # two chunks per CTA (one state per CTA, chunk b meets chunk a pairwise):
+    # an odd chunk count (the last CTA has one ragged chunk), n = 2 and n = 1
+    (1, 8, 3900, 16, 64, 3),
+    (2, 5, 2560, 16, 64, 2),
+    (1, 10, 1929, 16, 64, 1),
 ]
 
 
@@ -371,6 +376,28 @@ def test_prefill_from_state_continues_the_sequence(dtype, d, dv, n, N, cut):
     # in place: state_out aliasing state_in
     st2 = st_head.clone()
     cont(t_(q), t_(k), t_(v), st2, n, tau, state_out=st2)
+    torch.cuda.synchronize()
+    assert torch.equal(st2, st)
+
+
+def test_two_chunks_per_cta_prefill_from_a_carried_state():
+    """The one-launch prefill with two chunks per CTA (B1 H8, 3,900 new tokens:
+    31 chunks, 16 CTAs per head, the last with one ragged chunk) continuing
+    from the state of a 500-token prefix: every CTA, the first included, reads
+    out through a non-zero state.  Outputs of the tail and the final state
+    against the oracle's recursion; in place as well."""
+    B, H, d, dv, n, tau, cut, N = 1, 8, 16, 64, 3, 2.0, 500, 4400
+    q, k, v = synth.qkv(B, H, N, d, dv, seed=77, dtype="bf16")
+    h = lambda t: t[:, :, :cut].contiguous().to(DEV)  # noqa: E731
+    t_ = lambda t: t[:, :, cut:].contiguous().to(DEV)  # noqa: E731
+    _, st_head = TA.taylor_attn_prefill(h(q), h(k), h(v), n, tau, state_out=True)
+    out_tail, st = TA.taylor_attn_prefill_from_state(t_(q), t_(k), t_(v), st_head, n, tau, state_out=True)
+    torch.cuda.synchronize()
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    assert row_scaled_max_err(f64(out_tail), ref_out[:, :, cut:]) <= TOL["bf16"]
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL["bf16"]
+    st2 = st_head.clone()
+    TA.taylor_attn_prefill_from_state(t_(q), t_(k), t_(v), st2, n, tau, state_out=st2)
     torch.cuda.synchronize()
     assert torch.equal(st2, st)
 
