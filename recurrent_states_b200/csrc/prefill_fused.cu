@@ -408,66 +408,23 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = waitb(&ld, 0, bad);
         TA_PHASE(0, 1, tid == 0);
+        const float c1 = n >= 2 ? A.tau : 0.f, c2 = n >= 3 ? 0.5f * A.tau * A.tau : 0.f;
 
-        // Phi_K of chunk x, token `row`, features [80 half, 80 half + 80),
-        // hi and lo, into the MN-major operand
-        auto phik = [&](int x) {
-            float k16[16];
-            ld_row_sw32(sK + x * kQBytes, row, k16);
-            const bool valid = row < (x == 0 ? nval0 : nval1);
-            const float e0 = valid ? 1.f : 0.f, e1 = (valid && n >= 2) ? 1.f : 0.f, e2 = (valid && n >= 3) ? 1.f : 0.f;
-            auto emit = [&](auto fb) {
-                constexpr int F0 = decltype(fb)::value;
-                float o[16];
-                phi16_range<F0, F0 + 16>(k16, e0, e1, e2, o);
-                uint4 hi0, lo0, hi1, lo1;
-                split8(o, hi0, lo0);
-                split8(o + 8, hi1, lo1);
-                *reinterpret_cast<uint4*>(sPhi + mnmaj(row, F0 / 8, kLboPhi)) = hi0;
-                *reinterpret_cast<uint4*>(sPhi + mnmaj(row, F0 / 8 + 1, kLboPhi)) = hi1;
-                *reinterpret_cast<uint4*>(sPhi + kPhiBytes + mnmaj(row, F0 / 8, kLboPhi)) = lo0;
-                *reinterpret_cast<uint4*>(sPhi + kPhiBytes + mnmaj(row, F0 / 8 + 1, kLboPhi)) = lo1;
-            };
-            if (half == 0) {
-                emit(std::integral_constant<int, 0>());
-                emit(std::integral_constant<int, 16>());
-                emit(std::integral_constant<int, 32>());
-                emit(std::integral_constant<int, 48>());
-                emit(std::integral_constant<int, 64>());
-            } else {
-                emit(std::integral_constant<int, 80>());
-                emit(std::integral_constant<int, 96>());
-                emit(std::integral_constant<int, 112>());
-                emit(std::integral_constant<int, 128>());
-                emit(std::integral_constant<int, 144>());
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(&phik_full);
-        };
-        for (int x = 0; x < nch && ok; ++x) {
-            if (x > 0) {
-                ok = waitb(&phik_free, 0, bad);
+        // stage the CTA's state T^T (lane = v column, 160 feature columns) as
+        // [feature][column] rows in the Phi_K space, which the state MMAs have
+        // finished reading; the publishing warp takes them to L2
+        auto stage_state = [&]() {
+            ok = ok && waitb(&t_done, 0, bad);
+            TA_PHASE(0, 3, tid == 0);
+            if (ok) {
                 fence_after_sync();
-            }
-            if (ok) phik(x);
-        }
-        TA_PHASE(0, 2, tid == 0);
-
-        // stage the chunk states T_x^T (lane = v column, 160 feature columns)
-        // as [feature][column] rows in the Phi_K space, which the state MMAs
-        // have finished reading; the publishing warp takes them to L2
-        ok = ok && waitb(&t_done, 0, bad);
-        TA_PHASE(0, 3, tid == 0);
-        if (ok) {
-            fence_after_sync();
-            if ((warp & 3) < 3) {
-                const int vc = row;  // lanes 0..64: v columns 0..63 and z
-                for (int x = 0; x < 1; ++x) {  // the CTA's state (both chunks)
-                    float* tg = reinterpret_cast<float*>(sPhi) + x * kXFloats;
+                if ((warp & 3) < 3) {
+                    const int vc = row;  // lanes 0..64: v columns 0..63 and z
+                    float* tg = reinterpret_cast<float*>(sPhi);
 #pragma unroll
                     for (int p = 0; p < 5; ++p) {
                         float r[16];
-                        tmem_ld16(tb + kTT + 160 * x + lane_off + 80 * half + 16 * p, r);
+                        tmem_ld16(tb + kTT + lane_off + 80 * half + 16 * p, r);
                         tmem_ld_wait();
                         if (vc <= kDV) {
 #pragma unroll
@@ -475,33 +432,22 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                         }
                     }
                 }
+                fence_before_sync();
+                ptx::mbar_arrive(&t_free);
+                // E of chunk a: its groups past the last feature group stay zero
+                for (uint32_t o = (uint32_t)ngroups * kGroupBytes + 16u * tid; o < kEBytes; o += 16u * kCompute)
+                    *reinterpret_cast<uint4*>(sE + o) = make_uint4(0, 0, 0, 0);
             }
-            fence_before_sync();
-            ptx::mbar_arrive(&t_free);
-            // E of chunk a: its groups past the last feature group stay zero
-            for (uint32_t o = (uint32_t)ngroups * kGroupBytes + 16u * tid; o < kEBytes; o += 16u * kCompute)
-                *reinterpret_cast<uint4*>(sE + o) = make_uint4(0, 0, 0, 0);
-            // and so do the rows F .. 8 ngroups - 1 of the published operand,
-            // which no owner writes (this CTA's entry, all 20 column pieces)
-            for (int u = tid; u < (8 * ngroups - F) * 20; u += kCompute) {
-                const int f = F + u / 20, piece = u % 20;
-                uint8_t* d = A.EG + ((int64_t)bh * NS + seg) * kEBytes + (f >> 3) * kGroupBytes + piece * 128 +
-                             (f & 7) * 16;
-                *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
-            }
-        }
-        // the staged rows go to the publishing warp's bulk stores; the zeroed
-        // rows are read by this CTA's own bulk loads of E
-        ptx::fence_proxy_async_smem();
-        __threadfence();
-        compute_sync();
-        if (tid == 0 && ok && !*bad) ptx::mbar_arrive(&t_staged);
-        TA_PHASE(0, 4, tid == 0);
+            // the staged rows go to the publishing warp's bulk store
+            ptx::fence_proxy_async_smem();
+            compute_sync();
+            if (tid == 0 && ok && !*bad) ptx::mbar_arrive(&t_staged);
+            TA_PHASE(0, 4, tid == 0);
+        };
 
         // P = poly(tau q.k) of query `row` against keys [64 half, 64 half + 64),
         // each 32-key piece written in place over its own scores columns as
         // the TMEM A operand (16 hi words, then 16 lo words)
-        const float c1 = n >= 2 ? A.tau : 0.f, c2 = n >= 3 ? 0.5f * A.tau * A.tau : 0.f;
         auto p_rounds = [&](int r0, int r1) {
             for (int r = r0; r < r1 && ok; ++r) {
                 ok = waitb(&sc_full[r & 1], (r >> 1) & 1, bad);
@@ -534,20 +480,19 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                 ptx::mbar_arrive(&p_full[r & 1]);
             }
         };
-        // every round now, while the states are published and gathered
-        p_rounds(0, nrounds);
-        TA_PHASE(0, 5, tid == 0);
 
         // the scan: this CTA owns features [R seg, R seg + R) of its head (R =
         // ceil(F / NS)); it gathers those rows of every chunk state of the head
         // into shared memory, turns them in place into exclusive prefixes (one
         // thread per feature and column walks the chunks), then converts every
-        // chunk's prefix into its rows of that chunk's hi/lo operand
-        const float* sin = A.state_in ? A.state_in + (int64_t)bh * A.stride : nullptr;
-        float* gbuf = reinterpret_cast<float*>(sPhi);  // [NS][R][68]
-        const int R = (F + NS - 1) / NS;
-        const int f_lo = R * seg, nrows = max(0, min(R, F - f_lo));
-        if (nrows > 0) {
+        // chunk's prefix into its rows of that chunk's hi/lo operand; the owner
+        // of the last rows also writes the zero rows F .. 8 ngroups - 1
+        auto scan = [&]() {
+            const float* sin = A.state_in ? A.state_in + (int64_t)bh * A.stride : nullptr;
+            float* gbuf = reinterpret_cast<float*>(sPhi);  // [NS][R][68]
+            const int R = (F + NS - 1) / NS;
+            const int f_lo = R * seg, nrows = max(0, min(R, F - f_lo));
+            if (nrows == 0) return;
             // the publishing warp gathers this CTA's rows of every state of
             // the head into the Phi_K space once all of them are published
             const bool have = ok && !*bad && waitb(&gath, 0, bad);
@@ -577,13 +522,16 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             TA_PHASE(1, 7, tid == 0);
             if (have) {
                 // chunk c, column piece c8 (8 columns), feature row fr: 16 bytes hi, 16 lo
-                const int per_chunk = nrows * 10;
+                const int erows = f_lo + nrows == F ? 8 * ngroups - f_lo : nrows;
+                const int per_chunk = erows * 10;
                 uint8_t* ebase = A.EG + (int64_t)bh * NS * kEBytes;
                 for (int u = tid; u < NS * per_chunk; u += kCompute) {
-                    const int c = u / per_chunk, r = u % per_chunk, c8 = r / nrows, fr = r % nrows, f = f_lo + fr;
+                    const int c = u / per_chunk, r = u % per_chunk, c8 = r / erows, fr = r % erows, f = f_lo + fr;
                     const float* xr = gbuf + c * cstride + fr * kXStride + 8 * c8;
                     float x8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    if (c8 < 8) {
+                    if (fr >= nrows) {
+                        // padding row: stays zero
+                    } else if (c8 < 8) {
                         const float4 a0 = reinterpret_cast<const float4*>(xr)[0];
                         const float4 a1 = reinterpret_cast<const float4*>(xr)[1];
                         x8[0] = a0.x; x8[1] = a0.y; x8[2] = a0.z; x8[3] = a0.w;
@@ -598,66 +546,110 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                     *reinterpret_cast<uint4*>(d + 10 * 128) = lo;
                 }
             }
-            __threadfence();
             TA_PHASE(1, 8, tid == 0);
+            // every thread's rows, then one release at GPU scope (cumulative
+            // over the CTA barrier) for the head's count of scanned rows
             compute_sync();
             if (tid == 0 && !*bad) red_release_add(gcount, (unsigned)nrows);
-        }
-        if (A.state_out && seg == 0)
-            for (int64_t e = (int64_t)F * (kDV + 1) + tid; e < A.stride; e += kCompute)
-                A.state_out[(int64_t)bh * A.stride + e] = 0.f;
-        TA_PHASE(0, 6, tid == 0);
+        };
 
-        // the read-out operand E of the state before this CTA (both chunks
-        // read out through it; chunk b meets chunk a in the pairwise part),
-        // once every feature row of the head is scanned
-        // (the publishing warp loads it)
-        const bool inter_any = inter0;
-        if (inter_any) {
-            TA_PHASE(0, 7, tid == 0);
-            // c (.) Phi_Q,x into TMEM once the last P has been consumed: half 0
-            // features 0..79 (words 0..39), half 1 features 80..159 (words 40..79)
-            // every P consumed: buffer 0 was used (nrounds + 1) / 2 times, buffer 1 nrounds / 2
-            ok = ok && waitb(&p_free[0], (((nrounds + 1) >> 1) - 1) & 1, bad);
-            if (nrounds > 1) ok = ok && waitb(&p_free[1], ((nrounds >> 1) - 1) & 1, bad);
-            for (int x = 0; x < nch && ok; ++x) {
-                fence_after_sync();
-                float q16[16];
-                ld_row_sw32(sQ + x * kQBytes, row, q16);
-                const float e0 = row < (x == 0 ? nval0 : nval1) ? 1.f : 0.f;
-                const uint32_t th = tb + kTT + 160 * x + lane_off, tl = th + 80;
-                // 16 features a step: words F0 / 2 .. F0 / 2 + 7 of the hi and lo halves
-                auto emit = [&](auto fb) {
-                    constexpr int F0 = decltype(fb)::value;
-                    float o[16];
-                    phi16_range<F0, F0 + 16>(q16, e0, c1, c2, o);
-                    uint32_t hw[8], lw[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) split2(o[2 * i], o[2 * i + 1], hw[i], lw[i]);
-                    tmem_st8(th + F0 / 2, hw);
-                    tmem_st8(tl + F0 / 2, lw);
-                };
-                if (half == 0) {  // features 0..79
-                    emit(std::integral_constant<int, 0>());
-                    emit(std::integral_constant<int, 16>());
-                    emit(std::integral_constant<int, 32>());
-                    emit(std::integral_constant<int, 48>());
-                    emit(std::integral_constant<int, 64>());
-                } else {  // features 80..159
-                    emit(std::integral_constant<int, 80>());
-                    emit(std::integral_constant<int, 96>());
-                    emit(std::integral_constant<int, 112>());
-                    emit(std::integral_constant<int, 128>());
-                    emit(std::integral_constant<int, 144>());
+        // Feature rows, one code path for both sides, so that the query side
+        // runs on instructions the key side has already fetched: when the
+        // kernel's code is in no cache, L2 included (as after other work has
+        // streamed through L2), the first pass through this straight-line code
+        // takes several times as long as later ones.  Pass j < 2 writes Phi_K of chunk j, token `row`,
+        // features [80 half, 80 half + 80), hi and lo, into the MN-major
+        // shared-memory operand; pass j >= 2 writes c (.) Phi_Q of chunk j - 2
+        // into TMEM (half 0 features 0..79 = words 0..39 of the hi and lo
+        // halves, half 1 features 80..159).  Between the two sides: the staged
+        // state, the pairwise rounds and the scan.
+#pragma unroll 1
+        for (int j = 0; j < 4; ++j) {
+            const bool qside = j >= 2;
+            const int x = j & 1;
+            if (j == 2) {
+                TA_PHASE(0, 2, tid == 0);
+                stage_state();
+                // every round now, while the states are published and gathered
+                p_rounds(0, nrounds);
+                TA_PHASE(0, 5, tid == 0);
+                scan();
+                if (A.state_out && seg == 0)
+                    for (int64_t e = (int64_t)F * (kDV + 1) + tid; e < A.stride; e += kCompute)
+                        A.state_out[(int64_t)bh * A.stride + e] = 0.f;
+                TA_PHASE(0, 6, tid == 0);
+                // c (.) Phi_Q goes where the scores / P buffers were: every P
+                // consumed (buffer 0 was used (nrounds + 1) / 2 times, buffer 1
+                // nrounds / 2)
+                if (inter0) {
+                    TA_PHASE(0, 7, tid == 0);
+                    ok = ok && waitb(&p_free[0], (((nrounds + 1) >> 1) - 1) & 1, bad);
+                    if (nrounds > 1) ok = ok && waitb(&p_free[1], ((nrounds >> 1) - 1) & 1, bad);
                 }
+            }
+            if (!ok || x >= nch || (qside && !inter0)) continue;
+            if (!qside && x > 0) ok = waitb(&phik_free, 0, bad);
+            fence_after_sync();
+            if (!ok) continue;
+            float x16[16];
+            ld_row_sw32((qside ? sQ : sK) + x * kQBytes, row, x16);
+            const bool valid = row < (x == 0 ? nval0 : nval1);
+            const float e0 = valid ? 1.f : 0.f;
+            const float e1 = qside ? c1 : ((valid && n >= 2) ? 1.f : 0.f);
+            const float e2 = qside ? c2 : ((valid && n >= 3) ? 1.f : 0.f);
+            // all 80 features of this half first (hi and lo words in registers),
+            // then one store sequence per side
+            uint32_t hw[40], lw[40];
+            auto eval = [&](auto fb) {
+                constexpr int F0 = decltype(fb)::value;
+                constexpr int W = (F0 % 80) / 2;
+                float o[16];
+                phi16_range<F0, F0 + 16>(x16, e0, e1, e2, o);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) split2(o[2 * i], o[2 * i + 1], hw[W + i], lw[W + i]);
+            };
+            if (half == 0) {
+                eval(std::integral_constant<int, 0>());
+                eval(std::integral_constant<int, 16>());
+                eval(std::integral_constant<int, 32>());
+                eval(std::integral_constant<int, 48>());
+                eval(std::integral_constant<int, 64>());
+            } else {
+                eval(std::integral_constant<int, 80>());
+                eval(std::integral_constant<int, 96>());
+                eval(std::integral_constant<int, 112>());
+                eval(std::integral_constant<int, 128>());
+                eval(std::integral_constant<int, 144>());
+            }
+            if (qside) {
+                // words 40 half .. 40 half + 39 of the hi and lo TMEM rows
+                const uint32_t th = tb + kTT + 160 * x + lane_off + 40 * half, tl = th + 80;
+                tmem_st32(th, *reinterpret_cast<const uint32_t(*)[32]>(hw));
+                tmem_st8(th + 32, *reinterpret_cast<const uint32_t(*)[8]>(hw + 32));
+                tmem_st32(tl, *reinterpret_cast<const uint32_t(*)[32]>(lw));
+                tmem_st8(tl + 32, *reinterpret_cast<const uint32_t(*)[8]>(lw + 32));
+            } else {
+                // groups 10 half .. 10 half + 9 of the MN-major operand
+#pragma unroll
+                for (int g = 0; g < 10; ++g) {
+                    const uint32_t off = mnmaj(row, 10 * half + g, kLboPhi);
+                    *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(hw[4 * g], hw[4 * g + 1], hw[4 * g + 2], hw[4 * g + 3]);
+                    *reinterpret_cast<uint4*>(sPhi + kPhiBytes + off) =
+                        make_uint4(lw[4 * g], lw[4 * g + 1], lw[4 * g + 2], lw[4 * g + 3]);
+                }
+            }
+            if (qside) {
                 tmem_st_wait();
                 ptx::fence_proxy_async_smem();  // the zeroed tails of E
                 fence_before_sync();
                 ptx::mbar_arrive(&phiq_full[x]);
                 TA_PHASE(0, 11 + x, tid == 0);
+            } else {
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(&phik_full);
             }
-            TA_PHASE(0, 8, tid == 0);
         }
+        TA_PHASE(0, 8, tid == 0);
 
         // epilogues: o = numerator * (1 / denominator)
         for (int x = 0; x < nch; ++x) {
