@@ -556,18 +556,84 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         // Feature rows, one code path for both sides, so that the query side
         // runs on instructions the key side has already fetched: when the
         // kernel's code is in no cache, L2 included (as after other work has
-        // streamed through L2), the first pass through this straight-line code
-        // takes several times as long as later ones.  Pass j < 2 writes Phi_K of chunk j, token `row`,
-        // features [80 half, 80 half + 80), hi and lo, into the MN-major
-        // shared-memory operand; pass j >= 2 writes c (.) Phi_Q of chunk j - 2
-        // into TMEM (half 0 features 0..79 = words 0..39 of the hi and lo
-        // halves, half 1 features 80..159).  Between the two sides: the staged
-        // state, the pairwise rounds and the scan.
+        // streamed through L2), the first pass through this straight-line
+        // code takes several times as long as later ones.  Code laid out right
+        // after a wait is fetched during it, so the other phases follow the
+        // key side in the loop body, in the order they run.  Pass j < 2 writes
+        // Phi_K of chunk j, token `row`, features [80 half, 80 half + 80), hi
+        // and lo, into the MN-major shared-memory operand; pass j >= 2 writes
+        // c (.) Phi_Q of chunk j - 2 into TMEM (half 0 features 0..79 = words
+        // 0..39 of the hi and lo halves, half 1 features 80..159).  Between the
+        // two sides (after the second key-side pass): the staged state, the
+        // pairwise rounds and the scan.
 #pragma unroll 1
         for (int j = 0; j < 4; ++j) {
             const bool qside = j >= 2;
             const int x = j & 1;
-            if (j == 2) {
+            bool active = ok && x < nch && (!qside || inter0);
+            if (active && j == 1) active = ok = waitb(&phik_free, 0, bad);
+            if (active) {
+                fence_after_sync();
+                float x16[16];
+                ld_row_sw32((qside ? sQ : sK) + x * kQBytes, row, x16);
+                const bool valid = row < (x == 0 ? nval0 : nval1);
+                const float e0 = valid ? 1.f : 0.f;
+                const float e1 = qside ? c1 : ((valid && n >= 2) ? 1.f : 0.f);
+                const float e2 = qside ? c2 : ((valid && n >= 3) ? 1.f : 0.f);
+                // all 80 features of this half first (hi and lo words in registers),
+                // then one store sequence per side
+                uint32_t hw[40], lw[40];
+                auto eval = [&](auto fb) {
+                    constexpr int F0 = decltype(fb)::value;
+                    constexpr int W = (F0 % 80) / 2;
+                    float o[16];
+                    phi16_range<F0, F0 + 16>(x16, e0, e1, e2, o);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) split2(o[2 * i], o[2 * i + 1], hw[W + i], lw[W + i]);
+                };
+                if (half == 0) {
+                    eval(std::integral_constant<int, 0>());
+                    eval(std::integral_constant<int, 16>());
+                    eval(std::integral_constant<int, 32>());
+                    eval(std::integral_constant<int, 48>());
+                    eval(std::integral_constant<int, 64>());
+                } else {
+                    eval(std::integral_constant<int, 80>());
+                    eval(std::integral_constant<int, 96>());
+                    eval(std::integral_constant<int, 112>());
+                    eval(std::integral_constant<int, 128>());
+                    eval(std::integral_constant<int, 144>());
+                }
+                if (qside) {
+                    // words 40 half .. 40 half + 39 of the hi and lo TMEM rows
+                    const uint32_t th = tb + kTT + 160 * x + lane_off + 40 * half, tl = th + 80;
+                    tmem_st32(th, *reinterpret_cast<const uint32_t(*)[32]>(hw));
+                    tmem_st8(th + 32, *reinterpret_cast<const uint32_t(*)[8]>(hw + 32));
+                    tmem_st32(tl, *reinterpret_cast<const uint32_t(*)[32]>(lw));
+                    tmem_st8(tl + 32, *reinterpret_cast<const uint32_t(*)[8]>(lw + 32));
+                } else {
+                    // groups 10 half .. 10 half + 9 of the MN-major operand
+#pragma unroll
+                    for (int g = 0; g < 10; ++g) {
+                        const uint32_t off = mnmaj(row, 10 * half + g, kLboPhi);
+                        *reinterpret_cast<uint4*>(sPhi + off) =
+                            make_uint4(hw[4 * g], hw[4 * g + 1], hw[4 * g + 2], hw[4 * g + 3]);
+                        *reinterpret_cast<uint4*>(sPhi + kPhiBytes + off) =
+                            make_uint4(lw[4 * g], lw[4 * g + 1], lw[4 * g + 2], lw[4 * g + 3]);
+                    }
+                }
+                if (qside) {
+                    tmem_st_wait();
+                    ptx::fence_proxy_async_smem();  // the zeroed tails of E
+                    fence_before_sync();
+                    ptx::mbar_arrive(&phiq_full[x]);
+                    TA_PHASE(0, 11 + x, tid == 0);
+                } else {
+                    ptx::fence_proxy_async_smem();
+                    ptx::mbar_arrive(&phik_full);
+                }
+            }
+            if (j == 1) {
                 TA_PHASE(0, 2, tid == 0);
                 stage_state();
                 // every round now, while the states are published and gathered
@@ -586,67 +652,6 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
                     ok = ok && waitb(&p_free[0], (((nrounds + 1) >> 1) - 1) & 1, bad);
                     if (nrounds > 1) ok = ok && waitb(&p_free[1], ((nrounds >> 1) - 1) & 1, bad);
                 }
-            }
-            if (!ok || x >= nch || (qside && !inter0)) continue;
-            if (!qside && x > 0) ok = waitb(&phik_free, 0, bad);
-            fence_after_sync();
-            if (!ok) continue;
-            float x16[16];
-            ld_row_sw32((qside ? sQ : sK) + x * kQBytes, row, x16);
-            const bool valid = row < (x == 0 ? nval0 : nval1);
-            const float e0 = valid ? 1.f : 0.f;
-            const float e1 = qside ? c1 : ((valid && n >= 2) ? 1.f : 0.f);
-            const float e2 = qside ? c2 : ((valid && n >= 3) ? 1.f : 0.f);
-            // all 80 features of this half first (hi and lo words in registers),
-            // then one store sequence per side
-            uint32_t hw[40], lw[40];
-            auto eval = [&](auto fb) {
-                constexpr int F0 = decltype(fb)::value;
-                constexpr int W = (F0 % 80) / 2;
-                float o[16];
-                phi16_range<F0, F0 + 16>(x16, e0, e1, e2, o);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) split2(o[2 * i], o[2 * i + 1], hw[W + i], lw[W + i]);
-            };
-            if (half == 0) {
-                eval(std::integral_constant<int, 0>());
-                eval(std::integral_constant<int, 16>());
-                eval(std::integral_constant<int, 32>());
-                eval(std::integral_constant<int, 48>());
-                eval(std::integral_constant<int, 64>());
-            } else {
-                eval(std::integral_constant<int, 80>());
-                eval(std::integral_constant<int, 96>());
-                eval(std::integral_constant<int, 112>());
-                eval(std::integral_constant<int, 128>());
-                eval(std::integral_constant<int, 144>());
-            }
-            if (qside) {
-                // words 40 half .. 40 half + 39 of the hi and lo TMEM rows
-                const uint32_t th = tb + kTT + 160 * x + lane_off + 40 * half, tl = th + 80;
-                tmem_st32(th, *reinterpret_cast<const uint32_t(*)[32]>(hw));
-                tmem_st8(th + 32, *reinterpret_cast<const uint32_t(*)[8]>(hw + 32));
-                tmem_st32(tl, *reinterpret_cast<const uint32_t(*)[32]>(lw));
-                tmem_st8(tl + 32, *reinterpret_cast<const uint32_t(*)[8]>(lw + 32));
-            } else {
-                // groups 10 half .. 10 half + 9 of the MN-major operand
-#pragma unroll
-                for (int g = 0; g < 10; ++g) {
-                    const uint32_t off = mnmaj(row, 10 * half + g, kLboPhi);
-                    *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(hw[4 * g], hw[4 * g + 1], hw[4 * g + 2], hw[4 * g + 3]);
-                    *reinterpret_cast<uint4*>(sPhi + kPhiBytes + off) =
-                        make_uint4(lw[4 * g], lw[4 * g + 1], lw[4 * g + 2], lw[4 * g + 3]);
-                }
-            }
-            if (qside) {
-                tmem_st_wait();
-                ptx::fence_proxy_async_smem();  // the zeroed tails of E
-                fence_before_sync();
-                ptx::mbar_arrive(&phiq_full[x]);
-                TA_PHASE(0, 11 + x, tid == 0);
-            } else {
-                ptx::fence_proxy_async_smem();
-                ptx::mbar_arrive(&phik_full);
             }
         }
         TA_PHASE(0, 8, tid == 0);
