@@ -89,8 +89,10 @@ constexpr uint32_t kPhiSpace = 2 * kPhiBytes > kGatherMax ? 2 * kPhiBytes : kGat
 constexpr uint32_t kOffE = kOffPhi + kPhiSpace;     // E of chunk a
 constexpr uint32_t kSmemF = kOffE + kEBytes + 1024; // + alignment slack
 constexpr uint32_t kLboPhi = (kFP / 8) * 128;       // K-group stride of Phi_K (MN-major)
+constexpr uint32_t kOutTile = kC * 128;             // output staging: [128 rows][32 fp32], 128-byte swizzle
 constexpr uint32_t kLboE = kGroupBytes;             // K-group stride of E (MN-major)
 static_assert(kEBytes <= 2 * kPhiBytes, "E of chunk b fits the Phi_K space");
+static_assert(4 * kOutTile <= kPhiSpace, "the output tiles of both chunks fit the Phi_K space");
 static_assert(kSmemF <= 232448, "shared memory");
 
 // TMEM (512 columns): the CTA's state T^T [0, 160); later the scores / P of
@@ -177,13 +179,14 @@ struct FusedArgs {
 
 __global__ void __launch_bounds__(kThreadsF, 1)
 tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                        const __grid_constant__ CUtensorMap tmv, const FusedArgs A) {
+                        const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                        const FusedArgs A) {
     extern __shared__ uint8_t sm_raw[];
     uint8_t* sm = align1k(sm_raw);
     __shared__ __align__(8) uint64_t ld, phik_full, phik_free, t_done, t_free, sc_full[2], p_full[2], p_free[2], gath,
         e_loaded[2], phiq_full[2], ro_done[2], t_staged;
     __shared__ uint32_t tslot;
-    __shared__ int s_bad, s_e_issued[2], s_gath_issued;
+    __shared__ int s_bad, s_e_issued[2], s_gath_issued, s_out_issued;
     volatile int* bad = &s_bad;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -230,6 +233,7 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         }
         s_bad = 0;
         s_gath_issued = 0;
+        s_out_issued = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 8) {
@@ -656,24 +660,37 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
         }
         TA_PHASE(0, 8, tid == 0);
 
-        // epilogues: o = numerator * (1 / denominator)
+        // epilogues: o = numerator * (1 / denominator), staged as two
+        // [128 rows][32 columns] fp32 tiles a chunk under the 128-byte swizzle
+        // (in the Phi_K space, idle since the scan) and written by TMA tensor
+        // stores, which leave out the rows past the sequence.  Per-thread
+        // global stores would fill the SM's memory pipeline while the other
+        // chunk's read-out is still being issued.
         for (int x = 0; x < nch; ++x) {
             const bool done = waitb(&ro_done[x], 0, bad);
             fence_after_sync();
             TA_PHASE(0, 13 + x, tid == 0);
-            if (!done || *bad) break;
-            float o[32];
-            const uint32_t to = tb + kTO + 80 * x + lane_off;
-            tmem_ld32(to + 32 * half, o);
-            const float dn = tmem_ld1(to + kDV);
-            tmem_ld_wait();
-            if (row < (x == 0 ? nval0 : nval1)) {
+            if (done && !*bad) {
+                float o[32];
+                const uint32_t to = tb + kTO + 80 * x + lane_off;
+                tmem_ld32(to + 32 * half, o);
+                const float dn = tmem_ld1(to + kDV);
+                tmem_ld_wait();
                 const float rcp = __frcp_rn(dn);
-                float4* dst =
-                    reinterpret_cast<float4*>(A.out + ((int64_t)bh * A.N + t0 + x * kC + row) * kDV + 32 * half);
+                uint8_t* trow = sPhi + (2 * x + half) * kOutTile + row * 128;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    dst[i] = make_float4(o[4 * i] * rcp, o[4 * i + 1] * rcp, o[4 * i + 2] * rcp, o[4 * i + 3] * rcp);
+                    *reinterpret_cast<float4*>(trow + ((i ^ (row & 7)) << 4)) =
+                        make_float4(o[4 * i] * rcp, o[4 * i + 1] * rcp, o[4 * i + 2] * rcp, o[4 * i + 3] * rcp);
+            }
+            ptx::fence_proxy_async_smem();
+            compute_sync();
+            if (tid == 0 && !*bad) {
+                const int y = (int)(t0 + x * kC);
+                ptx::tma_store_3d(&tmo, 0, y, bh, sPhi + (2 * x) * kOutTile);
+                ptx::tma_store_3d(&tmo, 32, y, bh, sPhi + (2 * x + 1) * kOutTile);
+                ptx::bulk_commit();
+                s_out_issued = 1;
             }
         }
         TA_PHASE(0, 9, tid == 0);
@@ -689,6 +706,8 @@ tc_fused_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_co
             if (s_e_issued[x] && !ptx::mbar_wait(&e_loaded[x], 0, kWaitPolls)) s_bad = 1;
         // the last gather (each earlier one completed before the next was issued)
         if (s_gath_issued && !ptx::mbar_wait(&gath, 0, kWaitPolls)) s_bad = 1;
+        // the output stores this thread issued
+        if (s_out_issued) ptx::bulk_wait_all();
         if (s_bad) atomicOr(A.err, kErrPrefillPipe);
     }
     fence_before_sync();
@@ -754,10 +773,12 @@ int try_prefill_fused(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv
     unsigned int* err = device_error_word();
     if (!err) return TAYLOR_ERR_CUDA;
 
-    CUtensorMap tmq, tmk, tmv;
+    CUtensorMap tmq, tmk, tmv, tmo;
     if (make_tmap_bf16_3d(&tmq, q, 16, (uint64_t)N, (uint64_t)BH, 16, kC, 32) != cudaSuccess ||
         make_tmap_bf16_3d(&tmk, k, 16, (uint64_t)N, (uint64_t)BH, 16, kC, 32) != cudaSuccess ||
-        make_tmap_bf16_3d(&tmv, v, kDV, (uint64_t)N, (uint64_t)BH, kDV, 64, 128) != cudaSuccess)
+        make_tmap_bf16_3d(&tmv, v, kDV, (uint64_t)N, (uint64_t)BH, kDV, 64, 128) != cudaSuccess ||
+        make_tmap_f32_3d(&tmo, out, kDV, (uint64_t)N, (uint64_t)BH, (uint64_t)kDV * 4, (uint64_t)N * kDV * 4, 32, kC,
+                         128) != cudaSuccess)
         return kNotApplicable;
 
     // workspace: published chunk states, read-out operands, flags
@@ -799,7 +820,7 @@ int try_prefill_fused(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv
         at[0].val.cooperative = 1;
         cfg.attrs = at;
         cfg.numAttrs = 1;
-        TA_TIMED(stream, "tc_fused_prefill_kernel", e = cudaLaunchKernelEx(&cfg, tc_fused_prefill_kernel, tmq, tmk, tmv, a));
+        TA_TIMED(stream, "tc_fused_prefill_kernel", e = cudaLaunchKernelEx(&cfg, tc_fused_prefill_kernel, tmq, tmk, tmv, tmo, a));
     }
     const cudaError_t e2 = workspace_free(ws, stream);
     if (e == cudaSuccess) e = e2;
