@@ -641,8 +641,9 @@ def run_ours(args, world, rank, local):
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(byts / (cp_med * 1e-3) / 1e9 / hbm_peak, 4),
                              "algorithmic_bytes_per_step": byts,
-                             "note": "same inputs, outputs and state as the main prefill; the three per-degree "
-                                     "read-outs are fp32 CUDA-core work"},
+                             "note": "same inputs, outputs and state as the main prefill; chunk states, scan "
+                                     "and an output kernel with three per-degree TMEM accumulators (tcgen05), "
+                                     "three launches"},
             }
         if "decode" in blocks:
             line["multi_token_decode"] = {

@@ -126,6 +126,9 @@ int centred_prefill_impl(const Tin* q, const Tin* k, const Tin* v, float* out, f
     }
     if (!q || !k || !v || !out) return TAYLOR_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TAYLOR_ERR_MISALIGNED;
+    const int tc = ta::tc::try_centred_prefill(q, k, v, out, state_out, (int)BH, N, d_k, d_v, order, tau, F, stride,
+                                               stream);
+    if (tc != ta::tc::kNotApplicable) return tc;
     const ta::CcPlan plan = ta::plan_prefill_cc((int)BH, N, d_k, d_v, 3, F, stride);
     float* ws = nullptr;
     if (plan.NG > 1 || state_out != nullptr) {

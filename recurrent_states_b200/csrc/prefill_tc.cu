@@ -23,6 +23,7 @@
 // indices: phi = [1, x_i, w_ab x_a x_b (a <= b)], w = sqrt(2) for a < b, 1 for
 // a = b, times tau^m/m! on the query side; degrees >= n are zeroed.
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/taylor_attn.h"
 #include "common.cuh"
@@ -527,6 +528,381 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     TA_PHASE(1, 14, tid == 0);
 }
 
+// ---------------------------------------------------------------- 3'. centred outputs
+// Output kernel of the mean-centred softmax expansion (Su Jianlin's note on the
+// Taylor expansions of logsumexp and softmax, kexue.fm translation 11814,
+// sections "Calculating the Gradient" and "Linear Attention") on the tensor
+// cores, over the n = 3 chunk states of tc_chunk_state (their degree-0, 1 and 2
+// rows hold every prefix sum the expansion needs).  For query i the three
+// read-outs R_m = sum_{j <= i} (q_i . k_j)^m [v_j | 1] (no tau, no 1/m!) go to
+// three TMEM accumulators:
+//   pairwise   P_0 = mask (exact in bf16, shared memory), P_1 = s, P_2 = s^2
+//              (s = q_i . k_j, hi/lo, written over the scores in TMEM), each
+//              times [V | 1 | 0];
+//   carried    phi_m(q) S_<c,m, with the features laid out so that each degree
+//              starts a K step of 16: feature 0 at row 0 (rows 1..15 zero), the
+//              16 of degree 1 at rows 16..31, the 136 of degree 2 at rows
+//              32..167 (168..175 zero).
+// Then, per column,
+//   n = R_0[z], V = R_0[v], qkbar = R_1[z] / n,
+//   sum a v   = tau (R_1[v] - qkbar V),
+//   sum a^2 v = tau^2 (R_2[v] - 2 qkbar R_1[v] + qkbar^2 V),
+//   sum a^2   = tau^2 (R_2[z] - n qkbar^2),
+//   o = V/n + (sum a v)/n  [+ (sum a^2 v - (sum a^2) V/n) / (2n) at order 2].
+constexpr int kFC = 176;                          // features, degree-aligned
+constexpr uint32_t kSboPhiQC = (kFC / 8) * 128;   // Phi_Q: [128][176] K-major
+constexpr uint32_t kCOffQ = 0;
+constexpr uint32_t kCOffK = kCOffQ + kC * kD * 2;
+constexpr uint32_t kCOffV1 = kCOffK + kC * kD * 2;
+constexpr uint32_t kCOffP0 = kCOffV1 + kC * kNV * 2;
+constexpr uint32_t kCOffQh = kCOffP0 + kC * kC * 2;
+constexpr uint32_t kCOffQl = kCOffQh + kC * kFC * 2;
+constexpr uint32_t kCOffS = kCOffQl + kC * kFC * 2;
+constexpr uint32_t kSmemCentred = kCOffS + kFC * 2 * kNV * 2;  // 207,872 bytes
+static_assert(kSmemCentred <= 232448 - 256, "centred chunk_out shared memory");
+// TMEM: scores, then P_1 over them [0, 128); R_0, R_1, R_2 [128, 368); P_2 [368, 496)
+constexpr uint32_t kCR0 = 128, kCP2 = 368;
+
+// padded row of packed feature f (d_k 16, n 3): degree 0 at 0, degrees 1, 2 from 16
+__device__ __forceinline__ int centred_row(int f) { return f == 0 ? 0 : f + 15; }
+
+__global__ void __launch_bounds__(kOutThreads, 1)
+tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+                            const float* __restrict__ W, float* __restrict__ out, int N, int order, float tau,
+                            int F, int64_t stride, int NC, int carried, unsigned int* __restrict__ err) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    __shared__ __align__(8) uint64_t mb_s, mb_o, bar_qk, bar_p, bar_ops;
+    __shared__ uint32_t tslot;
+    __shared__ int mma_fail;
+    uint8_t* sQ = sm + kCOffQ;
+    uint8_t* sK = sm + kCOffK;
+    uint8_t* sV1 = sm + kCOffV1;
+    uint8_t* sP0 = sm + kCOffP0;
+    uint8_t* sQh = sm + kCOffQh;
+    uint8_t* sQl = sm + kCOffQl;
+    uint8_t* sS = sm + kCOffS;  // [176 rows][S hi in column groups 0..9 | lo in 10..19]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, bh = blockIdx.y;
+    const int64_t t0 = (int64_t)c * kC;
+    const int nv = (int)min64(kC, (int64_t)N - t0);
+    const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
+    const bool second = order >= 2;
+
+    if (tid == 0) {
+        ptx::mbar_init(&mb_s, 1);
+        ptx::mbar_init(&mb_o, 1);
+        ptx::mbar_init(&bar_qk, kThreads);
+        ptx::mbar_init(&bar_p, kThreads);
+        ptx::mbar_init(&bar_ops, kThreads);
+        mma_fail = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(&tslot, 512);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = tslot;
+    const uint32_t tA = tbase;  // scores, then P_1
+
+    if (warp == 8) {
+        // ------------------------------------------------ MMA issue (one thread)
+        if (lane == 0) {
+            const uint32_t id = idesc_bf16(128, kNV, 0, 1);
+            const uint64_t bv = smem_desc(sV1, kLboV1, 128);
+            bool good = ptx::mbar_wait(&bar_qk, 0, kWaitPolls);
+            fence_after_sync();
+            if (good) {
+                mma_bf16(tA, smem_desc(sQ, 128, kSboQK), smem_desc(sK, 128, kSboQK), idesc_bf16(128, 128, 0, 0), 0u);
+                mma_commit(&mb_s);
+                // R_0 = P_0 [V | 1 | 0] needs no scores
+                const uint64_t p0 = smem_desc(sP0, 128, kSboP);
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_bf16(tbase + kCR0, p0 + 16 * ks, bv + (2 * kLboV1 / 16) * ks, id, ks > 0 ? 1u : 0u);
+            } else {
+                mma_commit(&mb_s);
+            }
+            if (good) {
+                good = ptx::mbar_wait(&bar_p, 0, kWaitPolls);
+                fence_after_sync();
+                if (good) {
+                    // R_1 = P_1 [V | 1 | 0], R_2 = P_2 [V | 1 | 0]; P of keys 16 ks .. 16 ks + 15:
+                    // hi words at 32 (ks / 2) + 8 (ks % 2), lo 16 further
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks) {
+                        const uint64_t b = bv + (2 * kLboV1 / 16) * ks;
+                        const uint32_t a = 32 * (ks >> 1) + 8 * (ks & 1);
+                        mma_bf16_ts(tbase + kCR0 + 80, tA + a, b, id, ks > 0 ? 1u : 0u);
+                        mma_bf16_ts(tbase + kCR0 + 80, tA + a + 16, b, id, 1u);
+                        if (second) {
+                            mma_bf16_ts(tbase + kCR0 + 160, tbase + kCP2 + a, b, id, ks > 0 ? 1u : 0u);
+                            mma_bf16_ts(tbase + kCR0 + 160, tbase + kCP2 + a + 16, b, id, 1u);
+                        }
+                    }
+                }
+            }
+            if (good && inter) {
+                good = ptx::mbar_wait(&bar_ops, 0, kWaitPolls);
+                fence_after_sync();
+                if (good) {
+                    // K step 0 -> R_0 (Phi_Q of feature 0 is exact: no lo term),
+                    // step 1 -> R_1, steps 2..10 -> R_2
+                    const uint64_t ah = smem_desc(sQh, 128, kSboPhiQC), al = smem_desc(sQl, 128, kSboPhiQC);
+                    const uint64_t sh = smem_desc(sS, kLboS, 128), sl = smem_desc(sS + 10 * 128, kLboS, 128);
+                    const int nks = second ? kFC / 16 : 2;
+#pragma unroll 1
+                    for (int ks = 0; ks < nks; ++ks) {
+                        const uint32_t d = tbase + kCR0 + 80 * min(ks, 2);
+                        const uint64_t bh_ = sh + (2 * kLboS / 16) * ks, bl_ = sl + (2 * kLboS / 16) * ks;
+                        mma_bf16(d, ah + 16 * ks, bh_, id, 1u);
+                        mma_bf16(d, ah + 16 * ks, bl_, id, 1u);
+                        if (ks > 0) mma_bf16(d, al + 16 * ks, bh_, id, 1u);
+                    }
+                }
+            }
+            if (!good) {
+                mma_fail = 1;
+                atomicOr(err, kErrPrefillPipe);
+            }
+            mma_commit(&mb_o);  // tracks every MMA issued, also on the error path
+        }
+    } else {
+        // ------------------------------------------------ operands and epilogue
+        const int row = (warp & 3) * 32 + lane;
+        const int half = warp >> 2;
+        const bool valid = row < nv;
+        const int64_t tok = (int64_t)bh * N + t0 + row;
+
+        // q, k rows (K-major [128][16]); half of [v | 1 | 0] (MN-major [K=128][80]);
+        // row `row` of P_0, keys [64 half, 64 half + 64)
+        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;
+        if (valid) {
+            const uint4* qr = reinterpret_cast<const uint4*>(q + tok * kD);
+            q0 = __ldg(qr);
+            q1 = __ldg(qr + 1);
+        }
+        const uint4* vr = reinterpret_cast<const uint4*>(v + tok * kDV) + half * 4;
+        uint4 val[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) val[g] = valid ? __ldg(vr + g) : make_uint4(0, 0, 0, 0);
+        if (half == 0) {
+            uint4 k0 = make_uint4(0, 0, 0, 0), k1 = k0;
+            if (valid) {
+                const uint4* kr = reinterpret_cast<const uint4*>(k + tok * kD);
+                k0 = __ldg(kr);
+                k1 = __ldg(kr + 1);
+            }
+            *reinterpret_cast<uint4*>(sQ + kmaj(row, 0, kSboQK)) = q0;
+            *reinterpret_cast<uint4*>(sQ + kmaj(row, 1, kSboQK)) = q1;
+            *reinterpret_cast<uint4*>(sK + kmaj(row, 0, kSboQK)) = k0;
+            *reinterpret_cast<uint4*>(sK + kmaj(row, 1, kSboQK)) = k1;
+        } else {
+            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 8, kLboV1)) = make_uint4(valid ? 0x3F80u : 0u, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sV1 + mnmaj(row, 9, kLboV1)) = make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) *reinterpret_cast<uint4*>(sV1 + mnmaj(row, half * 4 + g, kLboV1)) = val[g];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int key = half * 64 + g * 8 + 2 * e;
+                w[e] = (key <= row ? 0x3F80u : 0u) | (key + 1 <= row ? 0x3F800000u : 0u);
+            }
+            *reinterpret_cast<uint4*>(sP0 + kmaj(row, half * 8 + g, kSboP)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&bar_qk);
+
+        // phi(q) for token `row` (multinomial weights only), degree-aligned:
+        // half 0 K steps 0..5, half 1 K steps 6..10
+        if (inter) {
+            float x[16];
+            const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                x[2 * i] = __uint_as_float(w[i] << 16);
+                x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+            }
+            const float e0 = valid ? 1.f : 0.f;
+            auto step = [&](auto kb) {
+                constexpr int KS = decltype(kb)::value;
+                float o[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = 0.f;
+                if (KS == 0) {
+                    o[0] = e0;
+                } else {
+                    // packed features 16 KS - 15 .. 16 KS (feature 160 and beyond stay zero)
+                    constexpr int F0 = 16 * KS - 15, F1 = F0 + 16 > 160 ? 160 : F0 + 16;
+                    float t[F1 - F0];
+                    phi16_range<F0, F1>(x, e0, 1.f, 1.f, t);
+#pragma unroll
+                    for (int i = 0; i < F1 - F0; ++i) o[i] = t[i];
+                }
+                uint4 hi0, lo0, hi1, lo1;
+                split8(o, hi0, lo0);
+                split8(o + 8, hi1, lo1);
+                *reinterpret_cast<uint4*>(sQh + kmaj(row, 2 * KS, kSboPhiQC)) = hi0;
+                *reinterpret_cast<uint4*>(sQh + kmaj(row, 2 * KS + 1, kSboPhiQC)) = hi1;
+                *reinterpret_cast<uint4*>(sQl + kmaj(row, 2 * KS, kSboPhiQC)) = lo0;
+                *reinterpret_cast<uint4*>(sQl + kmaj(row, 2 * KS + 1, kSboPhiQC)) = lo1;
+            };
+            if (half == 0) {
+                step(std::integral_constant<int, 0>());
+                step(std::integral_constant<int, 1>());
+                if (second) {
+                    step(std::integral_constant<int, 2>());
+                    step(std::integral_constant<int, 3>());
+                    step(std::integral_constant<int, 4>());
+                    step(std::integral_constant<int, 5>());
+                }
+            } else if (second) {
+                step(std::integral_constant<int, 6>());
+                step(std::integral_constant<int, 7>());
+                step(std::integral_constant<int, 8>());
+                step(std::integral_constant<int, 9>());
+                step(std::integral_constant<int, 10>());
+            }
+        }
+
+        // P_1 = s, P_2 = s^2 under the causal mask, hi/lo, into TMEM (P_1 over
+        // the scores, each 32-key piece: 16 hi words, then 16 lo words)
+        bool ok = ptx::mbar_wait(&mb_s, 0, kWaitPolls);
+        fence_after_sync();
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+#pragma unroll
+        for (int pc = 0; pc < 2; ++pc) {
+            const uint32_t col = lane_off + 64 * half + 32 * pc;
+            float s[32];
+            tmem_ld32(tA + col, s);
+            tmem_ld_wait();
+            uint32_t h1[16], l1[16], h2[16], l2[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float p1[2], p2[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const bool on = valid && 64 * half + 32 * pc + j + e <= row;
+                    p1[e] = on ? s[j + e] : 0.f;
+                    p2[e] = p1[e] * p1[e];
+                }
+                split2(p1[0], p1[1], h1[j >> 1], l1[j >> 1]);
+                split2(p2[0], p2[1], h2[j >> 1], l2[j >> 1]);
+            }
+            tmem_st16(tA + col, h1);
+            tmem_st16(tA + col + 16, l1);
+            if (second) {
+                tmem_st16(tbase + kCP2 + col, h2);
+                tmem_st16(tbase + kCP2 + col + 16, l2);
+            }
+        }
+        tmem_st_wait();
+        fence_before_sync();
+        ptx::mbar_arrive(&bar_p);
+
+        // the carried state S_<c: produced by the previous grid
+        if (inter) {
+            ptx::pdl_wait_primary();
+            const float* Sg = W + ((int64_t)bh * NC + c) * stride;
+            float4 sa[kSUnits], sb[kSUnits];
+#pragma unroll
+            for (int i = 0; i < kSUnits; ++i) {
+                const int u = tid + i * kThreads, f = u >> 3, g = u & 7;
+                if (f < F) {
+                    sa[i] = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8));
+                    sb[i] = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)f * kDV + g * 8) + 1);
+                } else {
+                    sa[i] = sb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            const float zf = tid < F ? __ldg(Sg + (int64_t)F * kDV + tid) : 0.f;
+#pragma unroll
+            for (int i = 0; i < kSUnits; ++i) {
+                const int u = tid + i * kThreads, f = u >> 3, g = u & 7;
+                if (f < F) {
+                    const float xs[8] = {sa[i].x, sa[i].y, sa[i].z, sa[i].w, sb[i].x, sb[i].y, sb[i].z, sb[i].w};
+                    uint4 hi, lo;
+                    split8(xs, hi, lo);
+                    const int r = centred_row(f);
+                    *reinterpret_cast<uint4*>(sS + mnmaj(r, g, kLboS)) = hi;
+                    *reinterpret_cast<uint4*>(sS + mnmaj(r, 10 + g, kLboS)) = lo;
+                }
+            }
+            if (tid < F) {
+                const float xs[8] = {zf, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                uint4 hi, lo;
+                split8(xs, hi, lo);
+                const int r = centred_row(tid);
+                *reinterpret_cast<uint4*>(sS + mnmaj(r, 8, kLboS)) = hi;
+                *reinterpret_cast<uint4*>(sS + mnmaj(r, 18, kLboS)) = lo;
+                *reinterpret_cast<uint4*>(sS + mnmaj(r, 9, kLboS)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(sS + mnmaj(r, 19, kLboS)) = make_uint4(0, 0, 0, 0);
+            }
+            // the rows no feature maps to: 1..15 and F + 15 .. 175
+            const int nzero = 15 + (kFC - (F + 15));
+            for (int u = tid; u < nzero * 20; u += kThreads) {
+                const int zr = u / 20, g = u % 20;
+                const int r = zr < 15 ? 1 + zr : F + 15 + (zr - 15);
+                *reinterpret_cast<uint4*>(sS + mnmaj(r, g, kLboS)) = make_uint4(0, 0, 0, 0);
+            }
+            fence_before_sync();
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&bar_ops);
+        }
+
+        // epilogue: the combination of R_0, R_1 (, R_2) per column
+        const bool done = ptx::mbar_wait(&mb_o, 0, kWaitPolls);
+        fence_after_sync();
+        ok = ok && done && mma_fail == 0;
+        if (ok) {
+            const uint32_t tr = tbase + kCR0 + lane_off;
+            float a0[32], a1[32], a2[32];
+            tmem_ld32(tr + half * 32, a0);
+            tmem_ld32(tr + 80 + half * 32, a1);
+            const float z0 = tmem_ld1(tr + kDV), z1 = tmem_ld1(tr + 80 + kDV);
+            float z2 = 0.f;
+            if (second) {
+                tmem_ld32(tr + 160 + half * 32, a2);
+                z2 = tmem_ld1(tr + 160 + kDV);
+            }
+            tmem_ld_wait();
+            if (valid) {
+                const float nn = z0, qkbar = z1 / nn, t2 = tau * tau;
+                const float sum_a2 = t2 * (z2 - nn * qkbar * qkbar);
+                float r[32];
+#pragma unroll
+                for (int c2 = 0; c2 < 32; ++c2) {
+                    const float V = a0[c2];
+                    float x = V / nn + tau * (a1[c2] - qkbar * V) / nn;
+                    if (second) {
+                        const float sum_a2v = t2 * (a2[c2] - 2.0f * qkbar * a1[c2] + qkbar * qkbar * V);
+                        x += (sum_a2v - sum_a2 * V / nn) / (2.0f * nn);
+                    }
+                    r[c2] = x;
+                }
+                float4* dst = reinterpret_cast<float4*>(out + tok * kDV + half * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+            }
+        } else {
+            if (tid == 0) atomicOr(err, kErrPrefillPipe);
+            if (!done) ptx::mbar_wait(&mb_o, 0, kWaitPolls);  // one more bound for MMAs in flight
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 8) {
+        fence_after_sync();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
 constexpr int kMaxDevices = 64;
 
 cudaError_t set_smem_once(const void* fn, int bytes, std::once_flag* once, cudaError_t* res) {
@@ -575,6 +951,49 @@ int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloa
         TA_TIMED(stream, "tc_chunk_out_kernel",
                  e = launch_maybe_pdl(tc_chunk_out_kernel, grid, dim3(kOutThreads), kSmemOut, stream, true, q, k, v,
                                       W, out, N, n, tau, (int)F, stride, NC, state_in != nullptr ? 1 : 0, err));
+        if (e == cudaSuccess) e = cudaGetLastError();
+    }
+    const cudaError_t e2 = workspace_free(W, stream);
+    if (e == cudaSuccess) e = e2;
+    if (e == cudaSuccess) return TAYLOR_OK;
+    return e == cudaErrorMemoryAllocation ? TAYLOR_ERR_OUT_OF_MEMORY : TAYLOR_ERR_CUDA;
+}
+
+int try_centred_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, float* out,
+                        float* state_out, int BH, int N, int d, int dv, int order, float tau, int64_t F,
+                        int64_t stride, cudaStream_t stream) {
+    if (d != kD || dv != kDV || F != 153 || N <= 0 || BH <= 0 || (order != 1 && order != 2)) return kNotApplicable;
+    unsigned int* err = device_error_word();
+    if (!err) return TAYLOR_ERR_CUDA;
+
+    static std::once_flag once_a[kMaxDevices], once_c[kMaxDevices];
+    static cudaError_t res_a[kMaxDevices], res_c[kMaxDevices];
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(tc_chunk_state_kernel), (int)kSmemState, once_a, res_a);
+    if (e == cudaSuccess)
+        e = set_smem_once(reinterpret_cast<const void*>(tc_centred_chunk_out_kernel), (int)kSmemCentred, once_c,
+                          res_c);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return TAYLOR_ERR_CUDA;
+    }
+
+    // the n = 3 chunk states and their exclusive scan, as the Taylor prefill forms them
+    const int NC = (N + kC - 1) / kC;
+    const size_t ws_bytes = (size_t)BH * NC * stride * sizeof(float);
+    float* W = nullptr;
+    if (workspace_alloc(reinterpret_cast<void**>(&W), ws_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return TAYLOR_ERR_OUT_OF_MEMORY;
+    }
+    const dim3 grid(NC, BH);
+    TA_TIMED(stream, "tc_chunk_state_kernel",
+             tc_chunk_state_kernel<<<grid, kThreads, kSmemState, stream>>>(k, v, W, N, 3, (int)F, stride, NC, err));
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = launch_state_scan(W, nullptr, state_out, BH, NC, stride, F * (dv + 1), stream, true);
+    if (e == cudaSuccess) {
+        TA_TIMED(stream, "tc_centred_chunk_out_kernel",
+                 e = launch_maybe_pdl(tc_centred_chunk_out_kernel, grid, dim3(kOutThreads), kSmemCentred, stream, true,
+                                      q, k, v, (const float*)W, out, N, order, tau, (int)F, stride, NC, 0, err));
         if (e == cudaSuccess) e = cudaGetLastError();
     }
     const cudaError_t e2 = workspace_free(W, stream);

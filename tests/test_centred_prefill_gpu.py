@@ -97,3 +97,21 @@ def test_centred_prefill_empty_and_invalid():
     with pytest.raises(TA.TaylorAttnError) as ei:
         TA.taylor_attn_centred_prefill(q.to(DEV), k.to(DEV), v.to(DEV), 3, 2.0)
     assert ei.value.status == TA.TAYLOR_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("order", [1, 2])
+@pytest.mark.parametrize("B,H,N", [(1, 1, 1), (1, 2, 2), (1, 1, 127), (2, 1, 128), (1, 2, 129), (3, 2, 1000)])
+def test_centred_prefill_tensor_core_shapes(B, H, N, order):
+    """bf16 d_k 16 d_v 64 takes the tensor-core kernel: single-chunk,
+    chunk-edge and many-chunk lengths against the per-row definition, the
+    state against the n = 3 Taylor state."""
+    tau = 2.0
+    q, k, v = synth.qkv(B, H, N, 16, 64, seed=100 + N + order, dtype="bf16")
+    out, st = _run("bf16", q, k, v, order, tau)
+    ref = O.centred_direct(f64(q), f64(k), f64(v), order, tau)
+    err = row_scaled_max_err(f64(out), ref)
+    print(f"centred prefill (tensor cores) {B}x{H}x{N} order {order}: {err:.3g}")
+    assert err <= TOL["bf16"]
+    assert state_block_errors(st, T.state_of(f64(k), f64(v), 3), 16, 64, 3) <= TOL["bf16"]
+    # a row of one token returns its value
+    np.testing.assert_allclose(f64(out)[..., 0, :], f64(v)[..., 0, :], rtol=1e-5, atol=1e-6)
