@@ -5,6 +5,8 @@ a capture can skip the first (cold) launches.
     python -m recurrent_states_b200.profile_cases <case>
 
 prefill  the main prefill, B1 H8 N4096 d_k 16 d_v 64 n 3 (tc_fused_prefill_kernel)
+cprefill the order-2 mean-centred prefill of the same inputs (tc_chunk_state_kernel,
+         scan_kernel, tc_centred_chunk_out_kernel)
 decode   one decode step on 1,024 random states, B64 H16 (decode_ws_kernel)
 centred  the same with the order-2 mean-centred read-out (decode_ws_kernel<.., 1>)
 multi4   4 new tokens per head on those states (decode_multi_ws_kernel)
@@ -18,7 +20,7 @@ import torch
 from . import synth
 from . import taylor_attn as TA
 
-CASES = ("prefill", "decode", "centred", "multi4", "multi16", "large")
+CASES = ("prefill", "cprefill", "decode", "centred", "multi4", "multi16", "large")
 
 
 def run(case: str, calls: int = 4) -> float:
@@ -35,12 +37,15 @@ def run(case: str, calls: int = 4) -> float:
         out = torch.empty((64, 16, T, dv), device=dev)
         for _ in range(calls):
             TA.taylor_attn_prefill_from_state(q, k, v, st, n, tau, out=out, state_out=st)
-    elif case == "prefill":
+    elif case in ("prefill", "cprefill"):
         q, k, v = (t.to(dev) for t in synth.qkv(1, 8, 4096, d, dv, seed=0))
         out = torch.empty((1, 8, 4096, dv), device=dev)
         st = torch.empty((1, 8, stride), device=dev)
         for _ in range(calls):
-            TA.taylor_attn_prefill(q, k, v, n, tau, out=out, state_out=st)
+            if case == "prefill":
+                TA.taylor_attn_prefill(q, k, v, n, tau, out=out, state_out=st)
+            else:
+                TA.taylor_attn_centred_prefill(q, k, v, 2, tau, out=out, state_out=st)
     elif case == "large":
         dl = 64
         q, k, v = (t.to(dev) for t in synth.qkv(1, 8, 32768, dl, dv, seed=3))
