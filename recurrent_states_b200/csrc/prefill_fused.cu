@@ -165,7 +165,6 @@ __device__ __forceinline__ void init_ones(uint8_t* atom, int tid, int nthreads) 
 }
 
 struct FusedArgs {
-    float* out;
     const float* state_in;
     float* state_out;
     float* TG;        // [BH][NS][160][68] published states, one per CTA (its chunks together)
@@ -792,7 +791,6 @@ int try_prefill_fused(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv
         return TAYLOR_ERR_OUT_OF_MEMORY;
     }
     FusedArgs a;
-    a.out = out;
     a.state_in = state_in;
     a.state_out = state_out;
     a.TG = reinterpret_cast<float*>(ws);
