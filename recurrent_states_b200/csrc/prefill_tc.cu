@@ -562,6 +562,10 @@ constexpr uint32_t kSmemCentred = kCOffS + kFC * 2 * kNV * 2;  // 207,872 bytes
 static_assert(kSmemCentred <= 232448 - 256, "centred chunk_out shared memory");
 // TMEM: scores, then P_1 over them [0, 128); R_0, R_1, R_2 [128, 368); P_2 [368, 496)
 constexpr uint32_t kCR0 = 128, kCP2 = 368;
+// chunks per CTA, one after the other on the same operand space and TMEM (the
+// main workload's 256 chunks then fit one wave, and the second chunk runs on
+// fetched code)
+constexpr int kCentredChunks = 2;
 
 // padded row of packed feature f (d_k 16, n 3): degree 0 at 0, degrees 1, 2 from 16
 __device__ __forceinline__ int centred_row(int f) { return f == 0 ? 0 : f + 15; }
@@ -583,10 +587,7 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
     uint8_t* sS = sm + kCOffS;  // [176 rows][S hi in column groups 0..9 | lo in 10..19]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, bh = blockIdx.y;
-    const int64_t t0 = (int64_t)c * kC;
-    const int nv = (int)min64(kC, (int64_t)N - t0);
-    const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
+    const int bh = blockIdx.y;
     const bool second = order >= 2;
 
     if (tid == 0) {
@@ -611,9 +612,15 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
     if (warp == 8) {
         // ------------------------------------------------ MMA issue (one thread)
         if (lane == 0) {
+          uint32_t ops_ph = 0;  // bar_ops completes a phase only for chunks with a carried state
+          for (int x = 0; x < kCentredChunks; ++x) {
+            const int c = kCentredChunks * blockIdx.x + x;
+            if (c >= NC) break;
+            const uint32_t ph = (uint32_t)x & 1u;
+            const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
             const uint32_t id = idesc_bf16(128, kNV, 0, 1);
             const uint64_t bv = smem_desc(sV1, kLboV1, 128);
-            bool good = ptx::mbar_wait(&bar_qk, 0, kWaitPolls);
+            bool good = ptx::mbar_wait(&bar_qk, ph, kWaitPolls);
             fence_after_sync();
             if (good) {
                 mma_bf16(tA, smem_desc(sQ, 128, kSboQK), smem_desc(sK, 128, kSboQK), idesc_bf16(128, 128, 0, 0), 0u);
@@ -627,7 +634,7 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
                 mma_commit(&mb_s);
             }
             if (good) {
-                good = ptx::mbar_wait(&bar_p, 0, kWaitPolls);
+                good = ptx::mbar_wait(&bar_p, ph, kWaitPolls);
                 fence_after_sync();
                 if (good) {
                     // R_1 = P_1 [V | 1 | 0], R_2 = P_2 [V | 1 | 0]; P of keys 16 ks .. 16 ks + 15:
@@ -646,7 +653,8 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
                 }
             }
             if (good && inter) {
-                good = ptx::mbar_wait(&bar_ops, 0, kWaitPolls);
+                good = ptx::mbar_wait(&bar_ops, ops_ph, kWaitPolls);
+                ops_ph ^= 1u;
                 fence_after_sync();
                 if (good) {
                     // K step 0 -> R_0 (Phi_Q of feature 0 is exact: no lo term),
@@ -669,11 +677,19 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
                 atomicOr(err, kErrPrefillPipe);
             }
             mma_commit(&mb_o);  // tracks every MMA issued, also on the error path
+          }
         }
     } else {
         // ------------------------------------------------ operands and epilogue
         const int row = (warp & 3) * 32 + lane;
         const int half = warp >> 2;
+        for (int x = 0; x < kCentredChunks; ++x) {
+        const int c = kCentredChunks * blockIdx.x + x;
+        if (c >= NC) break;
+        const uint32_t ph = (uint32_t)x & 1u;
+        const int64_t t0 = (int64_t)c * kC;
+        const int nv = (int)min64(kC, (int64_t)N - t0);
+        const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
         const bool valid = row < nv;
         const int64_t tok = (int64_t)bh * N + t0 + row;
 
@@ -706,8 +722,9 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) *reinterpret_cast<uint4*>(sV1 + mnmaj(row, half * 4 + g, kLboV1)) = val[g];
+        // (the causal mask is the same for every chunk)
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
+        for (int g = 0; g < 8 && x == 0; ++g) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -717,6 +734,7 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
             *reinterpret_cast<uint4*>(sP0 + kmaj(row, half * 8 + g, kSboP)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         ptx::fence_proxy_async_smem();
+        fence_before_sync();  // the previous chunk's TMEM loads, before its accumulators are rewritten
         ptx::mbar_arrive(&bar_qk);
 
         // phi(q) for token `row` (multinomial weights only), degree-aligned:
@@ -773,7 +791,7 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
 
         // P_1 = s, P_2 = s^2 under the causal mask, hi/lo, into TMEM (P_1 over
         // the scores, each 32-key piece: 16 hi words, then 16 lo words)
-        bool ok = ptx::mbar_wait(&mb_s, 0, kWaitPolls);
+        bool ok = ptx::mbar_wait(&mb_s, ph, kWaitPolls);
         fence_after_sync();
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
 #pragma unroll
@@ -857,42 +875,47 @@ tc_centred_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__
         }
 
         // epilogue: the combination of R_0, R_1 (, R_2) per column
-        const bool done = ptx::mbar_wait(&mb_o, 0, kWaitPolls);
+        const bool done = ptx::mbar_wait(&mb_o, ph, kWaitPolls);
         fence_after_sync();
         ok = ok && done && mma_fail == 0;
         if (ok) {
             const uint32_t tr = tbase + kCR0 + lane_off;
-            float a0[32], a1[32], a2[32];
-            tmem_ld32(tr + half * 32, a0);
-            tmem_ld32(tr + 80 + half * 32, a1);
             const float z0 = tmem_ld1(tr + kDV), z1 = tmem_ld1(tr + 80 + kDV);
-            float z2 = 0.f;
-            if (second) {
-                tmem_ld32(tr + 160 + half * 32, a2);
-                z2 = tmem_ld1(tr + 160 + kDV);
-            }
+            const float z2 = second ? tmem_ld1(tr + 160 + kDV) : 0.f;
             tmem_ld_wait();
-            if (valid) {
-                const float nn = z0, qkbar = z1 / nn, t2 = tau * tau;
-                const float sum_a2 = t2 * (z2 - nn * qkbar * qkbar);
-                float r[32];
+            const float nn = z0, qkbar = z1 / nn, t2 = tau * tau;
+            const float sum_a2 = t2 * (z2 - nn * qkbar * qkbar);
+            // 16 columns at a time
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                const uint32_t cc = half * 32 + cb * 16;
+                float a0[16], a1[16], a2[16];
+                tmem_ld16(tr + cc, a0);
+                tmem_ld16(tr + 80 + cc, a1);
+                if (second) tmem_ld16(tr + 160 + cc, a2);
+                tmem_ld_wait();
+                if (valid) {
+                    float r[16];
 #pragma unroll
-                for (int c2 = 0; c2 < 32; ++c2) {
-                    const float V = a0[c2];
-                    float x = V / nn + tau * (a1[c2] - qkbar * V) / nn;
-                    if (second) {
-                        const float sum_a2v = t2 * (a2[c2] - 2.0f * qkbar * a1[c2] + qkbar * qkbar * V);
-                        x += (sum_a2v - sum_a2 * V / nn) / (2.0f * nn);
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        const float V = a0[c2];
+                        float xo = V / nn + tau * (a1[c2] - qkbar * V) / nn;
+                        if (second) {
+                            const float sum_a2v = t2 * (a2[c2] - 2.0f * qkbar * a1[c2] + qkbar * qkbar * V);
+                            xo += (sum_a2v - sum_a2 * V / nn) / (2.0f * nn);
+                        }
+                        r[c2] = xo;
                     }
-                    r[c2] = x;
-                }
-                float4* dst = reinterpret_cast<float4*>(out + tok * kDV + half * 32);
+                    float4* dst = reinterpret_cast<float4*>(out + tok * kDV + cc);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+                }
             }
         } else {
             if (tid == 0) atomicOr(err, kErrPrefillPipe);
-            if (!done) ptx::mbar_wait(&mb_o, 0, kWaitPolls);  // one more bound for MMAs in flight
+            if (!done) ptx::mbar_wait(&mb_o, ph, kWaitPolls);  // one more bound for MMAs in flight
+        }
         }
     }
     fence_before_sync();
@@ -991,8 +1014,9 @@ int try_centred_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __
     e = cudaGetLastError();
     if (e == cudaSuccess) e = launch_state_scan(W, nullptr, state_out, BH, NC, stride, F * (dv + 1), stream, true);
     if (e == cudaSuccess) {
+        const dim3 grid_o((NC + kCentredChunks - 1) / kCentredChunks, BH);
         TA_TIMED(stream, "tc_centred_chunk_out_kernel",
-                 e = launch_maybe_pdl(tc_centred_chunk_out_kernel, grid, dim3(kOutThreads), kSmemCentred, stream, true,
+                 e = launch_maybe_pdl(tc_centred_chunk_out_kernel, grid_o, dim3(kOutThreads), kSmemCentred, stream, true,
                                       q, k, v, (const float*)W, out, N, order, tau, (int)F, stride, NC, 0, err));
         if (e == cudaSuccess) e = cudaGetLastError();
     }

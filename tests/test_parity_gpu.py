@@ -452,7 +452,8 @@ def test_multi_token_decode_many_heads(dtype, d, n):
 
 
 @pytest.mark.parametrize("d,n,T,inplace", [(8, 3, 16, True), (16, 1, 9, True), (16, 3, 10, False),
-                                           (16, 3, 13, False), (24, 2, 12, True), (16, 3, 6, False)])
+                                           (16, 3, 13, False), (24, 2, 12, True), (16, 3, 6, False),
+                                           (16, 2, 11, True), (16, 3, 16, True)])
 def test_multi_token_decode_tensor_core_shapes(d, n, T, inplace):
     """The tensor-core multi-token kernel (more than 8 tokens per call) over
     its range (F = 45, 1, 153, 153, 25; ragged T; in place and into a separate
