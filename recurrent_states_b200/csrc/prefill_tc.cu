@@ -22,6 +22,7 @@
 // The feature map for d_k = 16 is evaluated in closed form with compile-time
 // indices: phi = [1, x_i, w_ab x_a x_b (a <= b)], w = sqrt(2) for a < b, 1 for
 // a = b, times tau^m/m! on the query side; degrees >= n are zeroed.
+#include <algorithm>
 #include <mutex>
 #include <type_traits>
 
@@ -248,7 +249,7 @@ constexpr int kSUnits = kFP * 8 / kThreads;  // 8-column units of S_v per thread
 __global__ void __launch_bounds__(kOutThreads, 1)
 tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                     const float* __restrict__ W, float* __restrict__ out, int N, int n, float tau, int F,
-                    int64_t stride, int NC, int carried, unsigned int* __restrict__ err) {
+                    int64_t stride, int NC, int carried, int cpc, unsigned int* __restrict__ err) {
     extern __shared__ __align__(1024) uint8_t sm[];
     __shared__ __align__(8) uint64_t mb_s, mb_o, bar_qk, bar_p, bar_ops;
     __shared__ uint32_t tslot;
@@ -263,10 +264,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     uint8_t* sS = sm + kOffSh;  // S hi in column groups 0..9, lo in 10..19 (the Sh and Sl space)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, bh = blockIdx.y;
-    const int64_t t0 = (int64_t)c * kC;
-    const int nv = (int)min64(kC, (int64_t)N - t0);
-    const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
+    const int bh = blockIdx.y;
     TA_PHASE(1, 0, tid == 0);
     TA_PHASE(2, warp, lane == 0);
 
@@ -296,16 +294,22 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
     if (warp == 8) {
         // ------------------------------------------------ MMA issue (one thread)
         if (lane == 0) {
+          uint32_t ops_ph = 0;  // bar_ops completes a phase only for chunks with a carried state
+          for (int x = 0; x < cpc; ++x) {
+            const int c = cpc * blockIdx.x + x;
+            if (c >= NC) break;
+            const uint32_t ph = (uint32_t)x & 1u;
+            const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
             // descriptors are built once and advanced by constants (16-byte units)
             const uint32_t id = idesc_bf16(128, kNV, 0, 1);
             const uint32_t id160 = idesc_bf16(128, 2 * kNV, 0, 1);
-            bool good = ptx::mbar_wait(&bar_qk, 0, kWaitPolls);
+            bool good = ptx::mbar_wait(&bar_qk, ph, kWaitPolls);
             fence_after_sync();
             if (good)
                 mma_bf16(tA, smem_desc(sQ, 128, kSboQK), smem_desc(sK, 128, kSboQK), idesc_bf16(128, 128, 0, 0), 0u);
             mma_commit(&mb_s);
             if (good) {
-                good = ptx::mbar_wait(&bar_p, 0, kWaitPolls);
+                good = ptx::mbar_wait(&bar_p, ph, kWaitPolls);
                 fence_after_sync();
                 TA_PHASE(1, 11, true);
                 if (good) {
@@ -320,7 +324,8 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
                 }
             }
             if (good && inter) {
-                good = ptx::mbar_wait(&bar_ops, 0, kWaitPolls);
+                good = ptx::mbar_wait(&bar_ops, ops_ph, kWaitPolls);
+                ops_ph ^= 1u;
                 fence_after_sync();
                 TA_PHASE(1, 12, true);
                 if (good) {
@@ -340,11 +345,19 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
             }
             mma_commit(&mb_o);  // tracks every MMA issued, also on the error path
             TA_PHASE(1, 13, true);
+          }
         }
     } else {
         // ------------------------------------------------ operands and epilogue
         const int row = (warp & 3) * 32 + lane;
         const int half = warp >> 2;
+        for (int x = 0; x < cpc; ++x) {
+        const int c = cpc * blockIdx.x + x;
+        if (c >= NC) break;
+        const uint32_t ph = (uint32_t)x & 1u;
+        const int64_t t0 = (int64_t)c * kC;
+        const int nv = (int)min64(kC, (int64_t)N - t0);
+        const bool inter = c > 0 || carried != 0;   // S_<c is non-zero
         const bool valid = row < nv;
         const int64_t tok = (int64_t)bh * N + t0 + row;
 
@@ -377,6 +390,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
 #pragma unroll
         for (int g = 0; g < 4; ++g) *reinterpret_cast<uint4*>(sV1 + mnmaj(row, half * 4 + g, kLboV1)) = val[g];
         ptx::fence_proxy_async_smem();
+        fence_before_sync();  // the previous chunk's TMEM loads, before its accumulators are rewritten
         ptx::mbar_arrive(&bar_qk);
         TA_PHASE(1, 2, tid == 0);
 
@@ -400,7 +414,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
         TA_PHASE(1, 3, tid == 0);
 
         // pairwise weights P = poly(tau q.k) under the causal mask, hi/lo, K-major
-        bool ok = ptx::mbar_wait(&mb_s, 0, kWaitPolls);
+        bool ok = ptx::mbar_wait(&mb_s, ph, kWaitPolls);
         fence_after_sync();
         TA_PHASE(1, 4, tid == 0);
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -488,7 +502,7 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
         }
 
         // epilogue: o = numerator * (1 / denominator)
-        const bool done = ptx::mbar_wait(&mb_o, 0, kWaitPolls);
+        const bool done = ptx::mbar_wait(&mb_o, ph, kWaitPolls);
         fence_after_sync();
         TA_PHASE(1, 8, tid == 0);
         ok = ok && done && mma_fail == 0;
@@ -515,9 +529,10 @@ tc_chunk_out_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
             }
         } else {
             if (tid == 0) atomicOr(err, kErrPrefillPipe);
-            if (!done) ptx::mbar_wait(&mb_o, 0, kWaitPolls);  // one more bound for MMAs in flight
+            if (!done) ptx::mbar_wait(&mb_o, ph, kWaitPolls);  // one more bound for MMAs in flight
         }
         TA_PHASE(1, 9, tid == 0);
+        }
     }
     fence_before_sync();
     __syncthreads();
@@ -971,9 +986,20 @@ int try_prefill(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloa
     e = cudaGetLastError();
     if (e == cudaSuccess) e = launch_state_scan(W, state_in, state_out, BH, NC, stride, F * (dv + 1), stream, true);
     if (e == cudaSuccess) {
+        // up to four chunks a CTA (one after another), so that a call with more
+        // chunks than SMs runs in fewer waves and later chunks on fetched code
+        int sms = 148;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            sms = 148;
+        }
+        const int64_t total = (int64_t)NC * BH;
+        const int cpc = (int)std::min<int64_t>(4, std::max<int64_t>(1, (total + sms - 1) / sms));
+        const dim3 grid_o((NC + cpc - 1) / cpc, BH);
         TA_TIMED(stream, "tc_chunk_out_kernel",
-                 e = launch_maybe_pdl(tc_chunk_out_kernel, grid, dim3(kOutThreads), kSmemOut, stream, true, q, k, v,
-                                      W, out, N, n, tau, (int)F, stride, NC, state_in != nullptr ? 1 : 0, err));
+                 e = launch_maybe_pdl(tc_chunk_out_kernel, grid_o, dim3(kOutThreads), kSmemOut, stream, true, q, k, v,
+                                      W, out, N, n, tau, (int)F, stride, NC, state_in != nullptr ? 1 : 0, cpc, err));
         if (e == cudaSuccess) e = cudaGetLastError();
     }
     const cudaError_t e2 = workspace_free(W, stream);
