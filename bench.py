@@ -50,7 +50,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (6 x 40.8 MB > the 126 MB L2)
 DECODE_BUFFERS = 6
 DECODE_GRAPH_STEPS = 100  # dependent decode steps per CUDA-graph replay
-E2E_GROUPS = 4  # head groups of the end-to-end pipeline
+E2E_GROUPS = 2  # head groups of the end-to-end pipeline
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a
