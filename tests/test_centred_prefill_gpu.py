@@ -115,3 +115,12 @@ def test_centred_prefill_tensor_core_shapes(B, H, N, order):
     assert state_block_errors(st, T.state_of(f64(k), f64(v), 3), 16, 64, 3) <= TOL["bf16"]
     # a row of one token returns its value
     np.testing.assert_allclose(f64(out)[..., 0, :], f64(v)[..., 0, :], rtol=1e-5, atol=1e-6)
+
+
+def test_centred_prefill_tensor_core_without_state_out():
+    """The tensor-core path with no state requested gives the same outputs."""
+    q, k, v = synth.qkv(2, 3, 700, 16, 64, seed=77, dtype="bf16")
+    out, st = _run("bf16", q, k, v, 2, 2.0, state=False)
+    assert st is None
+    ref = O.centred_direct(f64(q), f64(k), f64(v), 2, 2.0)
+    assert row_scaled_max_err(f64(out), ref) <= TOL["bf16"]
