@@ -198,10 +198,12 @@ TAYLOR_API int taylor_attn_centred_decode_f32(const float* q, const float* k, co
  * Taylor state of the N tokens ([B][H][taylor_attn_state_stride(d_k, d_v,
  * 3)]), from which taylor_attn_centred_decode (or taylor_attn_decode with
  * n = 3) continues.  The three per-degree read-outs sum_j (q_i.k_j)^m [v_j | 1]
- * (m = 0, 1, 2) are accumulated in fp32 on CUDA cores, pairwise inside a token
- * group and through the group's exclusive n = 3 state across groups, and
- * combined per column.  order is 1 or 2 (else TAYLOR_ERR_UNSUPPORTED); sizes,
- * alignment and workspace as taylor_attn_prefill. */
+ * (m = 0, 1, 2) are accumulated apart, pairwise inside a chunk or token group
+ * and through the exclusive n = 3 state before it, and combined per column in
+ * fp32: with bf16 inputs, d_k 16 and d_v 64 on the tensor cores (hi/lo bf16
+ * operands, fp32 accumulators), else in fp32 on CUDA cores.  order is 1 or 2
+ * (else TAYLOR_ERR_UNSUPPORTED); sizes, alignment and workspace as
+ * taylor_attn_prefill. */
 TAYLOR_API int taylor_attn_centred_prefill(const void* q, const void* k, const void* v, float* out,
                                            float* state_out, int B, int H, int N, int d_k, int d_v, int order,
                                            float tau, cudaStream_t stream);
