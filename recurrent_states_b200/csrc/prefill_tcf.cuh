@@ -125,8 +125,8 @@ __device__ __forceinline__ void init_ones_atom(uint8_t* atom, int tid, int nthre
 // its rows, so that k loads run several stages ahead of the evaluation.
 template <int D>
 struct StSm {
-    static constexpr int kSlots = 4;
-    static constexpr int kKSlots = 6;
+    static constexpr int kSlots = 2;
+    static constexpr int kKSlots = 2;
     static constexpr uint32_t kK = kTok * D * 2;  // k rows, swizzled K-major
     static constexpr uint32_t kPhiBase = 0;
     static constexpr uint32_t kV1Base = kSlots * 2 * kPhiBytes;
@@ -139,7 +139,7 @@ struct StSm {
 constexpr int kStateThreads = kCompute + 32;
 
 template <int D, int N>
-__global__ void __launch_bounds__(kStateThreads, 1)
+__global__ void __launch_bounds__(kStateThreads, 2)
 tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  float* __restrict__ W, int Ntok, int n, int F, int64_t stride, int G, int NG,
                  unsigned int* __restrict__ err) {
@@ -716,6 +716,10 @@ int run(const bf16* q, const bf16* k, const bf16* v, float* out, const float* st
     std::call_once(once[dev], [&]() {
         res[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(tcf_state_kernel<D, N>),
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StSm<D>::kBytes);
+        // two CTAs an SM (each allocates 128 TMEM columns): the largest shared-memory carveout
+        if (res[dev] == cudaSuccess)
+            res[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(tcf_state_kernel<D, N>),
+                                            cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (res[dev] == cudaSuccess)
             res[dev] = cudaFuncSetAttribute(reinterpret_cast<const void*>(tcf_out_kernel<D, N>),
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSm<D>::kBytes);
