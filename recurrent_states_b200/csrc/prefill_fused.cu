@@ -23,7 +23,8 @@
 //      total into state_out), then raises the head's count of scanned rows;
 //   5. once that count reaches F, the CTA pulls its operand E_s with a bulk
 //      copy, evaluates c (.) Phi_Q,x into TMEM and adds (c (.) Phi_Q,x) E_s to
-//      O_x of both its chunks; o = O[:, :64] / O[:, 64].
+//      O_x of both its chunks; o = O[:, :64] / O[:, 64], staged in shared
+//      memory and written by TMA tensor stores.
 // The launch is cooperative, so all CTAs that wait on one another's flags are
 // resident together; every flag wait and every mbarrier wait is bounded, and
 // a wait that runs out sets a device error bit and skips the work that
@@ -37,8 +38,10 @@
 //
 // Roles: warps 0-7 (two per TMEM lane quadrant; thread = token or query row,
 // `half` = which half of the features or keys) evaluate Phi_K, P and Phi_Q,
-// publish the chunk states, do the scan for the groups this CTA owns and run
-// the epilogue; lane 0 of warp 8 issues the TMA loads and every tcgen05.mma.
+// stage the CTA's state, do the scan for the rows this CTA owns and run the
+// epilogue; lane 0 of warp 8 issues the TMA loads and every tcgen05.mma;
+// lane 0 of warp 9 publishes the state, gathers the scan's rows and loads
+// the read-out operand.
 #include <mutex>
 #include <type_traits>
 
