@@ -380,6 +380,24 @@ def test_prefill_from_state_continues_the_sequence(dtype, d, dv, n, N, cut):
     assert torch.equal(st2, st)
 
 
+@pytest.mark.parametrize("n", [1, 3])
+def test_several_chunks_per_cta_three_launch_prefill_from_a_carried_state(n):
+    """The three-launch prefill with several chunks per output CTA (B1 H8,
+    6,000 new tokens: 47 chunks a head, 376 in all, three a CTA, the last
+    CTA of a head with two) continuing from the state of a 2,000-token prefix:
+    outputs of the tail and the final state against the oracle's recursion."""
+    B, H, d, dv, tau, cut, N = 1, 8, 16, 64, 2.0, 2000, 8000
+    q, k, v = synth.qkv(B, H, N, d, dv, seed=91 + n, dtype="bf16")
+    h = lambda t: t[:, :, :cut].contiguous().to(DEV)  # noqa: E731
+    t_ = lambda t: t[:, :, cut:].contiguous().to(DEV)  # noqa: E731
+    _, st_head = TA.taylor_attn_prefill(h(q), h(k), h(v), n, tau, state_out=True)
+    out_tail, st = TA.taylor_attn_prefill_from_state(t_(q), t_(k), t_(v), st_head, n, tau, state_out=True)
+    torch.cuda.synchronize()
+    ref_out, ref_st = C.recurrent(f64(q), f64(k), f64(v), n, tau)
+    assert row_scaled_max_err(f64(out_tail), ref_out[:, :, cut:]) <= TOL["bf16"]
+    assert state_block_errors(st, ref_st, d, dv, n) <= TOL["bf16"]
+
+
 def test_two_chunks_per_cta_prefill_from_a_carried_state():
     """The one-launch prefill with two chunks per CTA (B1 H8, 3,900 new tokens:
     31 chunks, 16 CTAs per head, the last with one ragged chunk) continuing
