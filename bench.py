@@ -238,7 +238,8 @@ def run_ours(args, world, rank, local):
         # a spin kernel ahead of the timed work, outside every event pair, so
         # that the host has enqueued the steps before the device reaches them:
         # the events then time the device's work, not the host's launch rate
-        torch.cuda._sleep(int(LEAD_CYCLES_PER_STEP * steps))
+        if hasattr(torch.cuda, "_sleep"):
+            torch.cuda._sleep(int(LEAD_CYCLES_PER_STEP * steps))
 
     def timed(run, steps, flushed=True, kernels=False):
         """Enqueues run(i) for i < steps, each bracketed by events (L2 flushed
