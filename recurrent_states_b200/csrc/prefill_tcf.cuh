@@ -9,9 +9,9 @@
 //   1. tcf_state_kernel (group, 128-feature tile, head):
 //        dS_g[tile, :] = Phi_K[:, tile]^T (128 x G) . [V|1|0] (G x 80),
 //        accumulated in TMEM over 64-token stages;
-//   2. the exclusive scan over groups (shared with the other paths);
-//   3. tcf_pack_kernel: each S_<g cut into 64-feature read-out operand tiles,
-//      split into hi/lo bf16 once per group rather than once per query tile;
+//   2, 3. tcf_scan_pack_kernel: the exclusive scan over groups, each prefix
+//      S_<g written straight as 64-feature read-out operand tiles, split
+//      into hi/lo bf16 once per group rather than once per query tile;
 //   4. tcf_out_kernel (128 queries, head):
 //        O = sum over 64-key tiles of the group up to the diagonal of
 //              (poly(tau Q K^T) (.) mask) [V|1|0]
@@ -306,33 +306,69 @@ tcf_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
 }
 
-// ---------------------------------------------------------------- 3. read-out operand tiles
-// S_<g (fp32, the library's state layout) -> for each 64-feature tile r one
-// MN-major bf16 operand [K = 64 features][N = 160]: columns 0..79 the hi
-// parts, 80..159 the lo parts, of [S_v row | z | 0 ...]; features past F zero.
+// ---------------------------------------------------------------- 2 + 3. scan and operand tiles in one pass
+// The exclusive scan over the NG group states of a head fused with their
+// packing into read-out operand tiles: S_<g (fp32, the library's state
+// layout) becomes, for each 64-feature tile r, one MN-major bf16 operand
+// [K = 64 features][N = 160] (columns 0..79 the hi parts, 80..159 the lo
+// parts, of [S_v row | z | 0 ...]; features past F zero).  A thread owns 8 columns of one feature
+// row (its 16-byte unit of a tile row, hi and lo) and walks the groups,
+// writing the prefix before group g as group g's tile unit, then adding group
+// g's state.  The group states are read once and the exclusive prefixes never
+// go back to memory; the total goes to state_out (padding zero-filled by the
+// head's first block).  Units are ordered so that 8 consecutive threads fill
+// one 128-byte line of a tile (8 feature rows of one column group).
 __global__ void __launch_bounds__(256)
-tcf_pack_kernel(const float* __restrict__ W, uint8_t* __restrict__ PK, int F, int64_t stride, int NG, int R,
-                int g0) {
-    ptx::pdl_launch_dependents();
+tcf_scan_pack_kernel(const float* __restrict__ W, const float* __restrict__ state_in, float* __restrict__ state_out,
+                     uint8_t* __restrict__ PK, int F, int64_t stride, int NG, int R, int g0) {
     ptx::pdl_wait_primary();
-    const int r = blockIdx.x, g = g0 + blockIdx.y, bh = blockIdx.z;
-    const float* S = W + ((int64_t)bh * NG + g) * stride;
-    uint8_t* dst = PK + (((int64_t)bh * NG + g) * R + r) * kSTile;
-    for (int u = threadIdx.x; u < kRT * 10; u += 256) {
-        const int gq = u / kRT, j = u % kRT, f = r * kRT + j;
-        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (f < F) {
+    ptx::pdl_launch_dependents();
+    const int bh = blockIdx.y;
+    const int u = blockIdx.x * 256 + threadIdx.x;
+    const int f8 = u / 80, rem = u % 80, gq = rem >> 3, f = f8 * 8 + (rem & 7);
+    if (f < R * kRT) {
+        const int r = f / kRT, j = f % kRT;
+        const bool live = f < F && gq < 9;
+        const float* Sb = W + (int64_t)bh * NG * stride;
+        float run[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        auto ld8 = [&](const float* S, float (&x)[8]) {
             if (gq < 8) {
                 const float4 a = __ldg(reinterpret_cast<const float4*>(S + (int64_t)f * kDV + gq * 8));
                 const float4 b = __ldg(reinterpret_cast<const float4*>(S + (int64_t)f * kDV + gq * 8) + 1);
                 x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
                 x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-            } else if (gq == 8) {
+            } else {
                 x[0] = __ldg(S + (int64_t)F * kDV + f);
+#pragma unroll
+                for (int i = 1; i < 8; ++i) x[i] = 0.f;
+            }
+        };
+        if (live && state_in) ld8(state_in + (int64_t)bh * stride, run);
+        for (int g = 0; g < NG; ++g) {
+            if (g >= g0) {
+                uint8_t* dst = PK + (((int64_t)bh * NG + g) * R + r) * kSTile;
+                store_split8(run, dst + mnmaj(j, gq, kLboS), dst + mnmaj(j, 10 + gq, kLboS));
+            }
+            if (live) {
+                float x[8];
+                ld8(Sb + (int64_t)g * stride, x);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) run[i] += x[i];
             }
         }
-        store_split8(x, dst + mnmaj(j, gq, kLboS), dst + mnmaj(j, 10 + gq, kLboS));
+        if (live && state_out) {
+            float* so = state_out + (int64_t)bh * stride;
+            if (gq < 8) {
+                reinterpret_cast<float4*>(so + (int64_t)f * kDV + gq * 8)[0] = make_float4(run[0], run[1], run[2], run[3]);
+                reinterpret_cast<float4*>(so + (int64_t)f * kDV + gq * 8)[1] = make_float4(run[4], run[5], run[6], run[7]);
+            } else {
+                so[(int64_t)F * kDV + f] = run[0];
+            }
+        }
     }
+    if (state_out && blockIdx.x == 0)
+        for (int64_t e = (int64_t)F * (kDV + 1) + threadIdx.x; e < stride; e += 256)
+            state_out[(int64_t)bh * stride + e] = 0.f;
 }
 
 // ---------------------------------------------------------------- 4. outputs
@@ -760,12 +796,14 @@ int run(const bf16* q, const bf16* k, const bf16* v, float* out, const float* st
                  tcf_state_kernel<D, N><<<dim3(NG, NFT, BH), kStateThreads, StSm<D>::kBytes, stream>>>(
                      tmk, tmv, Wb, Ntok, n, (int)F, stride, G, NG, err));
         e = cudaGetLastError();
-        if (e == cudaSuccess)
-            e = launch_state_scan(Wb, state_in, state_out, BH, NG, stride, F * (kDV + 1), stream, true);
-        if (e == cudaSuccess && need_pk) {
-            TA_TIMED(stream, "tcf_pack_kernel",
-                     e = launch_maybe_pdl(tcf_pack_kernel, dim3(R, NG - g0, BH), dim3(256), 0, stream, true,
-                                          (const float*)Wb, PKb, (int)F, stride, NG, R, g0));
+        // the scan and the operand tiles in one pass: 8 columns of a feature
+        // row a thread, 10 column groups a row (hi 0..7, z, zero), rows to 64 R
+        if (e == cudaSuccess) {
+            const int units = R * kRT * 10;
+            TA_TIMED(stream, "tcf_scan_pack_kernel",
+                     e = launch_maybe_pdl(tcf_scan_pack_kernel, dim3((units + 255) / 256, BH), dim3(256), 0, stream,
+                                          true, (const float*)Wb, state_in, state_out, PKb, (int)F, stride, NG, R,
+                                          need_pk ? g0 : NG));
         }
     }
     if (e == cudaSuccess) {
